@@ -1,0 +1,48 @@
+"""Test helpers: torch tensors <-> NumPy views and Workload -> oracle Layer.
+
+Only conversions live here (exact bf16 -> float64, uint8 passthrough). No
+arithmetic of the method.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import moe as omoe
+from oracle import rawint4 as orq
+from workloads import LORA_NAMES, Workload
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return orq.bf16_bits_to_f64(bf16_bits(t))
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def u8(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.uint8
+    return t.detach().cpu().contiguous().numpy()
+
+
+def oracle_layer(wl: Workload) -> omoe.Layer:
+    c = wl.cfg
+    return omoe.Layer(
+        gate_q=u8(wl.gate_q), gate_s=f64(wl.gate_s),
+        up_q=u8(wl.up_q), up_s=f64(wl.up_s),
+        down_q=u8(wl.down_q), down_s=f64(wl.down_s),
+        lora={n: f64(wl.lora[n]) for n in LORA_NAMES},
+        alpha=c.alpha, swiglu_limit=c.swiglu_limit,
+    )
+
+
+def oracle_run(wl: Workload, experts=None):
+    layer = oracle_layer(wl)
+    out, ctx = omoe.forward(layer, f64(wl.x), wl.expert_ids.cpu().numpy(), f64(wl.route_weights), experts=experts)
+    gin, groute, grads = omoe.backward(layer, ctx, f64(wl.grad_out))
+    return layer, out, gin, groute, grads
