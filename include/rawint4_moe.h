@@ -1,0 +1,203 @@
+/*
+ * rawint4_moe.h - C ABI of the B200 (sm_100a) routed RAWINT4 MoE-LoRA layer.
+ *
+ * The layer (rawint4_sft_reference.py, routed_rawint4_lora): a routed top-k
+ * mixture of SwiGLU experts. Expert e's gate/up/down base projections are
+ * frozen signed group-32 RAWINT4 and carry trainable rank-r LoRA adapters.
+ * For token t, slot s, e = expert_ids[t,s], w = route_weights[t,s],
+ * c = alpha / rank, L = swiglu_limit:
+ *     G = W_g x + c B_g A_g x,  U = W_u x + c B_u A_u x
+ *     G' = L > 0 ? min(G, L) : G,  U' = L > 0 ? clamp(U, -L, L) : U
+ *     h = silu(G') U',  y = W_d h + c B_d A_d h,  out[t] = sum_s w y
+ *
+ * RAWINT4 storage (rawint4_sft_reference.py module docstring, unpack_rawint4):
+ * two 4-bit codes per byte, LOW nibble first; weight = (code - 8) * scale,
+ * one bf16 scale per 32 consecutive input features, no zero point.
+ *
+ * Conventions for every entry point:
+ *  - bf16 / fp16 values are passed as uint16_t bit patterns.
+ *  - Pointers named in the tensor lists are DEVICE pointers unless the
+ *    comment says "host". All tensors are dense, row-major, contiguous.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only
+ *    enqueue work on it and return; they never synchronise except
+ *    rawint4_moe_lora_status().
+ *  - The caller owns every buffer. The library allocates no device memory
+ *    and keeps no pointer after a call returns; all per-call state lives in
+ *    the caller's workspace.
+ *  - Return value: a RAWINT4_* status code. Argument errors are detected on
+ *    the host before anything is enqueued, and nothing is written then.
+ *
+ * Design note: matrix products run on the 5th-generation tensor cores with
+ * FP16 operands and FP32 accumulation. (code - 8) * scale has at most 12
+ * significant bits, so every decoded weight is exact in FP16 as long as
+ * |scale| lies in [2^-14, 8188]; activations are rounded once to FP16
+ * (relative error 2^-11) where they become MMA operands.
+ */
+#ifndef RAWINT4_MOE_H
+#define RAWINT4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RAWINT4_API __attribute__((visibility("default")))
+#else
+#define RAWINT4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- codes */
+enum {
+  RAWINT4_OK = 0,
+  RAWINT4_INVALID_ARGUMENT = 1, /* null pointer, bad size, workspace too small, ... */
+  RAWINT4_FROZEN_BASE = 2,      /* a base-weight gradient buffer was passed (see bwd) */
+  RAWINT4_NO_SAVED_FORWARD = 3, /* reported through the device status word */
+  RAWINT4_CUDA_ERROR = 4,       /* a CUDA runtime/driver call failed */
+  RAWINT4_BAD_EXPERT_ID = 5,    /* reported through the device status word */
+  RAWINT4_DEVICE_TIMEOUT = 6,   /* a bounded pipeline wait expired (device status) */
+  RAWINT4_FP16_OVERFLOW = 7,    /* an operand overflowed FP16 (device status) */
+  RAWINT4_UNSUPPORTED = 8       /* no sm_100 device, or shape outside the kernels' limits */
+};
+
+/* Bits of the device status word (rawint4_moe_lora_status). */
+enum {
+  RAWINT4_DEV_BAD_EXPERT_ID = 1u << 0,    /* an id outside [0, E): that slot contributed 0 */
+  RAWINT4_DEV_NO_SAVED_FORWARD = 1u << 1, /* bwd found no pending saved forward: it did nothing */
+  RAWINT4_DEV_TIMEOUT = 1u << 2,          /* a kernel gave up on a bounded wait: results invalid */
+  RAWINT4_DEV_FP16_OVERFLOW = 1u << 3     /* an activation exceeded the FP16 range: results invalid */
+};
+
+/* ------------------------------------------------------------- structs */
+
+/* Layer configuration. Mirrors the fields of the contract test's
+ * MOESFTConfig that the method uses (test_rawint4_sft_numerical.py,
+ * _make_backend): expert count, top_k, hidden size H, intermediate size I,
+ * LoRA rank r and alpha (scaling c = alpha / r), swiglu_limit L (0 disables
+ * the clamp; must be finite and >= 0) and max_tokens (the largest qlen a
+ * workspace is sized for; the reference's max_len).
+ * Limits: H % 128 == 0, I % 128 == 0, 1 <= rank <= 32, 1 <= top_k <= experts. */
+typedef struct rawint4_moe_cfg {
+  int32_t experts;
+  int32_t top_k;
+  int32_t hidden;
+  int32_t inter;
+  int32_t rank;
+  float alpha;
+  float swiglu_limit;
+  int32_t max_tokens;
+} rawint4_moe_cfg;
+
+/* Frozen base weights (device, read-only; never written).
+ * gate_q, up_q: uint8 [E, I, H/2]; gate_s, up_s: bf16 [E, I, H/32]
+ * down_q:       uint8 [E, H, I/2]; down_s:       bf16 [E, H, I/32]
+ * Layout of one projection: rawint4_sft_reference.py, _validate_rawint4_layout
+ * (packed uint8 [N_out, K_in/2], scales bf16 [N_out, K_in/32]). */
+typedef struct rawint4_moe_base {
+  const uint8_t *gate_q, *up_q, *down_q;
+  const uint16_t *gate_s, *up_s, *down_s;
+} rawint4_moe_base;
+
+/* LoRA adapters (device, bf16), the six tensors of the contract test
+ * (GRAD_SHAPES): gate_a [E, r, H], gate_b [E, I, r], up_a [E, r, H],
+ * up_b [E, I, r], down_a [E, r, I], down_b [E, H, r]. */
+typedef struct rawint4_moe_lora {
+  const uint16_t *gate_a, *gate_b, *up_a, *up_b, *down_a, *down_b;
+} rawint4_moe_lora;
+
+/* LoRA gradient buffers (device, bf16), same shapes as rawint4_moe_lora. */
+typedef struct rawint4_moe_lora_grads {
+  uint16_t *gate_a, *gate_b, *up_a, *up_b, *down_a, *down_b;
+} rawint4_moe_lora_grads;
+
+/* --------------------------------------------------------- entry points */
+
+/* Bytes of device workspace a layer with this configuration needs
+ * (*bytes, host). The workspace holds the routing permutation, the saved
+ * forward context and backward scratch; its size grows linearly with
+ * max_tokens * top_k. Returns RAWINT4_INVALID_ARGUMENT for a bad cfg. */
+RAWINT4_API int rawint4_moe_lora_workspace_size(const rawint4_moe_cfg* cfg, size_t* bytes);
+
+/* Forward (the contract test's forward_sft(qlen, top_k, ids, weights, in,
+ * out, save_for_backward)).
+ *   qlen          number of tokens Q, 0 <= qlen <= cfg->max_tokens (0: no-op
+ *                 that still records an empty saved context when saving)
+ *   expert_ids    int64 [Q, k]; ids outside [0, E) contribute nothing and
+ *                 raise RAWINT4_DEV_BAD_EXPERT_ID in the device status
+ *   route_weights fp32 [Q, k], used as given (no renormalisation)
+ *   x             bf16 [Q, H];  out  bf16 [Q, H] (overwritten)
+ *   save_for_backward  nonzero: keep the context for one rawint4_moe_lora_bwd
+ *                 on this workspace, replacing any pending one (checkpoint
+ *                 recompute). zero: the workspace's pending context, if any,
+ *                 is invalidated (the scratch is shared).
+ *   workspace     device buffer of at least rawint4_moe_lora_workspace_size
+ *                 bytes, 256-byte aligned; ws_bytes is its size.
+ * The base, LoRA and input buffers must stay valid until the enqueued work
+ * completes. */
+RAWINT4_API int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base,
+                         const rawint4_moe_lora* lora, int32_t qlen, const int64_t* expert_ids,
+                         const float* route_weights, const uint16_t* x, uint16_t* out,
+                         int save_for_backward, void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the most recent saving forward on this workspace (the
+ * contract test's backward(dY, dX, 6 LoRA grads, dRoute, 3 base grads,
+ * accumulate, grad_scale)). It consumes the saved context: exactly one
+ * backward per saving forward. cfg, base and lora must be the ones the
+ * forward used.
+ *   grad_out    bf16 [Q, H] (Q of the saved forward)
+ *   grad_in     bf16 [Q, H] (overwritten) = d(sum grad_out*out)/dx
+ *   grad_route  fp32 [Q, k] (overwritten; may be NULL) = <grad_out[t], y_{t,s}>
+ *   grads       six bf16 buffers: buf = (accumulate ? buf : 0)
+ *               + grad_scale * dLoRA, rounded once to bf16. Rows of experts
+ *               that no slot of this call reached are zeroed when
+ *               accumulate == 0 and left as they are otherwise
+ *               (authoritative gradient window of the contract test).
+ *               grad_scale multiplies only these six.
+ *   base_grad_gate/up/down  must be NULL: the base is frozen and no base
+ *               gradient is ever formed. Any non-NULL pointer returns
+ *               RAWINT4_FROZEN_BASE before anything is enqueued.
+ * Without a pending saved forward the call enqueues nothing that writes the
+ * outputs and sets RAWINT4_DEV_NO_SAVED_FORWARD in the device status. */
+RAWINT4_API int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base,
+                         const rawint4_moe_lora* lora, const uint16_t* grad_out, uint16_t* grad_in,
+                         float* grad_route, const rawint4_moe_lora_grads* grads,
+                         const void* base_grad_gate, const void* base_grad_up,
+                         const void* base_grad_down, int accumulate, float grad_scale,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word kept
+ * in `workspace` (*device_status, host: OR of RAWINT4_DEV_* bits raised by
+ * calls since the last read). */
+RAWINT4_API int rawint4_moe_lora_status(void* workspace, void* stream, uint32_t* device_status);
+
+/* Human-readable text of a RAWINT4_* code (static storage). */
+RAWINT4_API const char* rawint4_moe_lora_strerror(int code);
+
+/* Bit-exact check export: decode one packed projection with the same device
+ * routine the GEMM producers use.
+ *   q [N, K/2] uint8, s [N, K/32] bf16 (device); K % 32 == 0.
+ *   out_f32 [N, K] fp32 (device, may be NULL): (code - 8) * scale in fp32.
+ *   out_f16 [N, K] fp16 bits (device, may be NULL): the MMA operand, i.e.
+ *   the fp16 rounding of the same product (exact for scales in range). */
+RAWINT4_API int rawint4_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, float* out_f32,
+                   uint16_t* out_f16, void* stream);
+
+/* Bit-exact check export: the token->expert permutation of the forward.
+ * ids int64 [Q, k] (device). Outputs (device, int32):
+ *   offsets [E+1]  offsets[e] = first permuted row of expert e (exclusive
+ *                  prefix sum of the per-expert counts)
+ *   perm    [Q*k]  permuted row p -> flat slot f = t*k + s; stable (rows of
+ *                  one expert ascend in f); entries past offsets[E] are -1
+ *   inv     [Q*k]  flat slot -> permuted row, -1 for ids outside [0, E)
+ * workspace: device scratch of rawint4_moe_permute_workspace_size bytes. */
+RAWINT4_API int rawint4_moe_permute_workspace_size(int32_t qlen, int32_t top_k, int32_t experts, size_t* bytes);
+RAWINT4_API int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t experts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace,
+                        size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RAWINT4_MOE_H */

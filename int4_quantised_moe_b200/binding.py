@@ -1,0 +1,241 @@
+"""ctypes binding of librawint4_moe.so (include/rawint4_moe.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers,
+every computation happens in the library's CUDA kernels. There is no CPU
+fallback: importing this module fails loudly when the library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librawint4_moe.so")
+
+OK = 0
+INVALID_ARGUMENT = 1
+FROZEN_BASE = 2
+NO_SAVED_FORWARD = 3
+CUDA_ERROR = 4
+BAD_EXPERT_ID = 5
+DEVICE_TIMEOUT = 6
+FP16_OVERFLOW = 7
+UNSUPPORTED = 8
+
+DEV_BAD_EXPERT_ID = 1 << 0
+DEV_NO_SAVED_FORWARD = 1 << 1
+DEV_TIMEOUT = 1 << 2
+DEV_FP16_OVERFLOW = 1 << 3
+
+EXPORTED_SYMBOLS = (
+    "rawint4_moe_lora_workspace_size",
+    "rawint4_moe_lora_fwd",
+    "rawint4_moe_lora_bwd",
+    "rawint4_moe_lora_status",
+    "rawint4_moe_lora_strerror",
+    "rawint4_decode",
+    "rawint4_moe_permute_workspace_size",
+    "rawint4_moe_permute",
+)
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("rank", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("swiglu_limit", ctypes.c_float), ("max_tokens", ctypes.c_int32)]
+
+
+class Base(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s")]
+
+
+class Lora(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("gate_a", "gate_b", "up_a", "up_b", "down_a", "down_b")]
+
+
+class LoraGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("gate_a", "gate_b", "up_a", "up_b", "down_a", "down_b")]
+
+
+class RawInt4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} (code {code})")
+
+
+class FrozenBaseError(RawInt4Error, ValueError):
+    pass
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m int4_quantised_moe_b200.build` "
+            "(the layer has no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32, i64, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    P = ctypes.POINTER
+    lib.rawint4_moe_lora_workspace_size.argtypes = [P(Cfg), P(sz)]
+    lib.rawint4_moe_lora_fwd.argtypes = [P(Cfg), P(Base), P(Lora), i32, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]
+    lib.rawint4_moe_lora_bwd.argtypes = [P(Cfg), P(Base), P(Lora), vp, vp, vp, P(LoraGrads), vp, vp, vp,
+                                         ctypes.c_int, f32, vp, sz, vp]
+    lib.rawint4_moe_lora_status.argtypes = [vp, vp, P(ctypes.c_uint32)]
+    lib.rawint4_moe_lora_strerror.argtypes = [ctypes.c_int]
+    lib.rawint4_moe_lora_strerror.restype = ctypes.c_char_p
+    lib.rawint4_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+    lib.rawint4_moe_permute_workspace_size.argtypes = [i32, i32, i32, P(sz)]
+    lib.rawint4_moe_permute.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    for name in EXPORTED_SYMBOLS:
+        if name != "rawint4_moe_lora_strerror":
+            getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return _lib.rawint4_moe_lora_strerror(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code == FROZEN_BASE:
+        raise FrozenBaseError(code, what)
+    if code != OK:
+        raise RawInt4Error(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the layer must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens) -> Cfg:
+    return Cfg(int(experts), int(top_k), int(hidden), int(inter), int(rank), float(alpha), float(swiglu_limit),
+               int(max_tokens))
+
+
+def rawint4_moe_lora_workspace_size(cfg: Cfg) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.rawint4_moe_lora_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "rawint4_moe_lora_workspace_size")
+    return int(n.value)
+
+
+def make_base(gate_q, gate_s, up_q, up_s, down_q, down_s) -> Base:
+    return Base(_ptr(gate_q), _ptr(up_q), _ptr(down_q), _ptr(gate_s), _ptr(up_s), _ptr(down_s))
+
+
+def make_lora(lora: Dict[str, torch.Tensor]) -> Lora:
+    return Lora(*[_ptr(lora[n]) for n in ("gate_lora_a", "gate_lora_b", "up_lora_a", "up_lora_b",
+                                          "down_lora_a", "down_lora_b")])
+
+
+def make_grads(grads: Dict[str, torch.Tensor]) -> LoraGrads:
+    return LoraGrads(*[_ptr(grads[n]) for n in ("gate_lora_a", "gate_lora_b", "up_lora_a", "up_lora_b",
+                                                "down_lora_a", "down_lora_b")])
+
+
+def rawint4_moe_lora_fwd(cfg: Cfg, base: Base, lora: Lora, qlen: int, expert_ids, route_weights, x, out,
+                         save_for_backward: bool, workspace: torch.Tensor, stream=None) -> None:
+    rc = _lib.rawint4_moe_lora_fwd(ctypes.byref(cfg), ctypes.byref(base), ctypes.byref(lora), int(qlen),
+                                   _ptr(expert_ids), _ptr(route_weights), _ptr(x), _ptr(out),
+                                   1 if save_for_backward else 0, _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+    _check(rc, "rawint4_moe_lora_fwd")
+
+
+def rawint4_moe_lora_bwd(cfg: Cfg, base: Base, lora: Lora, grad_out, grad_in, grad_route, grads: LoraGrads,
+                         accumulate: bool, grad_scale: float, workspace: torch.Tensor, stream=None,
+                         base_grad_gate=None, base_grad_up=None, base_grad_down=None) -> None:
+    rc = _lib.rawint4_moe_lora_bwd(ctypes.byref(cfg), ctypes.byref(base), ctypes.byref(lora), _ptr(grad_out),
+                                   _ptr(grad_in), _ptr(grad_route), ctypes.byref(grads), _ptr(base_grad_gate),
+                                   _ptr(base_grad_up), _ptr(base_grad_down), 1 if accumulate else 0,
+                                   float(grad_scale), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rawint4_moe_lora_bwd")
+
+
+def rawint4_moe_lora_status(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    _check(_lib.rawint4_moe_lora_status(_ptr(workspace), _stream(stream), ctypes.byref(v)), "rawint4_moe_lora_status")
+    return int(v.value)
+
+
+def rawint4_decode(q: torch.Tensor, s: torch.Tensor, out_f32=None, out_f16=None, stream=None) -> None:
+    n, k2 = q.shape[-2], q.shape[-1]
+    rows = q.numel() // k2
+    _check(_lib.rawint4_decode(_ptr(q), _ptr(s), rows, 2 * k2, _ptr(out_f32), _ptr(out_f16), _stream(stream)),
+           "rawint4_decode")
+
+
+def rawint4_moe_permute(expert_ids: torch.Tensor, experts: int, offsets, perm, inv, stream=None) -> None:
+    q, k = expert_ids.shape
+    n = ctypes.c_size_t(0)
+    _check(_lib.rawint4_moe_permute_workspace_size(q, k, experts, ctypes.byref(n)), "permute_workspace_size")
+    ws = torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=expert_ids.device)
+    _check(_lib.rawint4_moe_permute(_ptr(expert_ids), q, k, experts, _ptr(offsets), _ptr(perm), _ptr(inv),
+                                    _ptr(ws), ws.numel(), _stream(stream)), "rawint4_moe_permute")
+
+
+# ---------------------------------------------------------------------------
+# Convenience holder used by tests and the bench: keeps the layer's tensors
+# and one workspace together and calls the two entry points.
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Layer:
+    cfg: Cfg
+    base: Base
+    lora: Lora
+    workspace: torch.Tensor
+    keep: tuple  # tensors whose pointers live in base/lora
+
+    @classmethod
+    def create(cls, experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens, gate_q, gate_s, up_q, up_s,
+               down_q, down_s, lora: Dict[str, torch.Tensor], device=None):
+        cfg = make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens)
+        nbytes = rawint4_moe_lora_workspace_size(cfg)
+        dev = device if device is not None else gate_q.device
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        ws[:256].zero_()
+        base = make_base(gate_q, gate_s, up_q, up_s, down_q, down_s)
+        lo = make_lora(lora)
+        return cls(cfg, base, lo, ws, (gate_q, gate_s, up_q, up_s, down_q, down_s, dict(lora)))
+
+    def forward(self, expert_ids, route_weights, x, out=None, save_for_backward=True, stream=None):
+        q = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        rawint4_moe_lora_fwd(self.cfg, self.base, self.lora, q, expert_ids, route_weights, x, out,
+                             save_for_backward, self.workspace, stream)
+        return out
+
+    def backward(self, grad_out, grads: Dict[str, torch.Tensor], accumulate=False, grad_scale=1.0, grad_in=None,
+                 grad_route=None, stream=None, **base_grads):
+        if grad_in is None:
+            grad_in = torch.empty_like(grad_out)
+        rawint4_moe_lora_bwd(self.cfg, self.base, self.lora, grad_out, grad_in, grad_route, make_grads(grads),
+                             accumulate, grad_scale, self.workspace, stream, **base_grads)
+        return grad_in
+
+    def status(self, stream=None) -> int:
+        return rawint4_moe_lora_status(self.workspace, stream)

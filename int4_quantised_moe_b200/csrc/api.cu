@@ -1,0 +1,519 @@
+// C ABI of the routed RAWINT4 MoE-LoRA layer: argument checks, workspace
+// carve-up, TMA descriptors and the launch sequences of forward and backward.
+// Entry points mirror forward_sft / backward of the contract test
+// (test_rawint4_sft_numerical.py, _forward and _backward).
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "aux.cuh"
+#include "gemm.cuh"
+#include "route.cuh"
+
+namespace r4 {
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Device buffers of one layer call, carved out of the caller's workspace.
+struct Layout {
+  size_t hdr, offsets, perm, inv, w_perm, tiles, hist;
+  size_t xp, xa, g, u, h, ha, hw, y, gp, gd, gdw, dgu, gb, dpart;
+  size_t total;
+  int64_t rows;  // padded permuted-row capacity
+  int max_tiles;
+};
+
+Layout make_layout(const rawint4_moe_cfg& c) {
+  Layout L{};
+  const int64_t R = (int64_t)c.max_tokens * c.top_k;
+  // capacity rounded to whole 256-row tiles plus one spare tile: TMA boxes of
+  // the last token tile and zero-padded LoRA side rows stay inside the buffers
+  L.rows = (R + kTileRows - 1) / kTileRows * kTileRows + kTileRows;
+  L.max_tiles = max_tok_tiles((int32_t)R, c.experts);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  const int64_t H = c.hidden, I = c.inter, E = c.experts, rows = L.rows;
+  L.hdr = take(sizeof(WsHeader));
+  L.offsets = take((E + 1) * 4);
+  L.perm = take(rows * 4);
+  L.inv = take(rows * 4);
+  L.w_perm = take(rows * 4);
+  L.tiles = take((size_t)L.max_tiles * 16);
+  L.hist = take(route_scratch_bytes((int32_t)R, c.experts));
+  L.xp = take(rows * H * 2);
+  L.xa = take(rows * kLoraPad * 2);
+  L.g = take(rows * I * 4);
+  L.u = take(rows * I * 4);
+  L.h = take(rows * I * 2);
+  L.ha = take(rows * kLoraPad * 2);
+  L.hw = take(rows * kLoraPad * 2);
+  L.y = take(rows * H * 4);
+  L.gp = take(rows * H * 2);
+  L.gd = take(rows * kLoraPad * 2);
+  L.gdw = take(rows * kLoraPad * 2);
+  L.dgu = take(rows * 2 * I * 2);
+  L.gb = take(rows * kLoraPad * 2);
+  L.dpart = take(rows * (I / 128) * 4);
+  L.total = off;
+  return L;
+}
+
+bool cfg_ok(const rawint4_moe_cfg* c) {
+  if (!c) return false;
+  if (c->experts < 1 || c->experts > 4096) return false;
+  if (c->top_k < 1 || c->top_k > c->experts) return false;
+  if (c->hidden < 128 || c->hidden % 128 != 0) return false;
+  if (c->inter < 128 || c->inter % 128 != 0) return false;
+  if (c->rank < 1 || c->rank > 32) return false;
+  if (!std::isfinite(c->alpha)) return false;
+  if (!std::isfinite(c->swiglu_limit) || c->swiglu_limit < 0.f) return false;
+  if (c->max_tokens < 1) return false;
+  if ((int64_t)c->max_tokens * c->top_k > (1 << 24)) return false;
+  return true;
+}
+
+bool base_ok(const rawint4_moe_base* b) {
+  return b && b->gate_q && b->up_q && b->down_q && b->gate_s && b->up_s && b->down_s;
+}
+bool lora_ok(const rawint4_moe_lora* l) {
+  return l && l->gate_a && l->gate_b && l->up_a && l->up_b && l->down_a && l->down_b;
+}
+bool grads_ok(const rawint4_moe_lora_grads* g) {
+  return g && g->gate_a && g->gate_b && g->up_a && g->up_b && g->down_a && g->down_b;
+}
+
+// --------------------------------------------------------------- device
+std::mutex g_mu;
+int g_checked_device = -1;
+int g_sm_count = 0;
+
+int check_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_checked_device != dev) {
+    int major = 0, minor = 0, count = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return RAWINT4_CUDA_ERROR;
+    if (major != 10 || minor != 0) return RAWINT4_UNSUPPORTED;
+    g_checked_device = dev;
+    g_sm_count = count;
+  }
+  *sms = g_sm_count;
+  return RAWINT4_OK;
+}
+
+// ------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1}, no swizzle
+bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kbytes, (cuuint64_t)rows, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)kbytes, (cuuint64_t)(kbytes * rows)};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 row-major [rows, cols]; box {64, 16}, 128-byte swizzle (UMMA K-major B layout)
+bool map_act(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int common_checks(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base, const rawint4_moe_lora* lora,
+                  void* workspace, size_t ws_bytes, Layout* L) {
+  if (!cfg_ok(cfg) || !base_ok(base) || !lora_ok(lora) || !workspace) return RAWINT4_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return RAWINT4_INVALID_ARGUMENT;
+  *L = make_layout(*cfg);
+  if (ws_bytes < L->total) return RAWINT4_INVALID_ARGUMENT;
+  return RAWINT4_OK;
+}
+
+int grid_for_tiles(int sms, int max_tiles, int rowblk) {
+  const int64_t t = (int64_t)max_tiles * rowblk;
+  return (int)(t < sms ? (t > 0 ? t : 1) : sms);
+}
+
+#define R4_TRY(x)                                \
+  do {                                           \
+    if ((x) != cudaSuccess) return RAWINT4_CUDA_ERROR; \
+  } while (0)
+
+}  // namespace
+}  // namespace r4
+
+using namespace r4;
+
+extern "C" {
+
+int rawint4_moe_lora_workspace_size(const rawint4_moe_cfg* cfg, size_t* bytes) {
+  if (!cfg_ok(cfg) || !bytes) return RAWINT4_INVALID_ARGUMENT;
+  *bytes = make_layout(*cfg).total;
+  return RAWINT4_OK;
+}
+
+const char* rawint4_moe_lora_strerror(int code) {
+  switch (code) {
+    case RAWINT4_OK: return "ok";
+    case RAWINT4_INVALID_ARGUMENT: return "invalid argument (null pointer, unsupported size or workspace too small)";
+    case RAWINT4_FROZEN_BASE: return "frozen base: base-weight gradients are never formed; pass NULL base gradient buffers";
+    case RAWINT4_NO_SAVED_FORWARD: return "backward without a pending saved forward on this workspace";
+    case RAWINT4_CUDA_ERROR: return "a CUDA runtime or driver call failed";
+    case RAWINT4_BAD_EXPERT_ID: return "an expert id outside [0, experts) was routed; that slot contributed nothing";
+    case RAWINT4_DEVICE_TIMEOUT: return "a device pipeline wait exceeded its bound; results are invalid";
+    case RAWINT4_FP16_OVERFLOW: return "an activation exceeded the fp16 operand range; results are invalid";
+    case RAWINT4_UNSUPPORTED: return "unsupported device (needs sm_100) or configuration";
+    default: return "unknown status code";
+  }
+}
+
+int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base, const rawint4_moe_lora* lora,
+                         int32_t qlen, const int64_t* expert_ids, const float* route_weights, const uint16_t* x,
+                         uint16_t* out, int save_for_backward, void* workspace, size_t ws_bytes, void* stream_) {
+  Layout L;
+  int rc = common_checks(cfg, base, lora, workspace, ws_bytes, &L);
+  if (rc != RAWINT4_OK) return rc;
+  if (qlen < 0 || qlen > cfg->max_tokens) return RAWINT4_INVALID_ARGUMENT;
+  if (qlen > 0 && (!expert_ids || !route_weights || !x || !out)) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_);
+  const rawint4_moe_cfg& c = *cfg;
+  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank;
+  const float scaling = c.alpha / (float)r;
+  void* ws = workspace;
+  WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+
+  R4_TRY(launch_header_begin_fwd(hdr, save_for_backward, st));
+  R4_TRY(launch_route(expert_ids, route_weights, qlen, k, E, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
+                      at<int32_t>(ws, L.inv), at<float>(ws, L.w_perm), at<int4>(ws, L.tiles), at<int32_t>(ws, L.hist),
+                      hdr, st));
+  if (qlen == 0) return RAWINT4_OK;
+  const int maxR = qlen * k;
+  R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, st));
+
+  // xa = c * X_perm [A_g; A_u]^T (rank-r side matrix of gate and up)
+  LoraRowsArgs la{};
+  la.L = at<uint16_t>(ws, L.xp);
+  la.ldL = H;
+  la.colL[0] = la.colL[1] = 0;
+  la.K = H;
+  la.R[0] = lora->gate_a;
+  la.R[1] = lora->up_a;
+  la.r_expert = (int64_t)r * H;
+  la.r_style = 0;
+  la.rank = r;
+  la.halves = 2;
+  la.scale = scaling;
+  la.out0 = at<uint16_t>(ws, L.xa);
+  la.out1 = nullptr;
+  la.w_perm = nullptr;
+  const int max_tiles = max_tok_tiles(maxR, E);
+  R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+
+  GemmMaps mp;
+  GemmParams gp{};
+  gp.tok_tiles = at<int4>(ws, L.tiles);
+  gp.hdr = hdr;
+  gp.status = &hdr->status;
+  gp.need_saved = 0;
+  gp.rank = r;
+  gp.w_perm = at<float>(ws, L.w_perm);
+  gp.inter = I;
+  gp.limit = c.swiglu_limit;
+
+  // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 64) ||
+      !map_act(&mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act(&mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
+    return RAWINT4_CUDA_ERROR;
+  gp.n_rowblk = I / 64;
+  gp.n_main = H / kBlockK;
+  gp.s0 = base->gate_s;
+  gp.s1 = base->up_s;
+  gp.s_expert = (int64_t)I * (H / 32);
+  gp.s_row = H / 32;
+  gp.stored_rows = I;
+  gp.lx0 = lora->gate_b;
+  gp.lx1 = lora->up_b;
+  gp.lx_expert = (int64_t)I * r;
+  gp.lx_ld = r;
+  gp.out_a = at<float>(ws, L.g);
+  gp.out_b = at<float>(ws, L.u);
+  gp.out_h = at<uint16_t>(ws, L.h);
+  gp.ld_out = I;
+  R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+
+  // ha = c * h A_d^T, hw = w * ha
+  LoraRowsArgs lb{};
+  lb.L = at<uint16_t>(ws, L.h);
+  lb.ldL = I;
+  lb.K = I;
+  lb.R[0] = lb.R[1] = lora->down_a;
+  lb.r_expert = (int64_t)r * I;
+  lb.r_style = 0;
+  lb.rank = r;
+  lb.halves = 1;
+  lb.scale = scaling;
+  lb.out0 = at<uint16_t>(ws, L.ha);
+  lb.out1 = at<uint16_t>(ws, L.hw);
+  lb.w_perm = at<float>(ws, L.w_perm);
+  R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+
+  // down: Yw = w * (h W_d^T + ha B_d^T)
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
+      !map_act(&mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act(&mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
+    return RAWINT4_CUDA_ERROR;
+  gp.n_rowblk = H / 128;
+  gp.n_main = I / kBlockK;
+  gp.s0 = gp.s1 = base->down_s;
+  gp.s_expert = (int64_t)H * (I / 32);
+  gp.s_row = I / 32;
+  gp.stored_rows = H;
+  gp.lx0 = gp.lx1 = lora->down_b;
+  gp.lx_expert = (int64_t)H * r;
+  gp.lx_ld = r;
+  gp.out_a = at<float>(ws, L.y);
+  gp.out_b = nullptr;
+  gp.out_h = nullptr;
+  gp.ld_out = H;
+  R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+
+  // out[t] = sum over slots, fixed order
+  R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, st));
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base, const rawint4_moe_lora* lora,
+                         const uint16_t* grad_out, uint16_t* grad_in, float* grad_route,
+                         const rawint4_moe_lora_grads* grads, const void* base_grad_gate, const void* base_grad_up,
+                         const void* base_grad_down, int accumulate, float grad_scale, void* workspace, size_t ws_bytes,
+                         void* stream_) {
+  // The base is frozen: refuse any base-gradient buffer before touching anything.
+  if (base_grad_gate || base_grad_up || base_grad_down) return RAWINT4_FROZEN_BASE;
+  Layout L;
+  int rc = common_checks(cfg, base, lora, workspace, ws_bytes, &L);
+  if (rc != RAWINT4_OK) return rc;
+  if (!grad_out || !grad_in || !grads_ok(grads) || !std::isfinite(grad_scale)) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_);
+  const rawint4_moe_cfg& c = *cfg;
+  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank;
+  const float scaling = c.alpha / (float)r;
+  void* ws = workspace;
+  WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  const int maxQ = c.max_tokens;
+  const int maxR = maxQ * k;
+  const int max_tiles = max_tok_tiles(maxR, E);
+
+  R4_TRY(launch_header_check_bwd(hdr, st));
+  R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR, &hdr->status, 1,
+                            st));
+
+  // gd = c * g B_d, gdw = w * gd (rank-r side of the down LoRA backward)
+  LoraRowsArgs la{};
+  la.L = at<uint16_t>(ws, L.gp);
+  la.ldL = H;
+  la.K = H;
+  la.R[0] = la.R[1] = lora->down_b;
+  la.r_expert = (int64_t)H * r;
+  la.r_style = 1;
+  la.rank = r;
+  la.halves = 1;
+  la.scale = scaling;
+  la.out0 = at<uint16_t>(ws, L.gd);
+  la.out1 = at<uint16_t>(ws, L.gdw);
+  la.w_perm = at<float>(ws, L.w_perm);
+  R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+
+  GemmMaps mp;
+  GemmParams gp{};
+  gp.tok_tiles = at<int4>(ws, L.tiles);
+  gp.hdr = hdr;
+  gp.status = &hdr->status;
+  gp.need_saved = 1;
+  gp.rank = r;
+  gp.w_perm = at<float>(ws, L.w_perm);
+  gp.inter = I;
+  gp.limit = c.swiglu_limit;
+
+  // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
+      !map_act(&mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act(&mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
+    return RAWINT4_CUDA_ERROR;
+  gp.n_rowblk = I / 128;
+  gp.n_main = H / kBlockK;
+  gp.s0 = gp.s1 = base->down_s;
+  gp.s_expert = (int64_t)H * (I / 32);
+  gp.s_row = I / 32;
+  gp.stored_rows = H;
+  gp.lx0 = gp.lx1 = lora->down_a;
+  gp.lx_expert = (int64_t)r * I;
+  gp.lx_ld = I;
+  gp.out_a = nullptr;
+  gp.out_b = nullptr;
+  gp.out_h = at<uint16_t>(ws, L.dgu);
+  gp.in_g = at<float>(ws, L.g);
+  gp.in_u = at<float>(ws, L.u);
+  gp.droute_part = at<float>(ws, L.dpart);
+  gp.ld_out = I;
+  R4_TRY(launch_gemm(kModeDownT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+
+  // gb = c * [dG B_g, dU B_u]
+  LoraRowsArgs lb{};
+  lb.L = at<uint16_t>(ws, L.dgu);
+  lb.ldL = 2 * I;
+  lb.colL[0] = 0;
+  lb.colL[1] = I;
+  lb.K = I;
+  lb.R[0] = lora->gate_b;
+  lb.R[1] = lora->up_b;
+  lb.r_expert = (int64_t)I * r;
+  lb.r_style = 1;
+  lb.rank = r;
+  lb.halves = 2;
+  lb.scale = scaling;
+  lb.out0 = at<uint16_t>(ws, L.gb);
+  lb.out1 = nullptr;
+  lb.w_perm = nullptr;
+  R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+
+  // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
+      !map_act(&mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act(&mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
+    return RAWINT4_CUDA_ERROR;
+  gp.n_rowblk = H / 128;
+  gp.n_main = 2 * I / kBlockK;
+  gp.s0 = base->gate_s;
+  gp.s1 = base->up_s;
+  gp.s_expert = (int64_t)I * (H / 32);
+  gp.s_row = H / 32;
+  gp.stored_rows = I;
+  gp.lx0 = lora->gate_a;
+  gp.lx1 = lora->up_a;
+  gp.lx_expert = (int64_t)r * H;
+  gp.lx_ld = H;
+  gp.out_a = at<float>(ws, L.y);
+  gp.out_h = nullptr;
+  gp.in_g = gp.in_u = nullptr;
+  gp.droute_part = nullptr;
+  gp.ld_out = H;
+  R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+
+  R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, st));
+  if (grad_route)
+    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), I / 128, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ, st));
+
+  // the six LoRA gradients with the authoritative window
+  GradJobs jobs{};
+  jobs.j[0] = GradJob{at<uint16_t>(ws, L.gp), H, 0, H, at<uint16_t>(ws, L.hw), 0, grads->down_b, 0};
+  jobs.j[1] = GradJob{at<uint16_t>(ws, L.h), I, 0, I, at<uint16_t>(ws, L.gdw), 0, grads->down_a, 1};
+  jobs.j[2] = GradJob{at<uint16_t>(ws, L.dgu), 2 * I, 0, I, at<uint16_t>(ws, L.xa), 0, grads->gate_b, 0};
+  jobs.j[3] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), 0, grads->gate_a, 1};
+  jobs.j[4] = GradJob{at<uint16_t>(ws, L.dgu), 2 * I, I, I, at<uint16_t>(ws, L.xa), r, grads->up_b, 0};
+  jobs.j[5] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), r, grads->up_a, 1};
+  R4_TRY(launch_lora_grads(jobs, 6, H > I ? H : I, at<int32_t>(ws, L.offsets), E, r, accumulate, grad_scale, hdr, st));
+
+  R4_TRY(launch_header_end_bwd(hdr, st));
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_lora_status(void* workspace, void* stream_, uint32_t* device_status) {
+  if (!workspace || !device_status) return RAWINT4_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_);
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  uint32_t v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  if (cudaMemcpy(&v, &hdr->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  if (cudaMemset(&hdr->status, 0, sizeof(v)) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  *device_status = v;
+  return RAWINT4_OK;
+}
+
+int rawint4_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, float* out_f32, uint16_t* out_f16,
+                   void* stream_) {
+  if (!q || !s || n < 0 || k < 0 || k % 32 != 0 || (!out_f32 && !out_f16)) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  if (launch_decode(q, s, n, k, out_f32, out_f16, static_cast<cudaStream_t>(stream_)) != cudaSuccess)
+    return RAWINT4_CUDA_ERROR;
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_permute_workspace_size(int32_t qlen, int32_t top_k, int32_t experts, size_t* bytes) {
+  if (!bytes || qlen < 0 || top_k < 1 || experts < 1 || experts > 4096 || (int64_t)qlen * top_k > (1 << 24))
+    return RAWINT4_INVALID_ARGUMENT;
+  const int32_t slots = qlen * top_k;
+  *bytes = align_up(sizeof(WsHeader), kAlign) + align_up((size_t)max_tok_tiles(slots, experts) * 16, kAlign) +
+           route_scratch_bytes(slots, experts);
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t experts, int32_t* offsets,
+                        int32_t* perm, int32_t* inv, void* workspace, size_t ws_bytes, void* stream_) {
+  size_t need = 0;
+  if (rawint4_moe_permute_workspace_size(qlen, top_k, experts, &need) != RAWINT4_OK) return RAWINT4_INVALID_ARGUMENT;
+  if (!offsets || !workspace || ws_bytes < need || reinterpret_cast<uintptr_t>(workspace) % kAlign) return RAWINT4_INVALID_ARGUMENT;
+  if (qlen > 0 && (!ids || !perm || !inv)) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_);
+  const int32_t slots = qlen * top_k;
+  WsHeader* hdr = static_cast<WsHeader*>(workspace);
+  int4* tiles = at<int4>(workspace, align_up(sizeof(WsHeader), kAlign));
+  int32_t* hist = at<int32_t>(workspace, align_up(sizeof(WsHeader), kAlign) +
+                                             align_up((size_t)max_tok_tiles(slots, experts) * 16, kAlign));
+  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  R4_TRY(launch_route(ids, nullptr, qlen, top_k, experts, offsets, perm, inv, nullptr, tiles, hist, hdr, st));
+  if (slots > 0) {
+    tail_fill_kernel<<<(slots + 255) / 256, 256, 0, st>>>(perm, offsets, experts, slots);
+    R4_TRY(cudaGetLastError());
+  }
+  return RAWINT4_OK;
+}
+
+}  // extern "C"

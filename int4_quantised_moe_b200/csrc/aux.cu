@@ -1,0 +1,332 @@
+// Memory-bound helpers of the layer: row gather into expert order (with the
+// bf16 -> fp16 operand conversion), the fixed-order top-k combines, the
+// rank-r LoRA side matrices, the per-expert LoRA gradient reductions with the
+// contract test's authoritative window, header bookkeeping and the decode
+// check export.
+#include "aux.cuh"
+
+namespace r4 {
+
+namespace {
+
+__device__ __forceinline__ bool bwd_enabled(const WsHeader* hdr) { return hdr->saved == 1u; }
+
+// ------------------------------------------------------------------ gather
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm, int top_k,
+                                   const WsHeader* hdr, uint4* __restrict__ dst, int vecs_per_row, uint32_t* status,
+                                   int need_saved) {
+  if (need_saved && !bwd_enabled(hdr)) return;
+  const int64_t rows = hdr->routed;
+  const int64_t total = rows * vecs_per_row;
+  bool overflow = false;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = idx / vecs_per_row;
+    const int c = (int)(idx - row * vecs_per_row);
+    const int32_t t = perm[row] / top_k;
+    const uint4 v = __ldg(src + (int64_t)t * vecs_per_row + c);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(in[j] << 16);
+      const float hi = __uint_as_float(in[j] & 0xFFFF0000u);
+      __half2 h = __floats2half2_rn(lo, hi);
+      overflow |= (__hisinf(__low2half(h)) | __hisinf(__high2half(h))) != 0 && isfinite(lo) && isfinite(hi);
+      out[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    dst[idx] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
+}
+
+// ----------------------------------------------------------------- combine
+__global__ void combine_rows_kernel(const float4* __restrict__ src, const int32_t* __restrict__ inv, int top_k,
+                                    const WsHeader* hdr, uint2* __restrict__ out, int vecs_per_row, int need_saved) {
+  if (need_saved && !bwd_enabled(hdr)) return;
+  const int64_t total = (int64_t)hdr->qlen * vecs_per_row;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = idx / vecs_per_row;
+    const int c = (int)(idx - t * vecs_per_row);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < top_k; ++s) {
+      const int32_t p = inv[t * top_k + s];
+      if (p >= 0) {
+        const float4 v = src[(int64_t)p * vecs_per_row + c];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+    }
+    const uint32_t lo = (uint32_t)bf16_bits_rn(acc.x) | ((uint32_t)bf16_bits_rn(acc.y) << 16);
+    const uint32_t hi = (uint32_t)bf16_bits_rn(acc.z) | ((uint32_t)bf16_bits_rn(acc.w) << 16);
+    out[idx] = make_uint2(lo, hi);
+  }
+}
+
+__global__ void combine_route_kernel(const float* __restrict__ part, int nparts, const int32_t* __restrict__ inv,
+                                     int top_k, const WsHeader* hdr, float* __restrict__ grad_route) {
+  if (!bwd_enabled(hdr)) return;
+  const int64_t total = (int64_t)hdr->qlen * top_k;
+  for (int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f < total; f += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t p = inv[f];
+    float acc = 0.f;
+    if (p >= 0)
+      for (int b = 0; b < nparts; ++b) acc += part[(int64_t)p * nparts + b];
+    grad_route[f] = acc;
+  }
+}
+
+// --------------------------------------------------------- LoRA side rows
+constexpr int kLrRows = 32;
+constexpr int kLrK = 64;
+
+__global__ void __launch_bounds__(256) lora_rows_kernel(LoraRowsArgs a, const int4* __restrict__ tok_tiles,
+                                                        const WsHeader* hdr, int need_saved) {
+  if (need_saved && !bwd_enabled(hdr)) return;
+  const int ntiles = hdr->n_tok_tiles;
+  const int routed = hdr->routed;
+  const int tile = blockIdx.x;
+  __shared__ float Ls[kLrRows][kLrK + 1];
+  __shared__ float Rs[32][kLrK + 1];
+  if (tile >= ntiles) {
+    // the first spare block clears the padding rows past the last routed row
+    if (tile == ntiles) {
+      const int pad_end = (routed + 15) / 16 * 16 + 16;
+      for (int idx = threadIdx.x; idx < (pad_end - routed) * 64; idx += blockDim.x) {
+        const int64_t row = routed + idx / 64;
+        a.out0[row * 64 + idx % 64] = 0;
+        if (a.out1) a.out1[row * 64 + idx % 64] = 0;
+      }
+    }
+    return;
+  }
+  const int4 tt = tok_tiles[tile];
+  const int e = tt.x;
+  const int t = threadIdx.x;
+  const int rr = t >> 3;       // row inside the 32-row chunk
+  const int jg = t & 7;        // j = jg + 8*u
+  const int rank = a.rank;
+  for (int rc = 0; rc < tt.z; rc += kLrRows) {
+    const int nrows = min(kLrRows, tt.z - rc);
+    float res[2][4];
+    for (int half = 0; half < a.halves; ++half) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint16_t* R = a.R[half] + (int64_t)e * a.r_expert;
+      for (int k0 = 0; k0 < a.K; k0 += kLrK) {
+        __syncthreads();
+        for (int idx = t; idx < kLrRows * kLrK; idx += 256) {
+          const int r_ = idx / kLrK, kk = idx % kLrK;
+          float v = 0.f;
+          if (r_ < nrows) v = f16_bits_to_float(a.L[(int64_t)(tt.y + rc + r_) * a.ldL + a.colL[half] + k0 + kk]);
+          Ls[r_][kk] = v;
+        }
+        for (int idx = t; idx < 32 * kLrK; idx += 256) {
+          const int j = idx / kLrK, kk = idx % kLrK;
+          float v = 0.f;
+          if (j < rank) {
+            const int64_t o = a.r_style == 0 ? (int64_t)j * a.K + k0 + kk : (int64_t)(k0 + kk) * rank + j;
+            v = bf16_bits_to_float(R[o]);
+          }
+          Rs[j][kk] = v;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kLrK; ++kk) {
+          const float l = Ls[rr][kk];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[u] += l * Rs[jg + 8 * u][kk];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) res[half][u] = acc[u];
+    }
+    // stage the chunk's outputs, then write all 64 columns (zero padding included)
+    __syncthreads();
+    for (int half = 0; half < a.halves; ++half)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jg + 8 * u;
+        if (j < rank) Ls[rr][half * rank + j] = a.scale * res[half][u];
+      }
+    __syncthreads();
+    for (int idx = t; idx < nrows * 64; idx += 256) {
+      const int r_ = idx >> 6, col = idx & 63;
+      const int64_t row = tt.y + rc + r_;
+      const float v = col < a.halves * rank ? Ls[r_][col] : 0.f;
+      a.out0[row * 64 + col] = f16_bits_rn(v);
+      if (a.out1) a.out1[row * 64 + col] = f16_bits_rn(a.w_perm[row] * v);
+    }
+  }
+}
+
+// ------------------------------------------------------------- LoRA grads
+constexpr int kGp = 64;    // features per block
+constexpr int kGrows = 32; // rows staged per step
+
+__global__ void __launch_bounds__(256) lora_grad_kernel(const GradJobs jobs, const int32_t* __restrict__ offsets,
+                                                        int rank, int accumulate, float grad_scale, const WsHeader* hdr) {
+  if (!bwd_enabled(hdr)) return;
+  const GradJob jb = jobs.j[blockIdx.z];
+  const int e = blockIdx.y;
+  const int p0 = blockIdx.x * kGp;
+  if (p0 >= jb.P) return;
+  const int t = threadIdx.x;
+  const int pl = t & 63;
+  const int jq = t >> 6;  // j = jq + 4u, u < 8
+  const int row0 = offsets[e];
+  const int row1 = offsets[e + 1];
+  __shared__ float Ss[kGrows][33];
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const bool pv = p0 + pl < jb.P;
+  for (int r0 = row0; r0 < row1; r0 += kGrows) {
+    const int nr = min(kGrows, row1 - r0);
+    __syncthreads();
+    for (int idx = t; idx < kGrows * 32; idx += 256) {
+      const int r_ = idx >> 5, j = idx & 31;
+      Ss[r_][j] = (r_ < nr && j < rank) ? f16_bits_to_float(jb.S[(int64_t)(r0 + r_) * 64 + jb.colS + j]) : 0.f;
+    }
+    __syncthreads();
+    if (pv) {
+      for (int r_ = 0; r_ < nr; ++r_) {
+        const float l = f16_bits_to_float(jb.L[(int64_t)(r0 + r_) * jb.ldL + jb.colL + p0 + pl]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] += l * Ss[r_][jq + 4 * u];
+      }
+    }
+  }
+  if (!pv) return;
+  const bool has_rows = row1 > row0;
+  if (!has_rows && accumulate) return;
+  for (int u = 0; u < 8; ++u) {
+    const int j = jq + 4 * u;
+    if (j >= rank) continue;
+    const int64_t o = jb.transposed ? ((int64_t)e * rank + j) * jb.P + p0 + pl : ((int64_t)e * jb.P + p0 + pl) * rank + j;
+    float v = grad_scale * acc[u];
+    if (accumulate) v += bf16_bits_to_float(jb.out[o]);
+    jb.out[o] = bf16_bits_rn(v);
+  }
+}
+
+// ---------------------------------------------------------------- header
+__global__ void header_begin_fwd_kernel(WsHeader* hdr, int save) {
+  hdr->magic = kWsMagic;
+  hdr->saved = save ? 1u : 0u;
+}
+__global__ void header_check_bwd_kernel(WsHeader* hdr) {
+  if (hdr->magic != kWsMagic || hdr->saved != 1u) {
+    hdr->saved = 0u;
+    atomicOr(&hdr->status, (uint32_t)RAWINT4_DEV_NO_SAVED_FORWARD);
+  }
+}
+__global__ void header_end_bwd_kernel(WsHeader* hdr) { hdr->saved = 0u; }
+
+__global__ void fill_u16_kernel(uint16_t* p, int64_t count, uint16_t value) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = value;
+}
+
+// ---------------------------------------------------------------- decode
+__global__ void decode_kernel(const uint8_t* __restrict__ q, const uint16_t* __restrict__ s, int64_t n, int64_t k,
+                              float* __restrict__ out_f32, uint16_t* __restrict__ out_f16) {
+  const int64_t groups = n * (k / 32);
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = g / (k / 32);
+    const int64_t grp = g - row * (k / 32);
+    const uint8_t* src = q + row * (k / 2) + grp * 16;
+    const uint16_t sb = s[row * (k / 32) + grp];
+    uint4 qv;
+    uint8_t* qb = reinterpret_cast<uint8_t*>(&qv);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) qb[i] = src[i];
+    const int64_t o = row * k + grp * 32;
+    if (out_f16) {
+      uint32_t w[16];
+      decode_group32(qv, bf16_scale_to_h2(sb), w);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        out_f16[o + 2 * i] = (uint16_t)(w[i] & 0xFFFFu);
+        out_f16[o + 2 * i + 1] = (uint16_t)(w[i] >> 16);
+      }
+    }
+    if (out_f32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out_f32[o + i] = decode_one_f32(qb[i >> 1], i & 1, sb);
+    }
+  }
+}
+
+int grid_for(int64_t work, int threads) {
+  int64_t g = (work + threads - 1) / threads;
+  if (g > 148 * 16) g = 148 * 16;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, const WsHeader* hdr,
+                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved,
+                               cudaStream_t stream) {
+  const int vecs = H / 8;
+  gather_rows_kernel<<<grid_for((int64_t)max_rows * vecs, 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src_bf16), perm, top_k, hdr, reinterpret_cast<uint4*>(dst_f16), vecs, status,
+      need_saved);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_rows(const float* src, const int32_t* inv, int top_k, const WsHeader* hdr, uint16_t* out_bf16,
+                                int H, int max_tokens, int need_saved, cudaStream_t stream) {
+  const int vecs = H / 4;
+  combine_rows_kernel<<<grid_for((int64_t)max_tokens * vecs, 256), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(src), inv, top_k, hdr, reinterpret_cast<uint2*>(out_bf16), vecs, need_saved);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_route(const float* part, int nparts, const int32_t* inv, int top_k, const WsHeader* hdr,
+                                 float* grad_route, int max_tokens, cudaStream_t stream) {
+  combine_route_kernel<<<grid_for((int64_t)max_tokens * top_k, 256), 256, 0, stream>>>(part, nparts, inv, top_k, hdr,
+                                                                                       grad_route);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_rows(const LoraRowsArgs& a, const int4* tok_tiles, const WsHeader* hdr, int max_tiles,
+                             int need_saved, cudaStream_t stream) {
+  lora_rows_kernel<<<max_tiles + 1, 256, 0, stream>>>(a, tok_tiles, hdr, need_saved);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_grads(const GradJobs& jobs, int njobs, int pmax, const int32_t* offsets, int experts, int rank,
+                              int accumulate, float grad_scale, const WsHeader* hdr, cudaStream_t stream) {
+  dim3 grid((pmax + kGp - 1) / kGp, experts, njobs);
+  lora_grad_kernel<<<grid, 256, 0, stream>>>(jobs, offsets, rank, accumulate, grad_scale, hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_header_begin_fwd(WsHeader* hdr, int save, cudaStream_t stream) {
+  header_begin_fwd_kernel<<<1, 1, 0, stream>>>(hdr, save);
+  return cudaGetLastError();
+}
+cudaError_t launch_header_check_bwd(WsHeader* hdr, cudaStream_t stream) {
+  header_check_bwd_kernel<<<1, 1, 0, stream>>>(hdr);
+  return cudaGetLastError();
+}
+cudaError_t launch_header_end_bwd(WsHeader* hdr, cudaStream_t stream) {
+  header_end_bwd_kernel<<<1, 1, 0, stream>>>(hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_u16(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream) {
+  if (count <= 0) return cudaSuccess;
+  fill_u16_kernel<<<grid_for(count, 256), 256, 0, stream>>>(p, count, value);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, float* out_f32, uint16_t* out_f16,
+                          cudaStream_t stream) {
+  if (n <= 0 || k <= 0) return cudaSuccess;
+  decode_kernel<<<grid_for(n * (k / 32), 128), 128, 0, stream>>>(q, s, n, k, out_f32, out_f16);
+  return cudaGetLastError();
+}
+
+}  // namespace r4

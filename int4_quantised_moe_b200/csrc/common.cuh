@@ -1,0 +1,260 @@
+// Shared device helpers for the sm_100a RAWINT4 MoE-LoRA kernels:
+// inline-PTX wrappers for mbarriers, TMA (cp.async.bulk.tensor), tcgen05
+// (TMEM alloc, UMMA issue/commit, TMEM loads), bounded waits, and the
+// RAWINT4 -> FP16 decode used by every GEMM producer and by the decode
+// check export.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rawint4_moe.h"
+
+namespace r4 {
+
+// ------------------------------------------------------------------ status
+// Workspace header shared by all kernels of one layer call. Lives at the
+// start of the caller's workspace.
+struct WsHeader {
+  uint32_t magic;        // RAWINT4_WS_MAGIC once a forward ran
+  uint32_t saved;        // 1: a saved forward context is pending
+  int32_t qlen;          // tokens of the saved / last forward
+  int32_t routed;        // valid permuted rows (ids in [0, E))
+  uint32_t status;       // OR of RAWINT4_DEV_* bits
+  int32_t n_tok_tiles;   // entries of the token-tile list
+  int32_t pad[10];
+};
+constexpr uint32_t kWsMagic = 0x52344d45u;  // "R4ME"
+
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s bound on any spin
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ------------------------------------------------------------- smem / misc
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;  // (a & b) | c
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on phase `parity`. Returns false (and raises the abort flag and
+// the device timeout bit) when the bound expires or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_status(status, RAWINT4_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
+                                            int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
+                                            int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, FP16 inputs, FP32 accumulator.
+__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on `bar` when all previously issued MMAs of this thread finish.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Instruction descriptor, kind::f16: FP16 A/B, FP32 D, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc_f16(uint32_t n, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                          // D format: F32
+         | (0u << 7) | (0u << 10)           // A, B format: F16
+         | ((a_mn_major ? 1u : 0u) << 15)   // A major
+         | ((b_mn_major ? 1u : 0u) << 16)   // B major
+         | ((n >> 3) << 17)                 // N / 8
+         | ((128u >> 4) << 24);             // M / 16
+}
+
+// Shared-memory matrix descriptor with 128-byte swizzling.
+// lbo/sbo in bytes (multiples of 16); the atom base must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// 32 lanes x 32 consecutive 32-bit columns of TMEM into registers.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ decode
+// bf16 bit pattern -> fp16 pair holding the same value twice (exact for
+// magnitudes in the fp16 normal range).
+__device__ __forceinline__ __half2 bf16_scale_to_h2(uint16_t bits) {
+  const float f = __uint_as_float(static_cast<uint32_t>(bits) << 16);
+  return __float2half2_rn(f);
+}
+
+// Decode 16 packed bytes (32 RAWINT4 codes, low nibble first) that share one
+// group scale into 16 fp16x2 words, element order preserved: word j holds
+// values 2j (low half) and 2j+1 (high half).
+//
+// Per byte b: replicate it, keep the low nibble in bits 0-3 of the low half
+// and the high nibble in bits 4-7 of the high half, and OR in the exponent
+// of 1024.0 (fp16 0x6400, whose ulp is 1). That yields exactly 1024 + lo and
+// 1024 + 16*hi; one fused multiply-add by (1, 1/16) plus (-1032, -72) gives
+// lo - 8 and hi - 8 exactly, and one multiply by the scale gives the weight
+// (exact: at most 11 significant bits).
+__device__ __forceinline__ void decode_group32(const uint4 q, const __half2 s2, uint32_t (&out)[16]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
+  const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t rep = __byte_perm(w[i], 0u, 0x1111u * j);
+      const uint32_t v = lop3_and_or(rep, 0x00F0000Fu, 0x64006400u);
+      __half2 h = __hfma2(*reinterpret_cast<const __half2*>(&v), mul, add);
+      h = __hmul2(h, s2);
+      out[i * 4 + j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+
+// Plain fp32 decode of one code (for the check export's fp32 output).
+__device__ __forceinline__ float decode_one_f32(uint8_t byte, int hi, uint16_t scale_bits) {
+  const int code = hi ? (byte >> 4) : (byte & 15);
+  return static_cast<float>(code - 8) * __uint_as_float(static_cast<uint32_t>(scale_bits) << 16);
+}
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t bits) {
+  return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+}
+__device__ __forceinline__ uint16_t f16_bits_rn(float f) {
+  __half h = __float2half_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ float f16_bits_to_float(uint16_t bits) {
+  __half h = *reinterpret_cast<__half*>(&bits);
+  return __half2float(h);
+}
+
+// SiLU pieces with the exponent argument clamped so that exp never
+// overflows (the tails give sigma = 0 or 1 without NaN).
+__device__ __forceinline__ float sigmoid_clamped(float z) {
+  const float e = __expf(fminf(-z, 88.0f));
+  return 1.0f / (1.0f + e);
+}
+
+}  // namespace r4

@@ -1,0 +1,69 @@
+#pragma once
+#include "common.cuh"
+
+namespace r4 {
+
+// The four dequant-fused grouped GEMMs of the layer. All put 128 weight rows
+// (output features) on the UMMA M side and up to 256 permuted tokens of one
+// expert on the N side: D[m, n] = sum_k A[m, k] * B[n, k].
+enum GemmMode : int {
+  kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
+  kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
+  kModeDownT = 2,    // bwd  dh = dY W_d (+ LoRA), SwiGLU' + dRoute epilogue   A: MN-major decode of W_d (transpose-free)
+  kModeGateUpT = 3,  // bwd  dx = dG W_g + dU W_u (+ LoRA)                     A: MN-major decode of W_g/W_u
+};
+
+constexpr int kBlockK = 64;        // reduction elements per pipeline stage
+constexpr int kRowsM = 128;        // UMMA M
+constexpr int kStagesA = 2;        // decoded FP16 A tiles (16 KB each)
+constexpr int kStagesB = 4;        // TMA-loaded B tiles (32 KB each)
+constexpr int kStagesP = 8;        // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kThreads = 512;      // 16 warps
+constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
+constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
+constexpr int kDecThreads = 256;
+constexpr int kLoraPad = 64;       // width of the LoRA side matrices (>= 2 * rank)
+
+struct GemmParams {
+  const int4* tok_tiles;     // {expert, first permuted row, rows, 0}
+  const WsHeader* hdr;       // n_tok_tiles
+  uint32_t* status;
+  int n_rowblk;              // output row blocks per token tile
+  int n_main;                // main reduction stages (K / 64)
+  int need_saved;            // backward: run only when a saved forward is pending
+  // frozen base (packed, scales) of projection 0 and 1
+  const uint16_t* s0;
+  const uint16_t* s1;
+  int64_t s_expert;          // scale elements per expert
+  int s_row;                 // scales per stored row
+  int stored_rows;           // stored rows per expert of one projection (GU_T: I)
+  // LoRA operand of the extra reduction stage (bf16 LoRA tensors)
+  const uint16_t* lx0;
+  const uint16_t* lx1;
+  int64_t lx_expert;         // elements per expert
+  int lx_ld;                 // row length of the LoRA tensor
+  int rank;
+  // epilogue
+  const float* w_perm;
+  float* out_a;              // GU: G; DOWN: Yw; GU_T: dx
+  float* out_b;              // GU: U
+  uint16_t* out_h;           // GU: h (fp16); DOWN_T: dG|dU (fp16)
+  const float* in_g;         // DOWN_T: saved G
+  const float* in_u;         // DOWN_T: saved U
+  float* droute_part;        // DOWN_T: [rows, n_rowblk]
+  int ld_out;                // row length of out_a / out_b / out_h / in_*
+  int inter;
+  float limit;
+};
+
+struct GemmMaps {
+  CUtensorMap q0;  // packed projection 0: 3D uint8 {stored K bytes, stored rows, E}
+  CUtensorMap q1;  // packed projection 1
+  CUtensorMap b;   // B main: 2D fp16 {K, rows}, 128B swizzle, box {64, 16}
+  CUtensorMap bx;  // B LoRA: 2D fp16 {64, rows}, 128B swizzle, box {64, 16}
+};
+
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t stream);
+
+}  // namespace r4

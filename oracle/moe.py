@@ -53,7 +53,8 @@ class Layer:
     """Frozen base (packed bytes + float scales) and float64 LoRA tensors.
 
     gate_q/up_q: uint8 [E, I, H/2]; down_q: uint8 [E, H, I/2];
-    *_s: float64 scales [E, N, K/32]; lora[name]: float64 with the shapes
+    *_s: scales [E, N, K/32], float64 or bf16 bit patterns (uint16);
+    lora[name]: float64 with the shapes
     A: [E, r, K_in], B: [E, N_out, r].
     """
 
@@ -87,11 +88,17 @@ class Layer:
     def scaling(self) -> float:
         return self.alpha / self.rank
 
+    @staticmethod
+    def _scale(arr: np.ndarray, e: int) -> np.ndarray:
+        """Scales of expert e as float64 (bf16 bit patterns are widened exactly)."""
+        s = arr[e]
+        return rawint4.bf16_bits_to_f64(s) if s.dtype == np.uint16 else s
+
     def dense(self, e: int):
         """Dense float64 W_g, W_u [I, H] and W_d [H, I] of expert e."""
-        return (rawint4.dequantize_rawint4(self.gate_q[e], self.gate_s[e]),
-                rawint4.dequantize_rawint4(self.up_q[e], self.up_s[e]),
-                rawint4.dequantize_rawint4(self.down_q[e], self.down_s[e]))
+        return (rawint4.dequantize_rawint4(self.gate_q[e], self._scale(self.gate_s, e)),
+                rawint4.dequantize_rawint4(self.up_q[e], self._scale(self.up_s, e)),
+                rawint4.dequantize_rawint4(self.down_q[e], self._scale(self.down_s, e)))
 
 
 # ---------------------------------------------------------------------------
@@ -288,7 +295,7 @@ def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
         dy = ec.w[:, None] * g
         gd = dy @ lo["down_lora_b"]
         if transpose_free:
-            dh_base = rawint4.transpose_free_dx(dy, layer.down_q[e], layer.down_s[e])
+            dh_base = rawint4.transpose_free_dx(dy, layer.down_q[e], Layer._scale(layer.down_s, e))
         else:
             dh_base = dy @ Wd
         dh = dh_base + c * gd @ lo["down_lora_a"]
@@ -298,8 +305,8 @@ def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
         gb_g = dG @ lo["gate_lora_b"]
         gb_u = dU @ lo["up_lora_b"]
         if transpose_free:
-            dx = (rawint4.transpose_free_dx(dG, layer.gate_q[e], layer.gate_s[e])
-                  + rawint4.transpose_free_dx(dU, layer.up_q[e], layer.up_s[e]))
+            dx = (rawint4.transpose_free_dx(dG, layer.gate_q[e], Layer._scale(layer.gate_s, e))
+                  + rawint4.transpose_free_dx(dU, layer.up_q[e], Layer._scale(layer.up_s, e)))
         else:
             dx = dG @ Wg + dU @ Wu
         dx = dx + c * gb_g @ lo["gate_lora_a"] + c * gb_u @ lo["up_lora_a"]

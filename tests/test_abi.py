@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every entry point include/rawint4_moe.h declares (no GPU).
+
+Only host-side argument checks run here: they return before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rawint4_moe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"RAWINT4_API\s+(?:const\s+)?\w+\*?\s+(\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from int4_quantised_moe_b200 import build as b
+    b.build()
+    from int4_quantised_moe_b200 import binding
+    return binding
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    for n in ("rawint4_moe_lora_fwd", "rawint4_moe_lora_bwd", "rawint4_moe_lora_workspace_size",
+              "rawint4_moe_lora_status", "rawint4_moe_lora_strerror", "rawint4_decode", "rawint4_moe_permute"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    cdll = lib.library()
+    for n in _declared():
+        assert hasattr(cdll, n), n
+    assert set(_declared()) <= set(lib.EXPORTED_SYMBOLS) | {"rawint4_moe_permute_workspace_size"}
+
+
+def test_workspace_size_and_cfg_validation(lib):
+    ok = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 32)
+    n = lib.rawint4_moe_lora_workspace_size(ok)
+    assert n > 0 and n % 256 == 0
+    big = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 1000)
+    assert lib.rawint4_moe_lora_workspace_size(big) > n
+    bad = [
+        lib.make_cfg(4, 2, 200, 256, 8, 16.0, 0.0, 32),   # H not a multiple of 128
+        lib.make_cfg(4, 2, 256, 96, 8, 16.0, 0.0, 32),    # I not a multiple of 128
+        lib.make_cfg(4, 5, 256, 256, 8, 16.0, 0.0, 32),   # top_k > experts
+        lib.make_cfg(4, 2, 256, 256, 0, 16.0, 0.0, 32),   # rank 0
+        lib.make_cfg(4, 2, 256, 256, 33, 16.0, 0.0, 32),  # rank > 32
+        lib.make_cfg(4, 2, 256, 256, 8, float("nan"), 0.0, 32),
+        lib.make_cfg(4, 2, 256, 256, 8, 16.0, -1.0, 32),  # negative clamp limit
+        lib.make_cfg(4, 2, 256, 256, 8, 16.0, float("inf"), 32),
+        lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 0),
+    ]
+    for cfg in bad:
+        with pytest.raises(lib.RawInt4Error) as ei:
+            lib.rawint4_moe_lora_workspace_size(cfg)
+        assert ei.value.code == lib.INVALID_ARGUMENT
+
+
+def test_frozen_base_rejected_before_anything_else(lib):
+    """A non-null base-gradient pointer fails first, even with every other argument null."""
+    cdll = lib.library()
+    cfg = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 32)
+    grads = lib.LoraGrads()
+    rc = cdll.rawint4_moe_lora_bwd(ctypes.byref(cfg), None, None, None, None, None, ctypes.byref(grads),
+                                   ctypes.c_void_p(16), None, None, 0, 1.0, None, 0, None)
+    assert rc == lib.FROZEN_BASE
+    assert "frozen" in lib.strerror(rc)
+
+
+def test_host_argument_errors(lib):
+    cdll = lib.library()
+    cfg = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 32)
+    base, lora = lib.Base(), lib.Lora()
+    # null base / lora pointers
+    rc = cdll.rawint4_moe_lora_fwd(ctypes.byref(cfg), ctypes.byref(base), ctypes.byref(lora), 5, None, None, None,
+                                   None, 1, None, 0, None)
+    assert rc == lib.INVALID_ARGUMENT
+    v = ctypes.c_uint32(0)
+    assert cdll.rawint4_moe_lora_status(None, None, ctypes.byref(v)) == lib.INVALID_ARGUMENT
+    assert cdll.rawint4_decode(None, None, 4, 64, None, None, None) == lib.INVALID_ARGUMENT
+    n = ctypes.c_size_t(0)
+    assert cdll.rawint4_moe_permute_workspace_size(5, 2, 4, ctypes.byref(n)) == lib.OK and n.value > 0
+    assert cdll.rawint4_moe_permute_workspace_size(5, 0, 4, ctypes.byref(n)) == lib.INVALID_ARGUMENT
+    for code in range(0, 9):
+        assert lib.strerror(code) != "unknown status code"

@@ -1,0 +1,314 @@
+"""GPU parity of the whole layer against the float64 oracle, through the C ABI.
+
+Covers the small configurations element by element, the contract test's
+lifecycle (test_rawint4_sft_numerical.py: GAS1 overwrite with sentinel
+buffers, accumulation, the lazy clear of a new window, checkpoint-recompute
+cache replacement, frozen-base fail-fast, base bytes unchanged), the
+clamp-boundary fixture, the rectangular multiblock variant, the inference
+regression with zero LoRA, bad expert ids, qlen = 0 and a missing saved
+forward.
+"""
+
+import hashlib
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import metrics, moe as omoe
+from tests._gpu import (TOL_DX, TOL_LORA, TOL_OUT, TOL_ROUTE, grad_buffers, make_layer, run_fwd_bwd)
+from tests._util import f64, oracle_layer
+from workloads import CONFIGS, LORA_NAMES, Workload, lora_shapes, make_workload, small_config
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def close(name, actual, expected, tol):
+    a = actual.float().cpu().numpy() if isinstance(actual, torch.Tensor) else np.asarray(actual)
+    e = np.asarray(expected, dtype=np.float64)
+    assert np.all(np.isfinite(a)), f"{name}: non-finite values"
+    assert np.count_nonzero(e), f"{name}: reference has no signal"
+    rel, cos = metrics.relative_l2_and_cosine(a, e)
+    assert rel <= tol[0] and cos >= tol[1], f"{name}: rel-L2 {rel:.3e} (<= {tol[0]}), cos {cos:.6f} (>= {tol[1]})"
+    return rel, cos
+
+
+def oracle(wl: Workload):
+    layer = oracle_layer(wl)
+    out, ctx = omoe.forward(layer, f64(wl.x), wl.expert_ids.cpu().numpy(), f64(wl.route_weights))
+    gin, groute, grads = omoe.backward(layer, ctx, f64(wl.grad_out))
+    return out, gin, groute, grads
+
+
+def base_hash(wl: Workload) -> str:
+    h = hashlib.sha256()
+    for t in (wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s):
+        b = t.detach().cpu().contiguous().view(torch.uint8).numpy().tobytes()
+        h.update(len(b).to_bytes(8, "little"))
+        h.update(b)
+    return h.hexdigest()
+
+
+# ----------------------------------------------------- contract-test fixtures
+
+def contract_workload(inter=256, qlen=5, limit=0.0, seed=20261001):
+    """Layer of the contract test (E=4, k=2, H=256, r=8, alpha=16): uniform codes,
+    scales U[0.01, 0.07), signed extremes, one zero scale, LoRA N(0, 0.04^2)."""
+    cfg = small_config("contract", 4, 2, 256, inter, 8, qlen, swiglu_limit=limit, alpha=16.0)
+    wl = make_workload(cfg, seed=seed)
+    for n in LORA_NAMES:
+        wl.lora[n] = (wl.lora[n].float() * 2.0).to(torch.bfloat16)  # std 0.04
+    wl.gate_q[0, 0].fill_(0x00)
+    wl.up_q[0, 0].fill_(0xFF)
+    wl.gate_q[0, 1].fill_(0xFF)
+    wl.up_q[0, 1].fill_(0x00)
+    wl.gate_s[0, :2].fill_(0.0625)
+    wl.up_s[0, :2].fill_(0.0625)
+    wl.down_s[3, -1, -1] = 0.0
+    return wl
+
+
+def contract_batch(wl: Workload, pair, seed):
+    """_make_batch of the contract test: x ~ N(0, 0.2^2) with rows 0/1 at +1/-1,
+    grad_output ~ N(0, 0.1^2), alternating expert pairs, linspace route weights."""
+    Q, H = wl.cfg.qlen, wl.cfg.hidden
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn((Q, H), generator=g) * 0.2).to(torch.bfloat16)
+    x[0].fill_(1.0)
+    x[1].fill_(-1.0)
+    dy = (torch.randn((Q, H), generator=g) * 0.1).to(torch.bfloat16)
+    a, b = pair
+    ids = torch.tensor([[a, b] if t % 2 == 0 else [b, a] for t in range(Q)], dtype=torch.int64)
+    w = torch.stack((torch.linspace(0.55, 0.75, Q), torch.linspace(0.45, 0.25, Q)), 1).float()
+    return Workload(wl.cfg, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora, x, ids, w, dy)
+
+
+def on_gpu(wl: Workload) -> Workload:
+    return wl.to(DEV)
+
+
+# ------------------------------------------------------------------ tests
+
+@pytest.mark.parametrize("cfg_id", [0, 1])
+def test_config_parity(cfg_id):
+    wl = make_workload(CONFIGS[cfg_id])
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("limit", [0.0, 2.0])
+def test_rectangular_multiblock(limit):
+    """I = 384, Q = 17: every active expert gets 17 rows (a ragged token tile)."""
+    wl = contract_workload(inter=384, qlen=17, limit=limit)
+    b = contract_batch(wl, (0, 1), 3000)
+    out_r, gin_r, groute_r, grads_r = oracle(b)
+    g = on_gpu(b)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads, grad_scale=0.5)
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], 0.5 * grads_r[n], TOL_LORA)
+        for e in (2, 3):
+            assert torch.count_nonzero(grads[n][e]) == 0
+
+
+def test_gradient_window_lifecycle():
+    """GAS1 overwrite (sentinel 7.0), GAS2/GAS8 accumulation, lazy clear of a new
+    window, checkpoint-recompute cache replacement, frozen base, base unchanged."""
+    wl = contract_workload()
+    h0 = base_hash(wl)
+    scale = 0.5
+    pairs = ((0, 1), (1, 2), (2, 3), (0, 3)) * 2
+    batches = [contract_batch(wl, p, 3000 + i) for i, p in enumerate(pairs)]
+    refs = [oracle(b) for b in batches]
+    gw = on_gpu(wl)
+    layer = make_layer(gw, max_tokens=32)
+    grads = grad_buffers(gw)  # sentinel 7.0
+    gb = [on_gpu(b) for b in batches]
+
+    out, gin, groute = run_fwd_bwd(layer, gb[0], grads, accumulate=False, grad_scale=scale)
+    close("gas1.out", out, refs[0][0], TOL_OUT)
+    close("gas1.dX", gin, refs[0][1], TOL_DX)
+    close("gas1.dRoute", groute, refs[0][2], TOL_ROUTE)
+
+    def window(stage, idx, active):
+        for n in LORA_NAMES:
+            exp = sum(refs[i][3][n] for i in idx) * scale
+            close(f"{stage}.{n}", grads[n], exp, TOL_LORA)
+            for e in range(4):
+                if e not in active:
+                    assert torch.count_nonzero(grads[n][e]) == 0, f"{stage}.{n}: stale expert {e}"
+
+    window("gas1", [0], {0, 1})
+    run_fwd_bwd(layer, gb[1], grads, accumulate=True, grad_scale=scale)
+    window("gas2", [0, 1], {0, 1, 2})
+    for i in range(2, 8):
+        run_fwd_bwd(layer, gb[i], grads, accumulate=True, grad_scale=scale)
+    window("gas8", list(range(8)), {0, 1, 2, 3})
+
+    nw = contract_batch(wl, (2, 3), 4001)
+    nref = oracle(nw)
+    run_fwd_bwd(layer, on_gpu(nw), grads, accumulate=False, grad_scale=scale)
+    for n in LORA_NAMES:
+        close(f"lazy_clear.{n}", grads[n], nref[3][n] * scale, TOL_LORA)
+        for e in (0, 1):
+            assert torch.count_nonzero(grads[n][e]) == 0
+
+    # two saved forwards, then one backward: the second replaces the first
+    first, second = contract_batch(wl, (0, 1), 5001), contract_batch(wl, (1, 3), 5002)
+    fr, sr = oracle(first), oracle(second)
+    f_g, s_g = on_gpu(first), on_gpu(second)
+    layer.forward(f_g.expert_ids, f_g.route_weights, f_g.x)
+    layer.forward(s_g.expert_ids, s_g.route_weights, s_g.x)
+    s_dx = torch.empty_like(s_g.x)
+    s_dr = torch.empty(s_g.expert_ids.shape, dtype=torch.float32, device=DEV)
+    layer.backward(s_g.grad_out, grads, accumulate=False, grad_scale=scale, grad_in=s_dx, grad_route=s_dr)
+    layer.forward(f_g.expert_ids, f_g.route_weights, f_g.x)
+    f_dx = torch.empty_like(f_g.x)
+    f_dr = torch.empty(f_g.expert_ids.shape, dtype=torch.float32, device=DEV)
+    layer.backward(f_g.grad_out, grads, accumulate=True, grad_scale=scale, grad_in=f_dx, grad_route=f_dr)
+    close("lifo.second.dX", s_dx, sr[1], TOL_DX)
+    close("lifo.second.dRoute", s_dr, sr[2], TOL_ROUTE)
+    close("lifo.first.dX", f_dx, fr[1], TOL_DX)
+    close("lifo.first.dRoute", f_dr, fr[2], TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(f"cache_replacement.{n}", grads[n], (sr[3][n] + fr[3][n]) * scale, TOL_LORA)
+        assert torch.count_nonzero(grads[n][2]) == 0
+    assert layer.status() == 0
+
+    # frozen base: a base-gradient buffer is refused before anything is written
+    from int4_quantised_moe_b200 import binding as B
+    fb = on_gpu(contract_batch(wl, (0, 1), 7001))
+    layer.forward(fb.expert_ids, fb.route_weights, fb.x)
+    sentinel = torch.full_like(fb.x, 3.0)
+    forbidden = torch.empty(1, dtype=torch.bfloat16, device=DEV)
+    before = {n: grads[n].clone() for n in LORA_NAMES}
+    with pytest.raises(ValueError, match="frozen"):
+        layer.backward(fb.grad_out, grads, grad_in=sentinel, base_grad_gate=forbidden)
+    torch.cuda.synchronize()
+    assert torch.all(sentinel == 3.0)
+    for n in LORA_NAMES:
+        assert torch.equal(grads[n], before[n])
+    # the saved context is still pending: the proper backward runs
+    layer.backward(fb.grad_out, grads, grad_in=sentinel)
+    assert layer.status() == 0
+    assert base_hash(gw) == h0 == base_hash(wl)
+
+
+def test_clamp_boundary_fixture():
+    """Contract test's clamp fixture: pre-activations below, on and above +-L,
+    two of them rounding onto the bound in bf16 but masked in exact arithmetic."""
+    from tests.test_oracle_moe import _clamp_fixture
+    gold, wl = _clamp_fixture()
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    close("clamp.out", out, out_r, TOL_OUT)
+    close("clamp.dX", gin, gin_r, TOL_DX)
+    close("clamp.dRoute", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        if np.count_nonzero(grads_r[n]):
+            close(f"clamp.{n}", grads[n], grads_r[n], TOL_LORA)
+        else:
+            assert torch.count_nonzero(grads[n]) == 0, n
+
+
+def test_inference_regression_zero_lora():
+    wl = contract_workload()
+    b = contract_batch(wl, (0, 2), 6001)
+    for n in LORA_NAMES:
+        b.lora[n] = torch.zeros_like(b.lora[n])
+    layer_o = oracle_layer(b)
+    out_r, _ = omoe.forward(layer_o, f64(b.x), b.expert_ids.numpy(), f64(b.route_weights))
+    g = on_gpu(b)
+    layer = make_layer(g)
+    out = layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False)
+    close("inference.out", out, out_r, TOL_OUT)
+
+
+def test_bad_expert_id_and_status():
+    wl = make_workload(CONFIGS[0])
+    ids = wl.expert_ids.clone()
+    ids[2, 1] = wl.cfg.experts  # sentinel id: that slot contributes nothing
+    bad = Workload(wl.cfg, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora, wl.x, ids,
+                   wl.route_weights, wl.grad_out)
+    out_r, gin_r, groute_r, grads_r = oracle(bad)
+    g = on_gpu(bad)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    from int4_quantised_moe_b200 import binding as B
+    st = layer.status()
+    assert st & B.DEV_BAD_EXPERT_ID
+    assert layer.status() == 0  # reading clears
+    close("bad.out", out, out_r, TOL_OUT)
+    close("bad.grad_in", gin, gin_r, TOL_DX)
+    assert float(groute[2, 1]) == 0.0
+
+
+def test_backward_without_saved_forward_does_nothing():
+    from int4_quantised_moe_b200 import binding as B
+    wl = on_gpu(make_workload(CONFIGS[0]))
+    layer = make_layer(wl)
+    grads = grad_buffers(wl)
+    gin = torch.full_like(wl.x, 3.0)
+    layer.backward(wl.grad_out, grads, grad_in=gin)
+    assert layer.status() & B.DEV_NO_SAVED_FORWARD
+    assert torch.all(gin == 3.0) and all(torch.all(grads[n] == 7.0) for n in LORA_NAMES)
+    # one backward per saving forward; a forward without saving invalidates
+    layer.forward(wl.expert_ids, wl.route_weights, wl.x, save_for_backward=True)
+    layer.backward(wl.grad_out, grads, grad_in=gin)
+    assert layer.status() == 0
+    gin2 = torch.full_like(wl.x, 3.0)
+    layer.backward(wl.grad_out, grads, grad_in=gin2)
+    assert layer.status() & B.DEV_NO_SAVED_FORWARD
+    assert torch.all(gin2 == 3.0)
+    layer.forward(wl.expert_ids, wl.route_weights, wl.x, save_for_backward=False)
+    layer.backward(wl.grad_out, grads, grad_in=gin2)
+    assert layer.status() & B.DEV_NO_SAVED_FORWARD
+
+
+def test_qlen_zero():
+    wl = on_gpu(make_workload(CONFIGS[0]))
+    layer = make_layer(wl)
+    grads = grad_buffers(wl)
+    empty_x = wl.x[:0]
+    out = layer.forward(wl.expert_ids[:0], wl.route_weights[:0], empty_x)
+    # the backward needs real buffers; with a saved qlen of 0 it writes none of them
+    layer.backward(wl.grad_out, grads, accumulate=True, grad_in=torch.empty_like(wl.x))
+    assert all(torch.all(grads[n] == 7.0) for n in LORA_NAMES)
+    layer.forward(wl.expert_ids[:0], wl.route_weights[:0], empty_x)
+    layer.backward(wl.grad_out, grads, accumulate=False, grad_in=torch.empty_like(wl.x))
+    assert all(torch.count_nonzero(grads[n]) == 0 for n in LORA_NAMES)
+    assert layer.status() == 0
+
+
+def test_smaller_qlen_than_workspace():
+    """A workspace sized for more tokens than the call uses (ragged last tile)."""
+    cfg = small_config("ragged", 8, 2, 256, 256, 16, 37, swiglu_limit=2.0, x_std=2.0)
+    wl = make_workload(cfg, seed=99)
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g, max_tokens=300)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
