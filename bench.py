@@ -1,0 +1,386 @@
+#!/usr/bin/env python3
+"""Throughput of one forward + backward of the routed RAWINT4 MoE-LoRA layer.
+
+A step is one pass of the whole layer (routing permutation, gate/up, down,
+combine; backward gather, down^T, gate/up^T, combine, six LoRA gradients)
+over one synthetic batch. Default workload: the largest layer (E=384, top-8,
+H=7168, I=2048, rank 32, alpha 64, 8192 tokens, no clamp) on one B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--config C]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs a data-parallel
+replica on its own batch (weak scaling) and the six LoRA gradient buffers are
+summed over ranks with NCCL after every backward.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import CONFIGS, LORA_NAMES, LayerConfig, expert_counts, lora_shapes, make_batch, make_workload  # noqa: E402
+
+METRIC = "routed tokens/s per MoE layer (fwd+bwd) and % of HBM/tensor roofline, 1×B200"
+UNIT = "routed tokens/s"
+
+
+# ----------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "tflops": d["bf16_tflops"], "tflops_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def algorithmic(cfg: LayerConfig, counts: torch.Tensor):
+    """Algorithmic bytes and FLOPs of one fwd+bwd (weights of hit experts read
+    in fwd and bwd, LoRA params read twice and grads written, x/out/dY/grad_in
+    and a second read of x in bf16; saved activations not counted)."""
+    Q, k, H, I, r = cfg.qlen, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank
+    R = int(counts.sum())
+    hit = int((counts > 0).sum())
+    flops = 12 * R * H * I + 18 * R * r * (H + I) + 2 * R * I
+    w_e = 3 * H * I * (0.5 + 1.0 / 16.0)
+    l_e = 2 * r * (3 * H + 3 * I)
+    nbytes = 2 * w_e * hit + 3 * l_e * hit + 10 * Q * H
+    return nbytes, flops, R, hit
+
+
+def gemm_flops(name: str, R: int, cfg: LayerConfig) -> float:
+    H, I, r = cfg.hidden, cfg.inter, cfg.rank
+    return {
+        "gemm_gate_up": 2 * R * H * 2 * I + 2 * R * 2 * I * r,
+        "gemm_down": 2 * R * I * H + 2 * R * H * r,
+        "gemm_down_t": 2 * R * H * I + 2 * R * I * r,
+        "gemm_gate_up_t": 2 * R * 2 * I * H + 2 * R * 2 * r * H,
+    }.get(name, 0.0)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, target_s: float):
+    """Time the float64 oracle on whole experts of the workload until about
+    `target_s` seconds of CPU work; returns (routed rows, seconds, experts)."""
+    import numpy as np
+    from oracle import moe as omoe
+    from oracle import rawint4 as orq
+
+    def bits(t):
+        return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    ids = wl.expert_ids.cpu().numpy()
+    counts = np.bincount(ids.reshape(-1)[(ids.reshape(-1) >= 0) & (ids.reshape(-1) < wl.cfg.experts)],
+                         minlength=wl.cfg.experts)
+    order = [int(e) for e in np.argsort(-counts, kind="stable") if counts[e] > 0]
+    rows = 0
+    spent = 0.0
+    used = []
+    for e in order:
+        sel = np.nonzero((ids == e).any(axis=1))[0]
+        sub_ids = np.where(ids[sel] == e, 0, -1)
+        layer = omoe.Layer(
+            gate_q=wl.gate_q[e:e + 1].cpu().numpy(), gate_s=bits(wl.gate_s[e:e + 1]),
+            up_q=wl.up_q[e:e + 1].cpu().numpy(), up_s=bits(wl.up_s[e:e + 1]),
+            down_q=wl.down_q[e:e + 1].cpu().numpy(), down_s=bits(wl.down_s[e:e + 1]),
+            lora={n: orq.bf16_bits_to_f64(bits(wl.lora[n][e:e + 1])) for n in LORA_NAMES},
+            alpha=wl.cfg.alpha, swiglu_limit=wl.cfg.swiglu_limit)
+        x = orq.bf16_bits_to_f64(bits(wl.x[torch.as_tensor(sel, device=wl.x.device)]))
+        dy = orq.bf16_bits_to_f64(bits(wl.grad_out[torch.as_tensor(sel, device=wl.x.device)]))
+        rw = wl.route_weights.cpu().numpy()[sel].astype(np.float64)
+        t0 = time.perf_counter()
+        _, ctx = omoe.forward(layer, x, sub_ids, rw)
+        omoe.backward(layer, ctx, dy)
+        spent += time.perf_counter() - t0
+        rows += int(counts[e])
+        used.append(e)
+        if spent >= target_s:
+            break
+    return rows, spent, used
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.config]
+    workload_name = (f"{cfg.name}: E={cfg.experts} top_k={cfg.top_k} H={cfg.hidden} I={cfg.inter} r={cfg.rank} "
+                     f"alpha={cfg.alpha:g} qlen={cfg.qlen} swiglu_limit={cfg.swiglu_limit:g} routing={cfg.routing}")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, cfg, workload_name)
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    from int4_quantised_moe_b200 import binding as B
+
+    # layer (same on every rank) and this rank's batch
+    wl = make_workload(cfg, device=dev)
+    if rank > 0:
+        x, ids, w, g = make_batch(cfg, seed=20261001 + 7919 * rank, device=dev)
+        wl.x, wl.expert_ids, wl.route_weights, wl.grad_out = x, ids, w, g
+    counts = expert_counts(wl.expert_ids, cfg.experts)
+    nbytes, flops, R, hit = algorithmic(cfg, counts)
+    layer = B.Layer.create(cfg.experts, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank, cfg.alpha, cfg.swiglu_limit,
+                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora)
+    grads = {n: torch.zeros(s, dtype=torch.bfloat16, device=dev) for n, s in lora_shapes(cfg).items()}
+    out = torch.empty_like(wl.x)
+    gin = torch.empty_like(wl.x)
+    groute = torch.empty(wl.expert_ids.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=True)
+        layer.backward(wl.grad_out, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
+        if pg is not None:
+            for n in LORA_NAMES:
+                pg.all_reduce(grads[n])
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = layer.status()
+    if st:
+        raise RuntimeError(f"device status after warm-up: {st:#x}")
+
+    # ---- device-timed region (inputs resident in HBM) with per-launch events
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    B.profile_begin(64 * args.steps)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = B.profile_end(64 * args.steps)
+    clocks = sampler.stop()
+    barrier()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_step = ms_total / args.steps
+    value = cfg.qlen * cfg.top_k * world / (ms_step / 1e3)
+
+    # per-kernel averages and the dominant kernel's roofline
+    per = {}
+    for name, ms in launches:
+        per.setdefault(name, []).append(ms)
+    kern = {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "share": sum(v) / max(1e-9, sum(sum(x) for x in per.values()))}
+            for n, v in per.items()}
+    pk = peaks()
+    dom = max((n for n in kern if n.startswith("gemm_")), key=lambda n: kern[n]["avg_ms"] * kern[n]["launches"])
+    dom_flops = gemm_flops(dom, R, cfg)
+    achieved = dom_flops / (kern[dom]["avg_ms"] / 1e3) / 1e12
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        tj = json.load(open(tfile))
+        if tj.get("kernel") == dom and tj.get("config") == args.config:
+            traffic = tj.get("dram_bytes_per_launch")
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2), "peak": pk["tflops_sustained"],
+                "unit": "TFLOP/s", "frac": round(achieved / pk["tflops_sustained"], 4), "traffic": traffic,
+                "peak_source": f"{pk['source']} bf16 sustained (fp16 dense rate equals bf16)"}
+    t_roof = max(nbytes / (pk["hbm_gbs"] * 1e9), flops / (pk["tflops_sustained"] * 1e12)) * 1e3
+    step_roofline = {"bound": "tensor" if flops / pk["tflops_sustained"] / 1e12 > nbytes / pk["hbm_gbs"] / 1e9 else "hbm",
+                     "t_roof_ms": round(t_roof, 4), "frac": round(t_roof / ms_step, 4),
+                     "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
+                     "routed_rows": R, "experts_hit": hit}
+
+    # ---- end to end through the public API from pinned host buffers
+    h_x = wl.x.cpu().pin_memory()
+    h_ids = wl.expert_ids.cpu().pin_memory()
+    h_w = wl.route_weights.cpu().pin_memory()
+    h_g = wl.grad_out.cpu().pin_memory()
+    h_out = torch.empty_like(h_x).pin_memory()
+    h_gin = torch.empty_like(h_x).pin_memory()
+    h_gr = torch.empty(groute.shape, dtype=torch.float32).pin_memory()
+    d_x, d_ids, d_w, d_g = torch.empty_like(wl.x), torch.empty_like(wl.expert_ids), torch.empty_like(
+        wl.route_weights), torch.empty_like(wl.grad_out)
+
+    def e2e_step():
+        d_x.copy_(h_x, non_blocking=True)
+        d_ids.copy_(h_ids, non_blocking=True)
+        d_w.copy_(h_w, non_blocking=True)
+        d_g.copy_(h_g, non_blocking=True)
+        layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
+        layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
+        if pg is not None:
+            for n in LORA_NAMES:
+                pg.all_reduce(grads[n])
+        h_out.copy_(out, non_blocking=True)
+        h_gin.copy_(gin, non_blocking=True)
+        h_gr.copy_(groute, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
+    h2d = sum(t.numel() * t.element_size() for t in (h_x, h_ids, h_w, h_g))
+    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_gin, h_gr))
+    e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e_ms, 4),
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    st = layer.status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows, secs, used = oracle_sample(wl, args.cpu_seconds)
+        cpu = {"value": round(rows / secs, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"float64 NumPy oracle fwd+bwd of {len(used)} whole expert(s) of this workload "
+                         f"({rows} routed rows, {secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": workload_name, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "global_batch_tokens": cfg.qlen * world, "routed_rows_per_gpu": R,
+                       "l2": "inputs larger than L2: every step streams all hit experts' packed weights "
+                             f"({2 * hit * 3 * cfg.hidden * cfg.inter * (0.5 + 1 / 16) / 1e9:.1f} GB)"},
+            "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": len(launches), "clocks": clocks, "device_status": st,
+            "kernels": {n: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 4), "share": round(v["share"], 4)}
+                        for n, v in sorted(kern.items(), key=lambda kv: -kv[1]["share"])},
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:
+    """The oracle as it stands on the host cores; each step a bounded sample."""
+    wl = make_workload(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+    per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, per_step)
+    rows_t, secs_t = 0, 0.0
+    for _ in range(args.steps):
+        rows, secs, used = oracle_sample(wl, per_step)
+        rows_t += rows
+        secs_t += secs
+    value = rows_t / secs_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_t / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"each step: float64 NumPy oracle fwd+bwd of whole experts for about {per_step:.1f} s"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -197,6 +197,16 @@ RAWINT4_API int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t to
                         int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/* Timing hook for measurement (no counterpart in the method): while enabled,
+ * every kernel launch of the library records a CUDA event pair on the
+ * launch's stream (at most max_launches launches). profile_end synchronises
+ * on the recorded events and returns, per launch in issue order, a static
+ * kernel name and its duration in ms (names/ms: host arrays of max_out
+ * entries, may be NULL; *n_out = number of launches recorded). Not meant for
+ * concurrent use from several threads. */
+RAWINT4_API int rawint4_moe_profile_begin(int max_launches);
+RAWINT4_API int rawint4_moe_profile_end(int max_out, int* n_out, const char** names, float* ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,7 +10,7 @@ raises ImportError (there is no CPU fallback).
 _EXPORTS = (
     "Layer", "RawInt4Error", "FrozenBaseError", "library", "make_base", "make_cfg", "make_grads", "make_lora",
     "rawint4_decode", "rawint4_moe_lora_bwd", "rawint4_moe_lora_fwd", "rawint4_moe_lora_status",
-    "rawint4_moe_lora_workspace_size", "rawint4_moe_permute", "strerror",
+    "rawint4_moe_lora_workspace_size", "rawint4_moe_permute", "strerror", "profile_begin", "profile_end",
 )
 
 

@@ -41,6 +41,8 @@ EXPORTED_SYMBOLS = (
     "rawint4_decode",
     "rawint4_moe_permute_workspace_size",
     "rawint4_moe_permute",
+    "rawint4_moe_profile_begin",
+    "rawint4_moe_profile_end",
 )
 
 
@@ -92,7 +94,7 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_permute.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
-            getattr(lib, name).restype = ctypes.c_int
+            getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
     return lib
 
 
@@ -239,3 +241,25 @@ class Layer:
 
     def status(self, stream=None) -> int:
         return rawint4_moe_lora_status(self.workspace, stream)
+
+
+# ---------------------------------------------------------------------------
+# Timing hook (measurement only)
+# ---------------------------------------------------------------------------
+
+def profile_begin(max_launches: int = 4096) -> None:
+    _lib.rawint4_moe_profile_begin.argtypes = [ctypes.c_int]
+    _lib.rawint4_moe_profile_begin.restype = ctypes.c_int
+    _check(_lib.rawint4_moe_profile_begin(int(max_launches)), "rawint4_moe_profile_begin")
+
+
+def profile_end(max_out: int = 4096):
+    """Per launch in issue order: (kernel name, milliseconds)."""
+    _lib.rawint4_moe_profile_end.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                             ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]
+    _lib.rawint4_moe_profile_end.restype = ctypes.c_int
+    n = ctypes.c_int(0)
+    names = (ctypes.c_char_p * max_out)()
+    ms = (ctypes.c_float * max_out)()
+    _check(_lib.rawint4_moe_profile_end(max_out, ctypes.byref(n), names, ms), "rawint4_moe_profile_end")
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, max_out))]

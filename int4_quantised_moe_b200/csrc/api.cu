@@ -8,6 +8,7 @@
 
 #include "aux.cuh"
 #include "gemm.cuh"
+#include "prof.cuh"
 #include "route.cuh"
 
 namespace r4 {
@@ -225,13 +226,22 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   void* ws = workspace;
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
 
-  R4_TRY(launch_header_begin_fwd(hdr, save_for_backward, st));
-  R4_TRY(launch_route(expert_ids, route_weights, qlen, k, E, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
+  {
+    R4_PROF("header_fwd", st);
+    R4_TRY(launch_header_begin_fwd(hdr, save_for_backward, st));
+  }
+  {
+    R4_PROF("route", st);
+    R4_TRY(launch_route(expert_ids, route_weights, qlen, k, E, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                       at<int32_t>(ws, L.inv), at<float>(ws, L.w_perm), at<int4>(ws, L.tiles), at<int32_t>(ws, L.hist),
                       hdr, st));
+  }
   if (qlen == 0) return RAWINT4_OK;
   const int maxR = qlen * k;
-  R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, st));
+  {
+    R4_PROF("gather_x", st);
+    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, st));
+  }
 
   // xa = c * X_perm [A_g; A_u]^T (rank-r side matrix of gate and up)
   LoraRowsArgs la{};
@@ -250,7 +260,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   la.out1 = nullptr;
   la.w_perm = nullptr;
   const int max_tiles = max_tok_tiles(maxR, E);
-  R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+  {
+    R4_PROF("lora_xa", st);
+    R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+  }
 
   GemmMaps mp;
   GemmParams gp{};
@@ -282,7 +295,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.out_b = at<float>(ws, L.u);
   gp.out_h = at<uint16_t>(ws, L.h);
   gp.ld_out = I;
-  R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  {
+    R4_PROF("gemm_gate_up", st);
+    R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  }
 
   // ha = c * h A_d^T, hw = w * ha
   LoraRowsArgs lb{};
@@ -298,7 +314,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   lb.out0 = at<uint16_t>(ws, L.ha);
   lb.out1 = at<uint16_t>(ws, L.hw);
   lb.w_perm = at<float>(ws, L.w_perm);
-  R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+  {
+    R4_PROF("lora_ha", st);
+    R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+  }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
   if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
@@ -317,10 +336,16 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.out_b = nullptr;
   gp.out_h = nullptr;
   gp.ld_out = H;
-  R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  {
+    R4_PROF("gemm_down", st);
+    R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  }
 
   // out[t] = sum over slots, fixed order
-  R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, st));
+  {
+    R4_PROF("combine_out", st);
+    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, st));
+  }
   return RAWINT4_OK;
 }
 
@@ -348,9 +373,15 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   const int maxR = maxQ * k;
   const int max_tiles = max_tok_tiles(maxR, E);
 
-  R4_TRY(launch_header_check_bwd(hdr, st));
-  R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR, &hdr->status, 1,
+  {
+    R4_PROF("header_bwd", st);
+    R4_TRY(launch_header_check_bwd(hdr, st));
+  }
+  {
+    R4_PROF("gather_dy", st);
+    R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR, &hdr->status, 1,
                             st));
+  }
 
   // gd = c * g B_d, gdw = w * gd (rank-r side of the down LoRA backward)
   LoraRowsArgs la{};
@@ -366,7 +397,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   la.out0 = at<uint16_t>(ws, L.gd);
   la.out1 = at<uint16_t>(ws, L.gdw);
   la.w_perm = at<float>(ws, L.w_perm);
-  R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+  {
+    R4_PROF("lora_gd", st);
+    R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+  }
 
   GemmMaps mp;
   GemmParams gp{};
@@ -399,7 +433,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.in_u = at<float>(ws, L.u);
   gp.droute_part = at<float>(ws, L.dpart);
   gp.ld_out = I;
-  R4_TRY(launch_gemm(kModeDownT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  {
+    R4_PROF("gemm_down_t", st);
+    R4_TRY(launch_gemm(kModeDownT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  }
 
   // gb = c * [dG B_g, dU B_u]
   LoraRowsArgs lb{};
@@ -418,7 +455,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   lb.out0 = at<uint16_t>(ws, L.gb);
   lb.out1 = nullptr;
   lb.w_perm = nullptr;
-  R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+  {
+    R4_PROF("lora_gb", st);
+    R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+  }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
   if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
@@ -440,11 +480,20 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.in_g = gp.in_u = nullptr;
   gp.droute_part = nullptr;
   gp.ld_out = H;
-  R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  {
+    R4_PROF("gemm_gate_up_t", st);
+    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+  }
 
-  R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, st));
+  {
+    R4_PROF("combine_dx", st);
+    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, st));
+  }
   if (grad_route)
+    {
+    R4_PROF("combine_route", st);
     R4_TRY(launch_combine_route(at<float>(ws, L.dpart), I / 128, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ, st));
+  }
 
   // the six LoRA gradients with the authoritative window
   GradJobs jobs{};
@@ -454,9 +503,15 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   jobs.j[3] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), 0, grads->gate_a, 1};
   jobs.j[4] = GradJob{at<uint16_t>(ws, L.dgu), 2 * I, I, I, at<uint16_t>(ws, L.xa), r, grads->up_b, 0};
   jobs.j[5] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), r, grads->up_a, 1};
-  R4_TRY(launch_lora_grads(jobs, 6, H > I ? H : I, at<int32_t>(ws, L.offsets), E, r, accumulate, grad_scale, hdr, st));
+  {
+    R4_PROF("lora_grads", st);
+    R4_TRY(launch_lora_grads(jobs, 6, H > I ? H : I, at<int32_t>(ws, L.offsets), E, r, accumulate, grad_scale, hdr, st));
+  }
 
-  R4_TRY(launch_header_end_bwd(hdr, st));
+  {
+    R4_PROF("header_end", st);
+    R4_TRY(launch_header_end_bwd(hdr, st));
+  }
   return RAWINT4_OK;
 }
 
@@ -508,7 +563,10 @@ int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t
   int32_t* hist = at<int32_t>(workspace, align_up(sizeof(WsHeader), kAlign) +
                                              align_up((size_t)max_tok_tiles(slots, experts) * 16, kAlign));
   if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return RAWINT4_CUDA_ERROR;
-  R4_TRY(launch_route(ids, nullptr, qlen, top_k, experts, offsets, perm, inv, nullptr, tiles, hist, hdr, st));
+  {
+    R4_PROF("route", st);
+    R4_TRY(launch_route(ids, nullptr, qlen, top_k, experts, offsets, perm, inv, nullptr, tiles, hist, hdr, st));
+  }
   if (slots > 0) {
     tail_fill_kernel<<<(slots + 255) / 256, 256, 0, st>>>(perm, offsets, experts, slots);
     R4_TRY(cudaGetLastError());

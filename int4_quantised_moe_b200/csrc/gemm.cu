@@ -113,10 +113,14 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Fill the A tile of the LoRA reduction stage (fp16, same layout as the main stages).
+// This thread's 32 values of the A tile of the LoRA reduction stage, as 16
+// fp16 pairs in the same order the decode produces (see a_chunk_off).
+// Loaded at the start of a work item, long before the stage is stored: a
+// decoder warp that stores operand data right after long-latency global loads
+// at the tail of a work item produced corrupted rows in earlier builds, and
+// the early load also takes that latency off the critical path.
 template <int MODE>
-__device__ __forceinline__ void fill_lora_a(const GemmParams& p, uint8_t* A, int e, int rb, int dt) {
-  uint32_t w[16];
+__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, int dt, uint32_t (&w)[16]) {
   const int r = p.rank;
   if constexpr (!kAMnMajor<MODE>) {
     // A[m, j] with j in [32*half, 32*half + 32): LoRA B rows (K-major, rank contiguous)
@@ -136,8 +140,7 @@ __device__ __forceinline__ void fill_lora_a(const GemmParams& p, uint8_t* A, int
       float v[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int j = 32 * half + 2 * t + u;
-        const int jj = j - jlo;
+        const int jj = 32 * half + 2 * t + u - jlo;
         v[u] = (jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
       }
       w[t] = pack_h2(v[0], v[1]);
@@ -146,27 +149,25 @@ __device__ __forceinline__ void fill_lora_a(const GemmParams& p, uint8_t* A, int
     // A[m, kr] with m in [32*qq, 32*qq + 32): LoRA A rows (MN-major, feature contiguous)
     const int kr = dt >> 2, qq = dt & 3;
     const uint16_t* src = nullptr;
-    if constexpr (MODE == kModeDownT) {
-      if (kr < r) src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + rb * 128 + 32 * qq;
-    } else {
-      if (kr < r)
-        src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + rb * 128 + 32 * qq;
-      else if (kr < 2 * r)
-        src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - r) * p.lx_ld + rb * 128 + 32 * qq;
-    }
+    if (kr < r)
+      src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + rb * 128 + 32 * qq;
+    else if (MODE == kModeGateUpT && kr < 2 * r)
+      src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - r) * p.lx_ld + rb * 128 + 32 * qq;
+    if (src) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float a = 0.f, b = 0.f;
-      if (src) {
-        a = bf16_bits_to_float(__ldg(src + 2 * t));
-        b = bf16_bits_to_float(__ldg(src + 2 * t + 1));
+      for (int c = 0; c < 4; ++c) {
+        const uint4 b = __ldg(s4 + c);
+        const uint32_t in[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[4 * c + t] = pack_h2(__uint_as_float(in[t] << 16), __uint_as_float(in[t] & 0xFFFF0000u));
       }
-      w[t] = pack_h2(a, b);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) w[t] = 0u;
     }
   }
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
 }
 
 template <int MODE>
@@ -455,6 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int rb = tile % n_rowblk;
       const int e = tt.x;
+      uint32_t lora_w[16];
+      lora_values<MODE>(p, e, rb, dt, lora_w);
       uint16_t scale_next = n_main > 0 ? load_scale<MODE>(p, e, rb, 0, dt) : 0;
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
@@ -474,7 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
                 make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         } else {
-          fill_lora_a<MODE>(p, A, e, rb, dt);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
+                make_uint4(lora_w[4 * j], lora_w[4 * j + 1], lora_w[4 * j + 2], lora_w[4 * j + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
