@@ -59,7 +59,8 @@ enum {
   RAWINT4_BAD_EXPERT_ID = 5,    /* reported through the device status word */
   RAWINT4_DEVICE_TIMEOUT = 6,   /* a bounded pipeline wait expired (device status) */
   RAWINT4_FP16_OVERFLOW = 7,    /* an operand overflowed FP16 (device status) */
-  RAWINT4_UNSUPPORTED = 8       /* no sm_100 device, or shape outside the kernels' limits */
+  RAWINT4_UNSUPPORTED = 8,      /* no sm_100 device, or shape outside the kernels' limits */
+  RAWINT4_STATIC_SCRATCH_TOO_SMALL = 9 /* rawint4_moe_permute_static: needs more than its fixed scratch */
 };
 
 /* Bits of the device status word (rawint4_moe_lora_status). */
@@ -196,6 +197,29 @@ RAWINT4_API int rawint4_moe_permute_workspace_size(int32_t qlen, int32_t top_k, 
 RAWINT4_API int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t experts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, void* workspace,
                         size_t ws_bytes, void* stream);
+
+/* Same permutation as rawint4_moe_permute, for callers that cannot call
+ * cudaMalloc to provide its scratch buffer (for example code running while
+ * another component owns all device memory, or code that must not risk the
+ * device-wide synchronisation a cudaMalloc can cause). No counterpart in the
+ * paper; it exists only to serve such callers.
+ *   ids, qlen, top_k, experts, offsets, perm, inv: as rawint4_moe_permute
+ *   (device pointers, caller-owned outputs).
+ * The scratch (header, tile list, per-block histograms: about
+ * 512 + 16*(E + ceil(Q*k/256)) + 4*E*ceil(Q*k/1024) bytes) lives in a fixed
+ * device array of rawint4_moe_permute_static_max_bytes() bytes (1 MiB)
+ * inside the library; every GPU that loads the library holds it until the
+ * process exits. Larger problems are rejected with
+ * RAWINT4_STATIC_SCRATCH_TOO_SMALL before anything is enqueued. The first
+ * call on a device looks up the array's device address (once per device, on
+ * the current device); make that first call before any stream capture. All
+ * calls share the one array, so calls whose work overlaps on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine. */
+RAWINT4_API int rawint4_moe_permute_static(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t experts,
+                                           int32_t* offsets, int32_t* perm, int32_t* inv, void* stream);
+RAWINT4_API size_t rawint4_moe_permute_static_max_bytes(void);
 
 /* Timing hook for measurement (no counterpart in the method): while enabled,
  * every kernel launch of the library records a CUDA event pair on the

@@ -26,6 +26,7 @@ BAD_EXPERT_ID = 5
 DEVICE_TIMEOUT = 6
 FP16_OVERFLOW = 7
 UNSUPPORTED = 8
+STATIC_SCRATCH_TOO_SMALL = 9
 
 DEV_BAD_EXPERT_ID = 1 << 0
 DEV_NO_SAVED_FORWARD = 1 << 1
@@ -43,6 +44,8 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_permute",
     "rawint4_moe_profile_begin",
     "rawint4_moe_profile_end",
+    "rawint4_moe_permute_static",
+    "rawint4_moe_permute_static_max_bytes",
 )
 
 
@@ -92,9 +95,12 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp]
     lib.rawint4_moe_permute_workspace_size.argtypes = [i32, i32, i32, P(sz)]
     lib.rawint4_moe_permute.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    lib.rawint4_moe_permute_static.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+    lib.rawint4_moe_permute_static_max_bytes.argtypes = []
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
+    lib.rawint4_moe_permute_static_max_bytes.restype = ctypes.c_size_t
     return lib
 
 
@@ -196,6 +202,18 @@ def rawint4_moe_permute(expert_ids: torch.Tensor, experts: int, offsets, perm, i
     ws = torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=expert_ids.device)
     _check(_lib.rawint4_moe_permute(_ptr(expert_ids), q, k, experts, _ptr(offsets), _ptr(perm), _ptr(inv),
                                     _ptr(ws), ws.numel(), _stream(stream)), "rawint4_moe_permute")
+
+
+def rawint4_moe_permute_static(expert_ids: torch.Tensor, experts: int, offsets, perm, inv, stream=None) -> None:
+    """rawint4_moe_permute without caller scratch: for callers that cannot
+    allocate device memory; uses the library's fixed 1 MiB device array."""
+    q, k = expert_ids.shape
+    _check(_lib.rawint4_moe_permute_static(_ptr(expert_ids), q, k, experts, _ptr(offsets), _ptr(perm), _ptr(inv),
+                                           _stream(stream)), "rawint4_moe_permute_static")
+
+
+def rawint4_moe_permute_static_max_bytes() -> int:
+    return int(_lib.rawint4_moe_permute_static_max_bytes())
 
 
 # ---------------------------------------------------------------------------

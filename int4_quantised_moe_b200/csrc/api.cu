@@ -204,6 +204,8 @@ const char* rawint4_moe_lora_strerror(int code) {
     case RAWINT4_DEVICE_TIMEOUT: return "a device pipeline wait exceeded its bound; results are invalid";
     case RAWINT4_FP16_OVERFLOW: return "an activation exceeded the fp16 operand range; results are invalid";
     case RAWINT4_UNSUPPORTED: return "unsupported device (needs sm_100) or configuration";
+    case RAWINT4_STATIC_SCRATCH_TOO_SMALL:
+      return "problem too large for the fixed scratch of rawint4_moe_permute_static; use rawint4_moe_permute";
     default: return "unknown status code";
   }
 }
