@@ -174,6 +174,9 @@ def main():
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--experts", type=int, default=None, help="override the expert count (profiling cases)")
+    ap.add_argument("--qlen", type=int, default=None, help="override the token count (profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -182,6 +185,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = CONFIGS[args.config]
+    if args.experts is not None or args.qlen is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, name=cfg.name + "_override", experts=args.experts or cfg.experts,
+                                  qlen=args.qlen or cfg.qlen)
     workload_name = (f"{cfg.name}: E={cfg.experts} top_k={cfg.top_k} H={cfg.hidden} I={cfg.inter} r={cfg.rank} "
                      f"alpha={cfg.alpha:g} qlen={cfg.qlen} swiglu_limit={cfg.swiglu_limit:g} routing={cfg.routing}")
 
@@ -287,6 +294,10 @@ def main():
                      "routed_rows": R, "experts_hit": hit}
 
     # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if args.no_e2e:
+        return finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline,
+                      e2e, launches, clocks, kern, hit)
     h_x = wl.x.cpu().pin_memory()
     h_ids = wl.expert_ids.cpu().pin_memory()
     h_w = wl.route_weights.cpu().pin_memory()
@@ -327,8 +338,13 @@ def main():
     d2h = sum(t.numel() * t.element_size() for t in (h_out, h_gin, h_gr))
     e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e_ms, 4),
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    st = layer.status()
+    return finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline,
+                  e2e, launches, clocks, kern, hit)
 
+
+def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline, e2e,
+           launches, clocks, kern, hit):
+    st = layer.status()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows, secs, used = oracle_sample(wl, args.cpu_seconds)

@@ -10,6 +10,7 @@
 #include "gemm.cuh"
 #include "prof.cuh"
 #include "route.cuh"
+#include "skinny.cuh"
 
 namespace r4 {
 namespace {
@@ -21,6 +22,8 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t hdr, offsets, perm, inv, w_perm, tiles, hist;
   size_t xp, xa, g, u, h, ha, hw, y, gp, gd, gdw, dgu, gb, dpart;
+  size_t gu16, ad16, bdt16, bgt16, but16;  // FP16 LoRA copies for the row products
+  int rpad;
   size_t total;
   int64_t rows;  // padded permuted-row capacity
   int max_tiles;
@@ -61,6 +64,13 @@ Layout make_layout(const rawint4_moe_cfg& c) {
   L.dgu = take(rows * 2 * I * 2);
   L.gb = take(rows * kLoraPad * 2);
   L.dpart = take(rows * (I / 128) * 4);
+  L.rpad = (c.rank + 15) / 16 * 16;
+  const int64_t rp = L.rpad;
+  L.gu16 = take(E * 2 * rp * H * 2);
+  L.ad16 = take(E * rp * I * 2);
+  L.bdt16 = take(E * rp * H * 2);
+  L.bgt16 = take(E * rp * I * 2);
+  L.but16 = take(E * rp * I * 2);
   L.total = off;
   return L;
 }
@@ -143,15 +153,29 @@ bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp16 row-major [rows, cols]; box {64, 16}, 128-byte swizzle (UMMA K-major B layout)
-bool map_act(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols) {
+// fp16 row-major [rows, cols]; box {64, box_rows}, 128-byte swizzle (UMMA
+// K-major operand rows, or MN-major atoms when rows are the reduction)
+bool map_act(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols, int box_rows = 16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
-  cuuint32_t box[2] = {64, 16};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 per-expert matrices [E, rows, cols]; box {64, rows, 1}, 128-byte swizzle
+bool map_expert_rows(CUtensorMap* m, const uint16_t* base, int64_t E, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(cols * rows * 2)};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -223,7 +247,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   if (rc != RAWINT4_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream_);
   const rawint4_moe_cfg& c = *cfg;
-  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank;
+  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank, rp = L.rpad;
   const float scaling = c.alpha / (float)r;
   void* ws = workspace;
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
@@ -235,36 +259,49 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("route", st);
     R4_TRY(launch_route(expert_ids, route_weights, qlen, k, E, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
-                      at<int32_t>(ws, L.inv), at<float>(ws, L.w_perm), at<int4>(ws, L.tiles), at<int32_t>(ws, L.hist),
-                      hdr, st));
+                        at<int32_t>(ws, L.inv), at<float>(ws, L.w_perm), at<int4>(ws, L.tiles),
+                        at<int32_t>(ws, L.hist), hdr, st));
   }
   if (qlen == 0) return RAWINT4_OK;
   const int maxR = qlen * k;
-  {
-    R4_PROF("gather_x", st);
-    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, st));
-  }
-
-  // xa = c * X_perm [A_g; A_u]^T (rank-r side matrix of gate and up)
-  LoraRowsArgs la{};
-  la.L = at<uint16_t>(ws, L.xp);
-  la.ldL = H;
-  la.colL[0] = la.colL[1] = 0;
-  la.K = H;
-  la.R[0] = lora->gate_a;
-  la.R[1] = lora->up_a;
-  la.r_expert = (int64_t)r * H;
-  la.r_style = 0;
-  la.rank = r;
-  la.halves = 2;
-  la.scale = scaling;
-  la.out0 = at<uint16_t>(ws, L.xa);
-  la.out1 = nullptr;
-  la.w_perm = nullptr;
   const int max_tiles = max_tok_tiles(maxR, E);
   {
+    R4_PROF("gather_x", st);
+    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0,
+                              st));
+  }
+  {
+    R4_PROF("lora_convert", st);
+    LoraCvt cv[2] = {{lora->gate_a, lora->up_a, at<uint16_t>(ws, L.gu16), r, rp, H, 0, 2},
+                     {lora->down_a, nullptr, at<uint16_t>(ws, L.ad16), r, rp, I, 0, 1}};
+    R4_TRY(launch_lora_convert(cv, 2, E, st));
+  }
+
+  SkParams sp{};
+  sp.tok_tiles = at<int4>(ws, L.tiles);
+  sp.hdr = hdr;
+  sp.status = &hdr->status;
+  sp.need_saved = 0;
+  sp.rank = r;
+  sp.rpad = rp;
+  sp.scale = scaling;
+  sp.w_perm = at<float>(ws, L.w_perm);
+  SkMaps sm;
+  const int rows_grid = grid_for_tiles(sms, 2 * max_tiles, 1);
+
+  // xa = c * X_perm [A_g; A_u]^T: gate in columns [0, r), up in [rp, rp + r)
+  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.xp), L.rows, H, 128) ||
+      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.gu16), E, 2 * rp, H))
+    return RAWINT4_CUDA_ERROR;
+  sp.nseg = 1;
+  sp.seg_lcol[0] = 0;
+  sp.nk = H / 64;
+  sp.sw = 2 * rp;
+  sp.out0 = at<uint16_t>(ws, L.xa);
+  sp.out1 = nullptr;
+  {
     R4_PROF("lora_xa", st);
-    R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+    R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
   }
 
   GemmMaps mp;
@@ -274,6 +311,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.status = &hdr->status;
   gp.need_saved = 0;
   gp.rank = r;
+  gp.rpad = rp;
   gp.w_perm = at<float>(ws, L.w_perm);
   gp.inter = I;
   gp.limit = c.swiglu_limit;
@@ -302,23 +340,17 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
 
-  // ha = c * h A_d^T, hw = w * ha
-  LoraRowsArgs lb{};
-  lb.L = at<uint16_t>(ws, L.h);
-  lb.ldL = I;
-  lb.K = I;
-  lb.R[0] = lb.R[1] = lora->down_a;
-  lb.r_expert = (int64_t)r * I;
-  lb.r_style = 0;
-  lb.rank = r;
-  lb.halves = 1;
-  lb.scale = scaling;
-  lb.out0 = at<uint16_t>(ws, L.ha);
-  lb.out1 = at<uint16_t>(ws, L.hw);
-  lb.w_perm = at<float>(ws, L.w_perm);
+  // ha = c * h A_d^T and hw = w * ha
+  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.h), L.rows, I, 128) ||
+      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.ad16), E, rp, I))
+    return RAWINT4_CUDA_ERROR;
+  sp.nk = I / 64;
+  sp.sw = rp;
+  sp.out0 = at<uint16_t>(ws, L.ha);
+  sp.out1 = at<uint16_t>(ws, L.hw);
   {
     R4_PROF("lora_ha", st);
-    R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 0, st));
+    R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
@@ -342,8 +374,6 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("gemm_down", st);
     R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
-
-  // out[t] = sum over slots, fixed order
   {
     R4_PROF("combine_out", st);
     R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, st));
@@ -367,7 +397,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   if (rc != RAWINT4_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream_);
   const rawint4_moe_cfg& c = *cfg;
-  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank;
+  const int H = c.hidden, I = c.inter, E = c.experts, k = c.top_k, r = c.rank, rp = L.rpad;
   const float scaling = c.alpha / (float)r;
   void* ws = workspace;
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
@@ -381,27 +411,42 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
   {
     R4_PROF("gather_dy", st);
-    R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR, &hdr->status, 1,
-                            st));
+    R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR,
+                              &hdr->status, 1, st));
+  }
+  {
+    R4_PROF("lora_convert", st);
+    LoraCvt cv[3] = {{lora->down_b, nullptr, at<uint16_t>(ws, L.bdt16), r, rp, H, 1, 1},
+                     {lora->gate_b, nullptr, at<uint16_t>(ws, L.bgt16), r, rp, I, 1, 1},
+                     {lora->up_b, nullptr, at<uint16_t>(ws, L.but16), r, rp, I, 1, 1}};
+    R4_TRY(launch_lora_convert(cv, 3, E, st));
   }
 
-  // gd = c * g B_d, gdw = w * gd (rank-r side of the down LoRA backward)
-  LoraRowsArgs la{};
-  la.L = at<uint16_t>(ws, L.gp);
-  la.ldL = H;
-  la.K = H;
-  la.R[0] = la.R[1] = lora->down_b;
-  la.r_expert = (int64_t)H * r;
-  la.r_style = 1;
-  la.rank = r;
-  la.halves = 1;
-  la.scale = scaling;
-  la.out0 = at<uint16_t>(ws, L.gd);
-  la.out1 = at<uint16_t>(ws, L.gdw);
-  la.w_perm = at<float>(ws, L.w_perm);
+  SkParams sp{};
+  sp.tok_tiles = at<int4>(ws, L.tiles);
+  sp.hdr = hdr;
+  sp.status = &hdr->status;
+  sp.need_saved = 1;
+  sp.rank = r;
+  sp.rpad = rp;
+  sp.scale = scaling;
+  sp.w_perm = at<float>(ws, L.w_perm);
+  SkMaps sm;
+  const int rows_grid = grid_for_tiles(sms, 2 * max_tiles, 1);
+
+  // gd = c * g B_d and gdw = w * gd
+  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.gp), L.rows, H, 128) ||
+      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.bdt16), E, rp, H))
+    return RAWINT4_CUDA_ERROR;
+  sp.nseg = 1;
+  sp.seg_lcol[0] = 0;
+  sp.nk = H / 64;
+  sp.sw = rp;
+  sp.out0 = at<uint16_t>(ws, L.gd);
+  sp.out1 = at<uint16_t>(ws, L.gdw);
   {
     R4_PROF("lora_gd", st);
-    R4_TRY(launch_lora_rows(la, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+    R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
   }
 
   GemmMaps mp;
@@ -411,6 +456,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.status = &hdr->status;
   gp.need_saved = 1;
   gp.rank = r;
+  gp.rpad = rp;
   gp.w_perm = at<float>(ws, L.w_perm);
   gp.inter = I;
   gp.limit = c.swiglu_limit;
@@ -440,26 +486,21 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_TRY(launch_gemm(kModeDownT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
 
-  // gb = c * [dG B_g, dU B_u]
-  LoraRowsArgs lb{};
-  lb.L = at<uint16_t>(ws, L.dgu);
-  lb.ldL = 2 * I;
-  lb.colL[0] = 0;
-  lb.colL[1] = I;
-  lb.K = I;
-  lb.R[0] = lora->gate_b;
-  lb.R[1] = lora->up_b;
-  lb.r_expert = (int64_t)I * r;
-  lb.r_style = 1;
-  lb.rank = r;
-  lb.halves = 2;
-  lb.scale = scaling;
-  lb.out0 = at<uint16_t>(ws, L.gb);
-  lb.out1 = nullptr;
-  lb.w_perm = nullptr;
+  // gb = c * [dG B_g, dU B_u]: gate in columns [0, r), up in [rp, rp + r)
+  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.dgu), L.rows, 2 * I, 128) ||
+      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.bgt16), E, rp, I) ||
+      !map_expert_rows(&sm.b[1], at<uint16_t>(ws, L.but16), E, rp, I))
+    return RAWINT4_CUDA_ERROR;
+  sp.nseg = 2;
+  sp.seg_lcol[0] = 0;
+  sp.seg_lcol[1] = I;
+  sp.nk = I / 64;
+  sp.sw = rp;
+  sp.out0 = at<uint16_t>(ws, L.gb);
+  sp.out1 = nullptr;
   {
     R4_PROF("lora_gb", st);
-    R4_TRY(launch_lora_rows(lb, at<int4>(ws, L.tiles), hdr, max_tiles, 1, st));
+    R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
@@ -486,30 +527,48 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("gemm_gate_up_t", st);
     R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
-
   {
     R4_PROF("combine_dx", st);
     R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, st));
   }
-  if (grad_route)
-    {
+  if (grad_route) {
     R4_PROF("combine_route", st);
-    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), I / 128, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ, st));
+    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), I / 128, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ,
+                                st));
   }
 
   // the six LoRA gradients with the authoritative window
-  GradJobs jobs{};
-  jobs.j[0] = GradJob{at<uint16_t>(ws, L.gp), H, 0, H, at<uint16_t>(ws, L.hw), 0, grads->down_b, 0};
-  jobs.j[1] = GradJob{at<uint16_t>(ws, L.h), I, 0, I, at<uint16_t>(ws, L.gdw), 0, grads->down_a, 1};
-  jobs.j[2] = GradJob{at<uint16_t>(ws, L.dgu), 2 * I, 0, I, at<uint16_t>(ws, L.xa), 0, grads->gate_b, 0};
-  jobs.j[3] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), 0, grads->gate_a, 1};
-  jobs.j[4] = GradJob{at<uint16_t>(ws, L.dgu), 2 * I, I, I, at<uint16_t>(ws, L.xa), r, grads->up_b, 0};
-  jobs.j[5] = GradJob{at<uint16_t>(ws, L.xp), H, 0, H, at<uint16_t>(ws, L.gb), r, grads->up_a, 1};
   {
+    SkParams gq{};
+    gq.hdr = hdr;
+    gq.status = &hdr->status;
+    gq.need_saved = 1;
+    gq.rank = r;
+    gq.rpad = rp;
+    gq.offsets = at<int32_t>(ws, L.offsets);
+    gq.experts = E;
+    gq.njobs = 4;
+    gq.accumulate = accumulate;
+    gq.grad_scale = grad_scale;
+    // L (features), S (rank side), split, transposed, output features, outputs
+    gq.job[0] = SkJob{H, 0, H / 128, kSplitNone, 0, H, grads->down_b, nullptr};
+    gq.job[1] = SkJob{I, 0, I / 128, kSplitNone, 1, I, grads->down_a, nullptr};
+    gq.job[2] = SkJob{2 * I, 0, 2 * I / 128, kSplitFeature, 0, I, grads->gate_b, grads->up_b};
+    gq.job[3] = SkJob{H, 0, H / 128, kSplitRank, 1, H, grads->gate_a, grads->up_a};
+    SkMaps gm;
+    if (!map_act(&gm.a[0], at<uint16_t>(ws, L.gp), L.rows, H, 64) ||
+        !map_act(&gm.b[0], at<uint16_t>(ws, L.hw), L.rows, kLoraPad, 64) ||
+        !map_act(&gm.a[1], at<uint16_t>(ws, L.h), L.rows, I, 64) ||
+        !map_act(&gm.b[1], at<uint16_t>(ws, L.gdw), L.rows, kLoraPad, 64) ||
+        !map_act(&gm.a[2], at<uint16_t>(ws, L.dgu), L.rows, 2 * I, 64) ||
+        !map_act(&gm.b[2], at<uint16_t>(ws, L.xa), L.rows, kLoraPad, 64) ||
+        !map_act(&gm.a[3], at<uint16_t>(ws, L.xp), L.rows, H, 64) ||
+        !map_act(&gm.b[3], at<uint16_t>(ws, L.gb), L.rows, kLoraPad, 64))
+      return RAWINT4_CUDA_ERROR;
+    const int items = E * (H / 128 + I / 128 + 2 * I / 128 + H / 128);
     R4_PROF("lora_grads", st);
-    R4_TRY(launch_lora_grads(jobs, 6, H > I ? H : I, at<int32_t>(ws, L.offsets), E, r, accumulate, grad_scale, hdr, st));
+    R4_TRY(launch_skinny(kSkGrads, gq, gm, grid_for_tiles(sms, items, 1), st));
   }
-
   {
     R4_PROF("header_end", st);
     R4_TRY(launch_header_end_bwd(hdr, st));

@@ -1,8 +1,6 @@
 // Memory-bound helpers of the layer: row gather into expert order (with the
-// bf16 -> fp16 operand conversion), the fixed-order top-k combines, the
-// rank-r LoRA side matrices, the per-expert LoRA gradient reductions with the
-// contract test's authoritative window, header bookkeeping and the decode
-// check export.
+// bf16 -> fp16 operand conversion), the fixed-order top-k combines, header
+// bookkeeping and the decode check export.
 #include "aux.cuh"
 
 namespace r4 {
@@ -74,137 +72,6 @@ __global__ void combine_route_kernel(const float* __restrict__ part, int nparts,
     if (p >= 0)
       for (int b = 0; b < nparts; ++b) acc += part[(int64_t)p * nparts + b];
     grad_route[f] = acc;
-  }
-}
-
-// --------------------------------------------------------- LoRA side rows
-constexpr int kLrRows = 32;
-constexpr int kLrK = 64;
-
-__global__ void __launch_bounds__(256) lora_rows_kernel(LoraRowsArgs a, const int4* __restrict__ tok_tiles,
-                                                        const WsHeader* hdr, int need_saved) {
-  if (need_saved && !bwd_enabled(hdr)) return;
-  const int ntiles = hdr->n_tok_tiles;
-  const int routed = hdr->routed;
-  const int tile = blockIdx.x;
-  __shared__ float Ls[kLrRows][kLrK + 1];
-  __shared__ float Rs[32][kLrK + 1];
-  if (tile >= ntiles) {
-    // the first spare block clears the padding rows past the last routed row
-    if (tile == ntiles) {
-      const int pad_end = (routed + 15) / 16 * 16 + 16;
-      for (int idx = threadIdx.x; idx < (pad_end - routed) * 64; idx += blockDim.x) {
-        const int64_t row = routed + idx / 64;
-        a.out0[row * 64 + idx % 64] = 0;
-        if (a.out1) a.out1[row * 64 + idx % 64] = 0;
-      }
-    }
-    return;
-  }
-  const int4 tt = tok_tiles[tile];
-  const int e = tt.x;
-  const int t = threadIdx.x;
-  const int rr = t >> 3;       // row inside the 32-row chunk
-  const int jg = t & 7;        // j = jg + 8*u
-  const int rank = a.rank;
-  for (int rc = 0; rc < tt.z; rc += kLrRows) {
-    const int nrows = min(kLrRows, tt.z - rc);
-    float res[2][4];
-    for (int half = 0; half < a.halves; ++half) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint16_t* R = a.R[half] + (int64_t)e * a.r_expert;
-      for (int k0 = 0; k0 < a.K; k0 += kLrK) {
-        __syncthreads();
-        for (int idx = t; idx < kLrRows * kLrK; idx += 256) {
-          const int r_ = idx / kLrK, kk = idx % kLrK;
-          float v = 0.f;
-          if (r_ < nrows) v = f16_bits_to_float(a.L[(int64_t)(tt.y + rc + r_) * a.ldL + a.colL[half] + k0 + kk]);
-          Ls[r_][kk] = v;
-        }
-        for (int idx = t; idx < 32 * kLrK; idx += 256) {
-          const int j = idx / kLrK, kk = idx % kLrK;
-          float v = 0.f;
-          if (j < rank) {
-            const int64_t o = a.r_style == 0 ? (int64_t)j * a.K + k0 + kk : (int64_t)(k0 + kk) * rank + j;
-            v = bf16_bits_to_float(R[o]);
-          }
-          Rs[j][kk] = v;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < kLrK; ++kk) {
-          const float l = Ls[rr][kk];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) acc[u] += l * Rs[jg + 8 * u][kk];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) res[half][u] = acc[u];
-    }
-    // stage the chunk's outputs, then write all 64 columns (zero padding included)
-    __syncthreads();
-    for (int half = 0; half < a.halves; ++half)
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = jg + 8 * u;
-        if (j < rank) Ls[rr][half * rank + j] = a.scale * res[half][u];
-      }
-    __syncthreads();
-    for (int idx = t; idx < nrows * 64; idx += 256) {
-      const int r_ = idx >> 6, col = idx & 63;
-      const int64_t row = tt.y + rc + r_;
-      const float v = col < a.halves * rank ? Ls[r_][col] : 0.f;
-      a.out0[row * 64 + col] = f16_bits_rn(v);
-      if (a.out1) a.out1[row * 64 + col] = f16_bits_rn(a.w_perm[row] * v);
-    }
-  }
-}
-
-// ------------------------------------------------------------- LoRA grads
-constexpr int kGp = 64;    // features per block
-constexpr int kGrows = 32; // rows staged per step
-
-__global__ void __launch_bounds__(256) lora_grad_kernel(const GradJobs jobs, const int32_t* __restrict__ offsets,
-                                                        int rank, int accumulate, float grad_scale, const WsHeader* hdr) {
-  if (!bwd_enabled(hdr)) return;
-  const GradJob jb = jobs.j[blockIdx.z];
-  const int e = blockIdx.y;
-  const int p0 = blockIdx.x * kGp;
-  if (p0 >= jb.P) return;
-  const int t = threadIdx.x;
-  const int pl = t & 63;
-  const int jq = t >> 6;  // j = jq + 4u, u < 8
-  const int row0 = offsets[e];
-  const int row1 = offsets[e + 1];
-  __shared__ float Ss[kGrows][33];
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  const bool pv = p0 + pl < jb.P;
-  for (int r0 = row0; r0 < row1; r0 += kGrows) {
-    const int nr = min(kGrows, row1 - r0);
-    __syncthreads();
-    for (int idx = t; idx < kGrows * 32; idx += 256) {
-      const int r_ = idx >> 5, j = idx & 31;
-      Ss[r_][j] = (r_ < nr && j < rank) ? f16_bits_to_float(jb.S[(int64_t)(r0 + r_) * 64 + jb.colS + j]) : 0.f;
-    }
-    __syncthreads();
-    if (pv) {
-      for (int r_ = 0; r_ < nr; ++r_) {
-        const float l = f16_bits_to_float(jb.L[(int64_t)(r0 + r_) * jb.ldL + jb.colL + p0 + pl]);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] += l * Ss[r_][jq + 4 * u];
-      }
-    }
-  }
-  if (!pv) return;
-  const bool has_rows = row1 > row0;
-  if (!has_rows && accumulate) return;
-  for (int u = 0; u < 8; ++u) {
-    const int j = jq + 4 * u;
-    if (j >= rank) continue;
-    const int64_t o = jb.transposed ? ((int64_t)e * rank + j) * jb.P + p0 + pl : ((int64_t)e * jb.P + p0 + pl) * rank + j;
-    float v = grad_scale * acc[u];
-    if (accumulate) v += bf16_bits_to_float(jb.out[o]);
-    jb.out[o] = bf16_bits_rn(v);
   }
 }
 
@@ -287,19 +154,6 @@ cudaError_t launch_combine_route(const float* part, int nparts, const int32_t* i
                                  float* grad_route, int max_tokens, cudaStream_t stream) {
   combine_route_kernel<<<grid_for((int64_t)max_tokens * top_k, 256), 256, 0, stream>>>(part, nparts, inv, top_k, hdr,
                                                                                        grad_route);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lora_rows(const LoraRowsArgs& a, const int4* tok_tiles, const WsHeader* hdr, int max_tiles,
-                             int need_saved, cudaStream_t stream) {
-  lora_rows_kernel<<<max_tiles + 1, 256, 0, stream>>>(a, tok_tiles, hdr, need_saved);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lora_grads(const GradJobs& jobs, int njobs, int pmax, const int32_t* offsets, int experts, int rank,
-                              int accumulate, float grad_scale, const WsHeader* hdr, cudaStream_t stream) {
-  dim3 grid((pmax + kGp - 1) / kGp, experts, njobs);
-  lora_grad_kernel<<<grid, 256, 0, stream>>>(jobs, offsets, rank, accumulate, grad_scale, hdr);
   return cudaGetLastError();
 }
 

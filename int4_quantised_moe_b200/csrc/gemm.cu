@@ -38,29 +38,15 @@ constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;
 constexpr int kSmemBytes = kOffEpi + kEpiFloats * 4 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-struct Ring {
-  int stage = 0;
-  uint32_t phase = 0;
-  __device__ __forceinline__ void advance(int n) {
-    if (++stage == n) {
-      stage = 0;
-      phase ^= 1u;
-    }
-  }
-};
-
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
-  return __all_sync(0xffffffffu, ok);
-}
-
 template <int MODE>
 constexpr bool kAMnMajor = (MODE == kModeDownT || MODE == kModeGateUpT);
 
+// 16-wide MMA steps of the LoRA stage: one rank block (padded to rpad) per
+// projection, two for the gate/up pair.
 template <int MODE>
-__device__ __forceinline__ int kext_steps(int rank) {
-  const int kext = (MODE == kModeGateUp || MODE == kModeGateUpT) ? 2 * rank : rank;
-  return (kext + 15) / 16;
+__device__ __forceinline__ int kext_steps(int rpad) {
+  const int kext = (MODE == kModeGateUp || MODE == kModeGateUpT) ? 2 * rpad : rpad;
+  return kext / 16;
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
@@ -130,7 +116,7 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, 
     if constexpr (MODE == kModeGateUp) {
       const bool up = m >= 64;
       src = (up ? p.lx1 : p.lx0) + (int64_t)e * p.lx_expert + (int64_t)(rb * 64 + (m & 63)) * p.lx_ld;
-      jlo = up ? r : 0;
+      jlo = up ? p.rpad : 0;
     } else {
       src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)(rb * 128 + m) * p.lx_ld;
       jlo = 0;
@@ -151,8 +137,8 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, 
     const uint16_t* src = nullptr;
     if (kr < r)
       src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + rb * 128 + 32 * qq;
-    else if (MODE == kModeGateUpT && kr < 2 * r)
-      src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - r) * p.lx_ld + rb * 128 + 32 * qq;
+    else if (MODE == kModeGateUpT && kr >= p.rpad && kr < p.rpad + r)
+      src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - p.rpad) * p.lx_ld + rb * 128 + 32 * qq;
     if (src) {
       const uint4* s4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -295,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ UMMA issuer
     Ring ra, rbr;
     int it = 0;
-    const int ksteps_x = kext_steps<MODE>(p.rank);
+    const int ksteps_x = kext_steps<MODE>(p.rpad);
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int n_mma = (tt.z + 15) & ~15;

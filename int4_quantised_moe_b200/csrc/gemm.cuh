@@ -43,6 +43,7 @@ struct GemmParams {
   int64_t lx_expert;         // elements per expert
   int lx_ld;                 // row length of the LoRA tensor
   int rank;
+  int rpad;                  // rank rounded up to 16 (width of one rank block in the side matrices)
   // epilogue
   const float* w_perm;
   float* out_a;              // GU: G; DOWN: Yw; GU_T: dx

@@ -1,0 +1,395 @@
+// Rank-r LoRA products on the tensor cores (see skinny.cuh).
+//
+// One persistent CTA per SM; warp 0 issues TMA loads of both operands into a
+// ring of stages, warp 1 issues the UMMAs into a double-buffered TMEM
+// accumulator, warps 2-5 run the epilogue. No thread ever writes an operand
+// tile except to clear the rows past an expert's last row in the gradient
+// mode (constant stores, fenced for the async proxy before the MMA reads).
+#include "skinny.cuh"
+
+namespace r4 {
+namespace {
+
+constexpr int kSkA = 128 * 64 * 2;  // A tile: 128 rows x 64 fp16
+constexpr int kSkB = 64 * 64 * 2;   // B tile: 64 rows x 64 fp16
+constexpr int kSkStage = kSkA + kSkB;
+constexpr int kSkOffBar = kSkStages * kSkStage;
+constexpr int kSkNumBars = 2 * kSkStages + 4;
+constexpr int kSkOffMisc = kSkOffBar + kSkNumBars * 8;
+constexpr int kSkSmem = kSkOffMisc + 16 + 1024;
+static_assert(kSkSmem <= 232448, "shared memory budget");
+constexpr uint32_t kSkTmemCols = 256;
+
+struct GradItem {
+  int job, e, fb;
+};
+
+__device__ __forceinline__ GradItem grad_item(const SkParams& p, int item) {
+  GradItem g{0, 0, 0};
+  int base = 0;
+  for (int j = 0; j < p.njobs; ++j) {
+    const int n = p.experts * p.job[j].nfb;
+    if (item < base + n) {
+      const int rem = item - base;
+      g.job = j;
+      g.e = rem / p.job[j].nfb;
+      g.fb = rem - g.e * p.job[j].nfb;
+      return g;
+    }
+    base += n;
+  }
+  return g;
+}
+
+__device__ __forceinline__ int total_items(const SkParams& p, int mode) {
+  if (mode == kSkRows) return p.hdr->n_tok_tiles * 2;
+  int n = 0;
+  for (int j = 0; j < p.njobs; ++j) n += p.experts * p.job[j].nfb;
+  return n;
+}
+
+// Zero rows [r0, r1) of a 64-row MN-major 128B-swizzled block (rows are 128 B).
+__device__ __forceinline__ void zero_rows(uint8_t* blk, int r0, int r1, int lane) {
+  const int n16 = (r1 - r0) * 8;
+  for (int i = lane; i < n16; i += 32) {
+    const int row = r0 + (i >> 3);
+    *reinterpret_cast<uint4*>(blk + (row >> 3) * 1024 + (row & 7) * 128 + ((i & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Authoritative-window store of one gradient element.
+__device__ __forceinline__ void grad_store(uint16_t* out, int64_t o, float v, int accumulate) {
+  if (accumulate) v += bf16_bits_to_float(out[o]);
+  out[o] = bf16_bits_rn(v);
+}
+
+// One (feature p, rank j) gradient element of job `jb` for expert e.
+__device__ __forceinline__ void grad_element(const SkJob& jb, int rank, int rpad, int e, int p, int j, const float* D,
+                                             float gs, int accumulate, bool zero) {
+  uint16_t* out = jb.out_lo;
+  int pp = p, dj = j;
+  if (jb.split == kSplitFeature) {
+    const int half = jb.P / 2;
+    if (p >= half) {
+      out = jb.out_hi;
+      pp = p - half;
+      dj = rpad + j;
+    }
+  }
+  auto put = [&](uint16_t* buf, int jj, int dcol) {
+    const int64_t o = jb.transposed ? ((int64_t)e * rank + jj) * jb.pout + pp : ((int64_t)e * jb.pout + pp) * rank + jj;
+    grad_store(buf, o, zero ? 0.f : gs * D[dcol], zero ? 0 : accumulate);
+  };
+  put(out, j, dj);
+  if (jb.split == kSplitRank) put(jb.out_hi, j, rpad + j);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kSkThreads, 1)
+    skinny_kernel(const __grid_constant__ SkParams p, const __grid_constant__ SkMaps maps) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kSkStages;
+  uint64_t* acc_full = empty + kSkStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSkOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkOffMisc + 4);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSkStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kSkTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  uint32_t* status = p.status;
+  const bool enabled = !(p.need_saved && p.hdr->saved != 1u);
+  const int n_items = enabled ? total_items(p, MODE) : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    Ring ring;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      if constexpr (MODE == kSkRows) {
+        const int4 tt = p.tok_tiles[item >> 1];
+        const int mb = item & 1;
+        if (mb * 128 >= tt.z) continue;
+        const int p0 = tt.y + mb * 128;
+        const int bb = p.sw * 128;  // R box: sw rows of 64 fp16
+        for (int s = 0; s < p.nseg; ++s) {
+          for (int k = 0; k < p.nk; ++k) {
+            if (!wait_all(&empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
+            if (lane == 0) {
+              uint8_t* st = smem + ring.stage * kSkStage;
+              mbar_expect_tx(&full[ring.stage], kSkA + bb);
+              tma_load_2d(st, &maps.a[0], &full[ring.stage], p.seg_lcol[s] + 64 * k, p0);
+              tma_load_3d(st + kSkA, &maps.b[s], &full[ring.stage], 64 * k, 0, tt.x);
+            }
+            __syncwarp();
+            ring.advance(kSkStages);
+          }
+        }
+      } else {
+        const GradItem g = grad_item(p, item);
+        const SkJob& jb = p.job[g.job];
+        const int row0 = p.offsets[g.e], row1 = p.offsets[g.e + 1];
+        const int nk = (row1 - row0 + 63) / 64;
+        for (int k = 0; k < nk; ++k) {
+          if (!wait_all(&empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
+          if (lane == 0) {
+            uint8_t* st = smem + ring.stage * kSkStage;
+            mbar_expect_tx(&full[ring.stage], kSkA + kSkB);
+            const int x = jb.lcol + 128 * g.fb;
+            tma_load_2d(st, &maps.a[g.job], &full[ring.stage], x, row0 + 64 * k);
+            tma_load_2d(st + kSkA / 2, &maps.a[g.job], &full[ring.stage], x + 64, row0 + 64 * k);
+            tma_load_2d(st + kSkA, &maps.b[g.job], &full[ring.stage], 0, row0 + 64 * k);
+          }
+          __syncwarp();
+          ring.advance(kSkStages);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    Ring ring;
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      int nk, nseg, row0 = 0, rows = 0;
+      if constexpr (MODE == kSkRows) {
+        const int4 tt = p.tok_tiles[item >> 1];
+        if ((item & 1) * 128 >= tt.z) continue;
+        nk = p.nk;
+        nseg = p.nseg;
+      } else {
+        const GradItem g = grad_item(p, item);
+        row0 = p.offsets[g.e];
+        rows = p.offsets[g.e + 1] - row0;
+        nk = (rows + 63) / 64;
+        nseg = 1;
+        if (nk == 0) continue;
+      }
+      const int ab = it & 1;
+      if (!wait_all(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status)) goto done;
+      tc_fence_after();
+      for (int s = 0; s < nseg; ++s) {
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * 128 + s * 64);
+        for (int k = 0; k < nk; ++k) {
+          if (!wait_all(&full[ring.stage], ring.phase, abort_flag, status)) goto done;
+          uint8_t* st = smem + ring.stage * kSkStage;
+          int ksteps = 4;
+          if constexpr (MODE == kSkGrads) {
+            const int rem = rows - 64 * k;
+            if (rem < 64) {
+              // rows past the expert's last row belong to other experts: clear
+              // them in both operands up to the next 16-row MMA step
+              ksteps = (rem + 15) / 16;
+              const int r1 = ksteps * 16;
+              zero_rows(st, rem, r1, lane);
+              zero_rows(st + kSkA / 2, rem, r1, lane);
+              zero_rows(st + kSkA, rem, r1, lane);
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_base = smem_u32(st);
+            const uint32_t b_base = smem_u32(st + kSkA);
+            for (int kk = 0; kk < ksteps; ++kk) {
+              uint64_t ad, bd;
+              uint32_t idesc;
+              if constexpr (MODE == kSkRows) {
+                ad = make_sdesc_sw128(a_base + kk * 32, 16, 1024);
+                bd = make_sdesc_sw128(b_base + kk * 32, 16, 1024);
+                idesc = make_idesc_f16(64, false, false);
+              } else {
+                ad = make_sdesc_sw128(a_base + kk * 2048, 8192, 1024);
+                bd = make_sdesc_sw128(b_base + kk * 2048, 8192, 1024);
+                idesc = make_idesc_f16(64, true, true);
+              }
+              umma_f16_ss(d_tmem, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[ring.stage]);
+          }
+          __syncwarp();
+          ring.advance(kSkStages);
+        }
+      }
+      if (lane == 0) umma_commit(&acc_full[ab]);
+      __syncwarp();
+      ++it;
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      if constexpr (MODE == kSkRows) {
+        const int4 tt = p.tok_tiles[item >> 1];
+        const int mb = item & 1;
+        if (mb * 128 >= tt.z) continue;
+        const int nrows = min(128, tt.z - mb * 128);
+        const int ab = it & 1;
+        if (!wait_all(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status)) goto done;
+        tc_fence_after();
+        const int m = 32 * q + lane;
+        const int64_t row = tt.y + mb * 128 + m;
+        const float w = (p.out1 && m < nrows) ? __ldg(p.w_perm + row) : 0.f;
+        // output column c = s * sw + j  <-  accumulator column s * 64 + j,
+        // kept when j lies inside a rank block (j % rpad < rank)
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          const int s = c0 / p.sw;
+          const int j0 = c0 - s * p.sw;
+          uint32_t v[16];
+          const bool live = s < p.nseg;
+          if (live) tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128 + s * 64 + j0), v);
+          if (m < nrows) {
+            uint32_t o0[8], o1[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const bool ka = live && ((j0 + 2 * t) % p.rpad) < p.rank;
+              const bool kb = live && ((j0 + 2 * t + 1) % p.rpad) < p.rank;
+              const float a = ka ? p.scale * __uint_as_float(v[2 * t]) : 0.f;
+              const float b = kb ? p.scale * __uint_as_float(v[2 * t + 1]) : 0.f;
+              __half2 h = __floats2half2_rn(a, b);
+              o0[t] = *reinterpret_cast<uint32_t*>(&h);
+              __half2 hw = __floats2half2_rn(w * a, w * b);
+              o1[t] = *reinterpret_cast<uint32_t*>(&hw);
+            }
+            uint4* d0 = reinterpret_cast<uint4*>(p.out0 + row * 64 + c0);
+            d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+            d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+            if (p.out1) {
+              uint4* d1 = reinterpret_cast<uint4*>(p.out1 + row * 64 + c0);
+              d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+              d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        ++it;
+      } else {
+        const GradItem g = grad_item(p, item);
+        const SkJob& jb = p.job[g.job];
+        const int rows = p.offsets[g.e + 1] - p.offsets[g.e];
+        const int pf = 128 * g.fb + 32 * q + lane;  // feature of this lane
+        float D[64];
+        if (rows == 0) {
+          // no rows of this expert in the call: cleared, or kept when accumulating
+          if (!p.accumulate && pf < jb.P)
+            for (int j = 0; j < p.rank; ++j) grad_element(jb, p.rank, p.rpad, g.e, pf, j, D, 0.f, 0, true);
+          continue;
+        }
+        const int ab = it & 1;
+        if (!wait_all(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status)) goto done;
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128), v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) D[j] = __uint_as_float(v[j]);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128 + 32), v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) D[32 + j] = __uint_as_float(v[j]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        ++it;
+        if (pf < jb.P)
+          for (int j = 0; j < p.rank; ++j) grad_element(jb, p.rank, p.rpad, g.e, pf, j, D, p.grad_scale, p.accumulate, false);
+      }
+    }
+  }
+
+done:
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kSkTmemCols);
+}
+
+template <int MODE>
+cudaError_t launch_sk(const SkParams& p, const SkMaps& m, int grid, cudaStream_t stream) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  skinny_kernel<MODE><<<grid, kSkThreads, kSkSmem, stream>>>(p, m);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------- LoRA to FP16
+__global__ void lora_convert_kernel(LoraCvt j0, LoraCvt j1, LoraCvt j2) {
+  const LoraCvt jb = blockIdx.z == 0 ? j0 : (blockIdx.z == 1 ? j1 : j2);
+  if (!jb.dst) return;
+  const int e = blockIdx.y;
+  const int r = jb.rank;
+  const int rows_out = jb.rpad * jb.nsrc;
+  const int c0 = blockIdx.x * 64;
+  if (c0 >= jb.cols) return;
+  uint16_t* dst = jb.dst + (int64_t)e * rows_out * jb.cols;
+  if (!jb.transpose) {
+    for (int idx = threadIdx.x; idx < rows_out * 64; idx += blockDim.x) {
+      const int row = idx >> 6, c = c0 + (idx & 63);
+      if (c >= jb.cols) continue;
+      const int blk = row / jb.rpad, j = row - blk * jb.rpad;
+      float v = 0.f;
+      if (j < r) {
+        const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * jb.cols;
+        v = bf16_bits_to_float(src[c]);
+      }
+      dst[(int64_t)row * jb.cols + c] = f16_bits_rn(v);
+    }
+  } else {
+    __shared__ float tile[64][33];
+    const uint16_t* src = jb.src0 + (int64_t)e * jb.cols * r;  // [cols, r]
+    for (int idx = threadIdx.x; idx < 64 * r; idx += blockDim.x) {
+      const int c = idx / r, j = idx % r;
+      tile[c][j] = (c0 + c < jb.cols) ? bf16_bits_to_float(src[(int64_t)(c0 + c) * r + j]) : 0.f;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 64 * jb.rpad; idx += blockDim.x) {
+      const int j = idx >> 6, c = idx & 63;
+      if (c0 + c < jb.cols) dst[(int64_t)j * jb.cols + c0 + c] = f16_bits_rn(j < r ? tile[c][j] : 0.f);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_skinny(int mode, const SkParams& p, const SkMaps& m, int grid, cudaStream_t stream) {
+  return mode == kSkRows ? launch_sk<kSkRows>(p, m, grid, stream) : launch_sk<kSkGrads>(p, m, grid, stream);
+}
+
+cudaError_t launch_lora_convert(const LoraCvt* jobs, int njobs, int experts, cudaStream_t stream) {
+  LoraCvt z{};
+  LoraCvt j[3] = {njobs > 0 ? jobs[0] : z, njobs > 1 ? jobs[1] : z, njobs > 2 ? jobs[2] : z};
+  int cols = 0;
+  for (int i = 0; i < njobs && i < 3; ++i) cols = j[i].cols > cols ? j[i].cols : cols;
+  if (cols == 0) return cudaSuccess;
+  dim3 grid((cols + 63) / 64, experts, 3);
+  lora_convert_kernel<<<grid, 256, 0, stream>>>(j[0], j[1], j[2]);
+  return cudaGetLastError();
+}
+
+}  // namespace r4
