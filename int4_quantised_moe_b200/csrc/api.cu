@@ -167,6 +167,13 @@ bool map_act(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// the four row-box variants {64, 16/32/64/128} of one fp16 activation matrix
+bool map_act_boxes(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols) {
+  for (int i = 0; i < 4; ++i)
+    if (!map_act(&m[i], base, rows, cols, 16 << i)) return false;
+  return true;
+}
+
 // fp16 per-expert matrices [E, rows, cols]; box {64, rows, 1}, 128-byte swizzle
 bool map_expert_rows(CUtensorMap* m, const uint16_t* base, int64_t E, int64_t rows, int64_t cols) {
   EncodeTiledFn fn = encode_fn();
@@ -318,7 +325,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
   if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 64) ||
-      !map_act(&mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act(&mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
+      !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = I / 64;
   gp.n_main = H / kBlockK;
@@ -355,7 +362,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
   if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
-      !map_act(&mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act(&mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
+      !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = H / 128;
   gp.n_main = I / kBlockK;
@@ -463,7 +470,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
   if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
-      !map_act(&mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act(&mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
+      !map_act_boxes(mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = I / 128;
   gp.n_main = H / kBlockK;
@@ -505,7 +512,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
   if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
-      !map_act(&mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act(&mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
+      !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = H / 128;
   gp.n_main = 2 * I / kBlockK;

@@ -158,9 +158,9 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, 
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tq0,
-                const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap tb,
-                const __grid_constant__ CUtensorMap tbx) {
+    gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  const CUtensorMap& tq0 = maps.q0;
+  const CUtensorMap& tq1 = maps.q1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + kOffA;
@@ -205,8 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tq0);
     tma_prefetch_desc(&tq1);
-    tma_prefetch_desc(&tb);
-    tma_prefetch_desc(&tbx);
+    for (int i = 0; i < 4; ++i) {
+      tma_prefetch_desc(&maps.b[i]);
+      tma_prefetch_desc(&maps.bx[i]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -266,11 +268,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t* bar = &b_full[ring.stage];
           uint8_t* dst = sB + ring.stage * kBBytes;
           mbar_expect_tx(bar, nbox * 2048);
-          for (int j = 0; j < nbox; ++j) {
-            if (s < n_main)
-              tma_load_2d(dst + j * 2048, &tb, bar, s * kBlockK, tt.y + 16 * j);
-            else
-              tma_load_2d(dst + j * 2048, &tbx, bar, 0, tt.y + 16 * j);
+          // the tile's rows in at most a few boxes of 128/64/32/16 rows
+          int row = 0;
+          for (int lvl = 3; lvl >= 0; --lvl) {
+            const int h = 16 << lvl;
+            while (16 * nbox - row >= h) {
+              if (s < n_main)
+                tma_load_2d(dst + row * 128, &maps.b[lvl], bar, s * kBlockK, tt.y + row);
+              else
+                tma_load_2d(dst + row * 128, &maps.bx[lvl], bar, 0, tt.y + row);
+              row += h;
+            }
           }
         }
         __syncwarp();
@@ -444,13 +452,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e = tt.x;
       uint32_t lora_w[16];
       lora_values<MODE>(p, e, rb, dt, lora_w);
-      uint16_t scale_next = n_main > 0 ? load_scale<MODE>(p, e, rb, 0, dt) : 0;
+      // group scales of the next four stages, loaded well before their use
+      uint16_t sq0 = n_main > 0 ? load_scale<MODE>(p, e, rb, 0, dt) : 0;
+      uint16_t sq1 = n_main > 1 ? load_scale<MODE>(p, e, rb, 1, dt) : 0;
+      uint16_t sq2 = n_main > 2 ? load_scale<MODE>(p, e, rb, 2, dt) : 0;
+      uint16_t sq3 = n_main > 3 ? load_scale<MODE>(p, e, rb, 3, dt) : 0;
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
         uint8_t* A = sA + ra.stage * kABytes;
         if (s < n_main) {
-          const uint16_t scale = scale_next;
-          if (s + 1 < n_main) scale_next = load_scale<MODE>(p, e, rb, s + 1, dt);
+          const uint16_t scale = sq0;
+          sq0 = sq1;
+          sq1 = sq2;
+          sq2 = sq3;
+          sq3 = (s + 4 < n_main) ? load_scale<MODE>(p, e, rb, s + 4, dt) : 0;
           if (!wait_all(&p_full[rp.stage], rp.phase, abort_flag, status)) goto done;
           const uint4 qv = *reinterpret_cast<const uint4*>(sP + rp.stage * kPBytes + dt * 16);
           __syncwarp();
@@ -491,7 +506,7 @@ cudaError_t launch_mode(const GemmParams& p, const GemmMaps& m, int grid, cudaSt
     if (err != cudaSuccess) return err;
     attr_set = true;
   }
-  gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, stream>>>(p, m.q0, m.q1, m.b, m.bx);
+  gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, stream>>>(p, m);
   return cudaGetLastError();
 }
 

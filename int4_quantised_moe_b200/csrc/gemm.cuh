@@ -15,9 +15,9 @@ enum GemmMode : int {
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
 constexpr int kRowsM = 128;        // UMMA M
-constexpr int kStagesA = 2;        // decoded FP16 A tiles (16 KB each)
+constexpr int kStagesA = 3;        // decoded FP16 A tiles (16 KB each)
 constexpr int kStagesB = 4;        // TMA-loaded B tiles (32 KB each)
-constexpr int kStagesP = 8;        // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kStagesP = 6;        // TMA-loaded packed int4 tiles (4 KB each)
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
@@ -58,10 +58,10 @@ struct GemmParams {
 };
 
 struct GemmMaps {
-  CUtensorMap q0;  // packed projection 0: 3D uint8 {stored K bytes, stored rows, E}
-  CUtensorMap q1;  // packed projection 1
-  CUtensorMap b;   // B main: 2D fp16 {K, rows}, 128B swizzle, box {64, 16}
-  CUtensorMap bx;  // B LoRA: 2D fp16 {64, rows}, 128B swizzle, box {64, 16}
+  CUtensorMap q0;     // packed projection 0: 3D uint8 {stored K bytes, stored rows, E}
+  CUtensorMap q1;     // packed projection 1
+  CUtensorMap b[4];   // B main: 2D fp16 {K, rows}, 128B swizzle, boxes {64, 16 << i}
+  CUtensorMap bx[4];  // B LoRA: 2D fp16 {64, rows}, 128B swizzle, boxes {64, 16 << i}
 };
 
 size_t gemm_smem_bytes();
