@@ -63,7 +63,7 @@ Layout make_layout(const rawint4_moe_cfg& c) {
   L.gdw = take(rows * kLoraPad * 2);
   L.dgu = take(rows * 2 * I * 2);
   L.gb = take(rows * kLoraPad * 2);
-  L.dpart = take(rows * (I / 128) * 4);
+  L.dpart = take(rows * ((I + 255) / 256) * 4);
   L.rpad = (c.rank + 15) / 16 * 16;
   const int64_t rp = L.rpad;
   L.gu16 = take(E * 2 * rp * H * 2);
@@ -140,7 +140,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1}, no swizzle
+// packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1};
+// 128-byte swizzling for the 128-byte-wide boxes the transposed modes read
 bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -149,8 +150,8 @@ bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, in
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // fp16 row-major [rows, cols]; box {64, box_rows}, 128-byte swizzle (UMMA
@@ -324,10 +325,11 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 128) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 128) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
-  gp.n_rowblk = I / 64;
+  gp.n_rowblk = I / 128;
+  gp.feat = I;
   gp.n_main = H / kBlockK;
   gp.s0 = base->gate_s;
   gp.s1 = base->up_s;
@@ -361,10 +363,11 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 256) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 256) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
-  gp.n_rowblk = H / 128;
+  gp.n_rowblk = (H + 255) / 256;
+  gp.feat = H;
   gp.n_main = I / kBlockK;
   gp.s0 = gp.s1 = base->down_s;
   gp.s_expert = (int64_t)H * (I / 32);
@@ -469,10 +472,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 128, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
-  gp.n_rowblk = I / 128;
+  gp.n_rowblk = (I + 255) / 256;
+  gp.feat = I;
   gp.n_main = H / kBlockK;
   gp.s0 = gp.s1 = base->down_s;
   gp.s_expert = (int64_t)H * (I / 32);
@@ -511,10 +515,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 128, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
-  gp.n_rowblk = H / 128;
+  gp.n_rowblk = (H + 255) / 256;
+  gp.feat = H;
   gp.n_main = 2 * I / kBlockK;
   gp.s0 = base->gate_s;
   gp.s1 = base->up_s;
@@ -540,7 +545,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
   if (grad_route) {
     R4_PROF("combine_route", st);
-    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), I / 128, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ,
+    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), (I + 255) / 256, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ,
                                 st));
   }
 

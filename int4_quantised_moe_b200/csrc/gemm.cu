@@ -1,18 +1,26 @@
 // Dequant-fused grouped GEMMs of the routed RAWINT4 MoE-LoRA layer on
 // sm_100a tensor cores (tcgen05, TMEM accumulators, TMA-fed operands).
 //
-// One persistent CTA per SM walks (token tile, output row block) work items.
-// A token tile is up to 256 permuted rows of one expert; a row block is 128
-// output features (64 gate + 64 up features in the gate/up mode). Warp roles:
+// One persistent CTA per SM walks (token tile, feature block) work items. A
+// token tile is up to 256 permuted rows of one expert; a feature block is 256
+// weight rows (gate/up: the same 128 features of gate and of up). Each
+// K-stage issues two M=128 UMMAs (weight rows 0-127 and 128-255) on the same
+// B tile, so every activation tile read from L2 feeds 256 weight rows.
+// Warp roles:
 //   warp 0      TMA producer of packed int4 weight tiles   (ring of kStagesP)
 //   warp 2      TMA producer of B tiles (activations)      (ring of kStagesB)
 //   warps 8-15  decoders: int4 -> fp16 into the UMMA A layout (ring of kStagesA)
 //   warp 1      UMMA issuer (one elected lane) and TMEM owner
 //   warps 4-7   epilogue: TMEM -> registers -> fused math -> global
+// TMEM (512 columns) holds two halves of 256 columns. A tile of at most 128
+// tokens keeps both of its accumulators in one half, so consecutive narrow
+// items alternate halves and the epilogue of one overlaps the MMAs of the
+// next; a wider tile takes both halves.
+//
 // The LoRA side product of each projection runs as one extra 64-wide
-// reduction stage in the same accumulator: its A operand is the LoRA tensor
-// of the expert (copied/converted by the decoders), its B operand the
-// precomputed c-scaled rank-r side matrix of the tokens.
+// reduction stage in the same accumulators: its A operand is the LoRA tensor
+// of the expert (loaded into registers at the start of the item and stored
+// by the decoders), its B operand the precomputed c-scaled rank-r side matrix.
 //
 // The backward modes read the packed base along its stored output dimension
 // (transpose-free dX, rawint4_sft_reference.py transpose_free_rawint4_dx):
@@ -24,9 +32,10 @@ namespace r4 {
 
 namespace {
 
-constexpr int kABytes = kRowsM * kBlockK * 2;  // 16 KB
+constexpr int kABytes = kRowsM * kBlockK * 2;  // 32 KB
+constexpr int kAHalf = kABytes / 2;            // weight rows 128-255 start here (both layouts)
 constexpr int kBBytes = 256 * kBlockK * 2;     // 32 KB
-constexpr int kPBytes = kRowsM * kBlockK / 2;  // 4 KB
+constexpr int kPBytes = kRowsM * kBlockK / 2;  // 8 KB
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStagesA * kABytes;
 constexpr int kOffP = kOffB + kStagesB * kBBytes;
@@ -49,6 +58,18 @@ __device__ __forceinline__ int kext_steps(int rpad) {
   return kext / 16;
 }
 
+// First output feature of block rb.
+template <int MODE>
+__device__ __forceinline__ int block_f0(int rb) {
+  return MODE == kModeGateUp ? rb * 128 : rb * 256;
+}
+
+// Whether block rb has its second 128-row half (always, for gate/up).
+template <int MODE>
+__device__ __forceinline__ bool block_two(const GemmParams& p, int rb) {
+  return MODE == kModeGateUp || block_f0<MODE>(rb) + 128 < p.feat;
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
 // 128B-swizzled block whose rows are 128 bytes and whose 8-row atoms are
 // 1024 bytes apart.
@@ -56,42 +77,68 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// MN-major decode: thread dt owns K row kr of the 64 features [64 qq, +64),
+// which form one 8 KB MN block of the A tile. Each group of 8 consecutive
+// lanes takes 8 consecutive K rows of one block, so its 16-byte stores (and
+// its reads of the swizzled packed tile) hit 8 distinct bank groups.
+__device__ __forceinline__ int mn_kr(int dt) { return 8 * (dt >> 5) + (dt & 7); }
+__device__ __forceinline__ int mn_qq(int dt) { return (dt >> 3) & 3; }
+
+// Offset of output chunk c (0..7, 8 fp16 each) of decoder thread dt in the A
+// tile. K-major: thread dt owns weight row dt (all 64 K of the stage).
 template <int MODE>
-__device__ __forceinline__ uint32_t a_chunk_off(int dt, int j) {
+__device__ __forceinline__ uint32_t a_chunk_off(int dt, int c) {
   if constexpr (!kAMnMajor<MODE>) {
-    const int m = dt >> 1, half = dt & 1;
-    return sw128_off(m, 4 * half + j);
+    return sw128_off(dt, c);
   } else {
-    const int kr = dt >> 2, qq = dt & 3;
-    return (uint32_t)((qq >> 1) * 8192) + sw128_off(kr, 4 * (qq & 1) + j);
+    return (uint32_t)(mn_qq(dt) * 8192) + sw128_off(mn_kr(dt), c);
   }
 }
 
+// The 32 packed bytes decoder thread dt decodes at one stage: two groups of
+// 32 weights (q0 first). K-major tiles hold row dt at dt * 32, and the two
+// halves are read in an order that spreads each 8-lane group over all bank
+// groups. MN-major tiles are loaded with 128-byte swizzling.
 template <int MODE>
-__device__ __forceinline__ uint16_t load_scale(const GemmParams& p, int e, int rb, int s, int dt) {
-  if constexpr (MODE == kModeGateUp) {
-    const int m = dt >> 1, half = dt & 1;
-    const uint16_t* sp = (m < 64) ? p.s0 : p.s1;
-    const int row = rb * 64 + (m & 63);
-    return __ldg(sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + 2 * s + half);
-  } else if constexpr (MODE == kModeDown) {
-    const int m = dt >> 1, half = dt & 1;
-    const int row = rb * 128 + m;
-    return __ldg(p.s0 + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + 2 * s + half);
-  } else if constexpr (MODE == kModeDownT) {
-    const int kr = dt >> 2, qq = dt & 3;
-    const int row = s * kBlockK + kr;
-    return __ldg(p.s0 + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + rb * 4 + qq);
+__device__ __forceinline__ void packed_pair(const uint8_t* P, int dt, uint4& q0, uint4& q1) {
+  if constexpr (!kAMnMajor<MODE>) {
+    const int sw = (dt >> 2) & 1;
+    const uint4 a = *reinterpret_cast<const uint4*>(P + dt * 32 + sw * 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(P + dt * 32 + (sw ^ 1) * 16);
+    q0 = sw ? b : a;
+    q1 = sw ? a : b;
   } else {
-    const int kr = dt >> 2, qq = dt & 3;
+    const int kr = mn_kr(dt), qq = mn_qq(dt);
+    q0 = *reinterpret_cast<const uint4*>(P + sw128_off(kr, 2 * qq));
+    q1 = *reinterpret_cast<const uint4*>(P + sw128_off(kr, 2 * qq + 1));
+  }
+}
+
+// The two group scales decoder thread dt needs at K-stage s, as bf16 bits
+// (first group low, second high); 0 past the mode's features.
+template <int MODE>
+__device__ __forceinline__ uint32_t load_scales(const GemmParams& p, int e, int rb, int s, int dt) {
+  const int f0 = block_f0<MODE>(rb);
+  const uint16_t* sp = p.s0;
+  int64_t idx;
+  if constexpr (MODE == kModeGateUp) {
+    sp = dt < 128 ? p.s0 : p.s1;
+    idx = (int64_t)(f0 + (dt & 127)) * p.s_row + 2 * s;
+  } else if constexpr (MODE == kModeDown) {
+    if (f0 + dt >= p.feat) return 0u;
+    idx = (int64_t)(f0 + dt) * p.s_row + 2 * s;
+  } else {
+    const int kr = mn_kr(dt), qq = mn_qq(dt);
+    if (f0 + 64 * qq >= p.feat) return 0u;
     int row = s * kBlockK + kr;
-    const uint16_t* sp = p.s0;
-    if (row >= p.stored_rows) {
+    if (MODE == kModeGateUpT && row >= p.stored_rows) {
       row -= p.stored_rows;
       sp = p.s1;
     }
-    return __ldg(sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + rb * 4 + qq);
+    idx = (int64_t)row * p.s_row + (f0 + 64 * qq) / 32;
   }
+  sp += (int64_t)e * p.s_expert + idx;
+  return (uint32_t)__ldg(sp) | ((uint32_t)__ldg(sp + 1) << 16);
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
@@ -99,50 +146,50 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// This thread's 32 values of the A tile of the LoRA reduction stage, as 16
-// fp16 pairs in the same order the decode produces (see a_chunk_off).
+// This thread's 64 values of the A tile of the LoRA reduction stage, as 32
+// fp16 pairs in decode order (chunk c = words 4c..4c+3, see a_chunk_off).
 // Loaded at the start of a work item, long before the stage is stored: a
-// decoder warp that stores operand data right after long-latency global loads
+// decoder warp that stored operand data right after long-latency global loads
 // at the tail of a work item produced corrupted rows in earlier builds, and
 // the early load also takes that latency off the critical path.
 template <int MODE>
-__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, int dt, uint32_t (&w)[16]) {
+__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, int dt, uint32_t (&w)[32]) {
   const int r = p.rank;
+  const int f0 = block_f0<MODE>(rb);
   if constexpr (!kAMnMajor<MODE>) {
-    // A[m, j] with j in [32*half, 32*half + 32): LoRA B rows (K-major, rank contiguous)
-    const int m = dt >> 1, half = dt & 1;
-    const uint16_t* src;
-    int jlo;  // first reduction column that holds this row's values
+    // A[m, j], j in [0, 64): LoRA B rows (rank contiguous)
+    const uint16_t* src = nullptr;
+    int jlo = 0;  // first reduction column holding this row's values
     if constexpr (MODE == kModeGateUp) {
-      const bool up = m >= 64;
-      src = (up ? p.lx1 : p.lx0) + (int64_t)e * p.lx_expert + (int64_t)(rb * 64 + (m & 63)) * p.lx_ld;
-      jlo = up ? p.rpad : 0;
+      src = (dt < 128 ? p.lx0 : p.lx1) + (int64_t)e * p.lx_expert + (int64_t)(f0 + (dt & 127)) * p.lx_ld;
+      jlo = dt < 128 ? 0 : p.rpad;
     } else {
-      src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)(rb * 128 + m) * p.lx_ld;
-      jlo = 0;
+      if (f0 + dt < p.feat) src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)(f0 + dt) * p.lx_ld;
     }
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
+    for (int t = 0; t < 32; ++t) {
       float v[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int jj = 32 * half + 2 * t + u - jlo;
-        v[u] = (jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
+        const int jj = 2 * t + u - jlo;
+        v[u] = (src != nullptr && jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
       }
       w[t] = pack_h2(v[0], v[1]);
     }
   } else {
-    // A[m, kr] with m in [32*qq, 32*qq + 32): LoRA A rows (MN-major, feature contiguous)
-    const int kr = dt >> 2, qq = dt & 3;
+    // A[m, kr], m in [64 qq, 64 qq + 64): LoRA A rows (feature contiguous)
+    const int kr = mn_kr(dt), qq = mn_qq(dt);
     const uint16_t* src = nullptr;
-    if (kr < r)
-      src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + rb * 128 + 32 * qq;
-    else if (MODE == kModeGateUpT && kr >= p.rpad && kr < p.rpad + r)
-      src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - p.rpad) * p.lx_ld + rb * 128 + 32 * qq;
-    if (src) {
+    if (f0 + 64 * qq < p.feat) {
+      if (kr < r)
+        src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + f0 + 64 * qq;
+      else if (MODE == kModeGateUpT && kr >= p.rpad && kr < p.rpad + r)
+        src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - p.rpad) * p.lx_ld + f0 + 64 * qq;
+    }
+    if (src != nullptr) {
       const uint4* s4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const uint4 b = __ldg(s4 + c);
         const uint32_t in[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -151,10 +198,27 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, 
       }
     } else {
 #pragma unroll
-      for (int t = 0; t < 16; ++t) w[t] = 0u;
+      for (int t = 0; t < 32; ++t) w[t] = 0u;
     }
   }
 }
+
+// Which TMEM half (or both) an item's accumulators occupy. The MMA issuer and
+// the epilogue step identical copies through the same item sequence.
+struct AccTrack {
+  uint32_t uses[2] = {0u, 0u};  // completed items per half (phase parity source)
+  int next = 0;                 // half the next narrow item takes
+  __device__ __forceinline__ void retire(bool wide) {
+    if (wide) {
+      ++uses[0];
+      ++uses[1];
+      next = 0;
+    } else {
+      ++uses[next];
+      next ^= 1;
+    }
+  }
+};
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -229,27 +293,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     Ring ring;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
-      const int rb = tile % n_rowblk;
+      const int f0 = block_f0<MODE>(tile % n_rowblk);
       const int e = tt.x;
       for (int s = 0; s < n_main; ++s) {
         if (!wait_all(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
         if (lane == 0) {
           uint64_t* bar = &p_full[ring.stage];
           uint8_t* dst = sP + ring.stage * kPBytes;
+          // every box is counted in full, also where it reaches past the
+          // tensor (zero-filled rows of a half block)
           mbar_expect_tx(bar, kPBytes);
           if constexpr (MODE == kModeGateUp) {
-            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), rb * 64, e);
-            tma_load_3d(dst + kPBytes / 2, &tq1, bar, s * (kBlockK / 2), rb * 64, e);
+            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), f0, e);
+            tma_load_3d(dst + kPBytes / 2, &tq1, bar, s * (kBlockK / 2), f0, e);
           } else if constexpr (MODE == kModeDown) {
-            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), rb * 128, e);
+            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), f0, e);
           } else if constexpr (MODE == kModeDownT) {
-            tma_load_3d(dst, &tq0, bar, rb * 64, s * kBlockK, e);
+            tma_load_3d(dst, &tq0, bar, f0 / 2, s * kBlockK, e);
           } else {
             const int k0 = s * kBlockK;
             if (k0 < p.stored_rows)
-              tma_load_3d(dst, &tq0, bar, rb * 64, k0, e);
+              tma_load_3d(dst, &tq0, bar, f0 / 2, k0, e);
             else
-              tma_load_3d(dst, &tq1, bar, rb * 64, k0 - p.stored_rows, e);
+              tma_load_3d(dst, &tq1, bar, f0 / 2, k0 - p.stored_rows, e);
           }
         }
         __syncwarp();
@@ -288,17 +354,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     Ring ra, rbr;
-    int it = 0;
+    AccTrack acc;
     const int ksteps_x = kext_steps<MODE>(p.rpad);
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const bool two = block_two<MODE>(p, tile % n_rowblk);
       const int n_mma = (tt.z + 15) & ~15;
+      const bool wide = n_mma > 128;
       const uint32_t idesc = make_idesc_f16((uint32_t)n_mma, kAMnMajor<MODE>, false);
-      const int ab = it & 1;
-      const uint32_t acc_ph = (uint32_t)(it >> 1) & 1u;
-      if (!wait_all(&acc_empty[ab], acc_ph ^ 1u, abort_flag, status)) goto done;
+      uint32_t d0;
+      if (wide) {
+        if (!wait_all(&acc_empty[0], (acc.uses[0] & 1u) ^ 1u, abort_flag, status)) goto done;
+        if (!wait_all(&acc_empty[1], (acc.uses[1] & 1u) ^ 1u, abort_flag, status)) goto done;
+        d0 = tmem;
+      } else {
+        if (!wait_all(&acc_empty[acc.next], (acc.uses[acc.next] & 1u) ^ 1u, abort_flag, status)) goto done;
+        d0 = tmem + (uint32_t)(acc.next * 256);
+      }
+      const uint32_t d1 = d0 + (wide ? 256u : 128u);
       tc_fence_after();
-      const uint32_t d_tmem = tmem + (uint32_t)(ab * 256);
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_full[ra.stage], ra.phase, abort_flag, status)) goto done;
         if (!wait_all(&b_full[rbr.stage], rbr.phase, abort_flag, status)) goto done;
@@ -308,13 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(sB + rbr.stage * kBBytes);
           const int ksteps = (s < n_main) ? (kBlockK / 16) : ksteps_x;
           for (int kk = 0; kk < ksteps; ++kk) {
-            uint64_t adesc;
-            if constexpr (kAMnMajor<MODE>)
-              adesc = make_sdesc_sw128(a_base + kk * 2048, 8192, 1024);
-            else
-              adesc = make_sdesc_sw128(a_base + kk * 32, 16, 1024);
+            const uint32_t a_off = kAMnMajor<MODE> ? (uint32_t)kk * 2048u : (uint32_t)kk * 32u;
+            const uint32_t lbo = kAMnMajor<MODE> ? 8192u : 16u;
+            const uint64_t a0 = make_sdesc_sw128(a_base + a_off, lbo, 1024);
+            const uint64_t a1 = make_sdesc_sw128(a_base + kAHalf + a_off, lbo, 1024);
             const uint64_t bdesc = make_sdesc_sw128(b_base + kk * 32, 16, 1024);
-            umma_f16_ss(d_tmem, adesc, bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t accum = (s > 0 || kk > 0) ? 1u : 0u;
+            umma_f16_ss(d0, a0, bdesc, idesc, accum);
+            if (two) umma_f16_ss(d1, a1, bdesc, idesc, accum);
           }
           umma_commit(&a_empty[ra.stage]);
           umma_commit(&b_empty[rbr.stage]);
@@ -323,103 +398,147 @@ __global__ void __launch_bounds__(kThreads, 1)
         ra.advance(kStagesA);
         rbr.advance(kStagesB);
       }
-      if (lane == 0) umma_commit(&acc_full[ab]);
+      if (lane == 0) {
+        if (wide) {
+          umma_commit(&acc_full[0]);
+          umma_commit(&acc_full[1]);
+        } else {
+          umma_commit(&acc_full[acc.next]);
+        }
+      }
       __syncwarp();
+      acc.retire(wide);
     }
   } else if (warp >= kEpiWarp0 && warp < kDecWarp0) {
     // --------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+    const int q = warp & 3;       // TMEM lane quarter this warp may access
+    const int m = 32 * q + lane;  // accumulator row of this thread in each MMA
+    AccTrack acc;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int rb = tile % n_rowblk;
+      const bool two = block_two<MODE>(p, rb);
+      const int f0 = block_f0<MODE>(rb);
       const int n_rows = tt.z;
       const int p0 = tt.y;
       const int n_mma = (n_rows + 15) & ~15;
-      const int ab = it & 1;
-      const uint32_t acc_ph = (uint32_t)(it >> 1) & 1u;
-      if (!wait_all(&acc_full[ab], acc_ph, abort_flag, status)) goto done;
+      const bool wide = n_mma > 128;
+      uint32_t d0;
+      if (wide) {
+        if (!wait_all(&acc_full[0], acc.uses[0] & 1u, abort_flag, status)) goto done;
+        if (!wait_all(&acc_full[1], acc.uses[1] & 1u, abort_flag, status)) goto done;
+        d0 = tmem;
+      } else {
+        if (!wait_all(&acc_full[acc.next], acc.uses[acc.next] & 1u, abort_flag, status)) goto done;
+        d0 = tmem + (uint32_t)(acc.next * 256);
+      }
+      const uint32_t d1 = d0 + (wide ? 256u : 128u);
       tc_fence_after();
+      const uint32_t lane_base = (uint32_t)(32 * q) << 16;
       for (int c0 = 0; c0 < n_mma; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 256 + c0), v);
+        uint32_t v0[32], v1[32];
+        if constexpr (MODE != kModeDownT) {
+          tmem_ld32(d0 + lane_base + (uint32_t)c0, v0);
+          if (two) {
+            tmem_ld32(d1 + lane_base + (uint32_t)c0, v1);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v1[c] = 0u;
+          }
+        }
         if constexpr (MODE == kModeGateUp) {
-          float* xch = epi + (q & 1) * 32 * 33;
-          if (q >= 2) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) xch[lane * 33 + c] = __uint_as_float(v[c]);
-          }
-          named_bar_sync(1 + (q & 1), 64);
-          if (q < 2) {
-            const int i = rb * 64 + 32 * q + lane;
-            const float L = p.limit;
-            bool overflow = false;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int n = c0 + c;
-              if (n < n_rows) {
-                const int64_t o = (int64_t)(p0 + n) * p.ld_out + i;
-                const float g = __uint_as_float(v[c]);
-                const float u = xch[lane * 33 + c];
-                const float gc = L > 0.f ? fminf(g, L) : g;
-                const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
-                const float h = gc * sigmoid_clamped(gc) * uc;
-                const __half hh = __float2half_rn(h);
-                overflow |= __hisinf(hh) != 0;
-                p.out_a[o] = g;
-                p.out_b[o] = u;
-                p.out_h[o] = *reinterpret_cast<const uint16_t*>(&hh);
-              }
-            }
-            if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
-          }
-          named_bar_sync(1 + (q & 1), 64);
-        } else if constexpr (MODE == kModeDown || MODE == kModeGateUpT) {
-          const int m = rb * 128 + 32 * q + lane;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int n = c0 + c;
-            if (n < n_rows) {
-              const int64_t row = p0 + n;
-              float val = __uint_as_float(v[c]);
-              if constexpr (MODE == kModeDown) val *= __ldg(p.w_perm + row);
-              p.out_a[row * p.ld_out + m] = val;
-            }
-          }
-        } else {  // kModeDownT
-          const int i = rb * 128 + 32 * q + lane;
+          // row m of the first MMA is gate feature f0 + m, of the second up feature f0 + m
+          const int i = f0 + m;
           const float L = p.limit;
-          float* red = epi + q * 32 * 33;
-          float* red2 = epi + 4 * 32 * 33;
           bool overflow = false;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int n = c0 + c;
-            float prod = 0.f;
             if (n < n_rows) {
-              const int64_t row = p0 + n;
-              const float acc = __uint_as_float(v[c]);
-              const float w = __ldg(p.w_perm + row);
-              const float g = p.in_g[row * p.ld_out + i];
-              const float u = p.in_u[row * p.ld_out + i];
+              const int64_t o = (int64_t)(p0 + n) * p.ld_out + i;
+              const float g = __uint_as_float(v0[c]);
+              const float u = __uint_as_float(v1[c]);
               const float gc = L > 0.f ? fminf(g, L) : g;
               const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
-              const bool pass_g = !(L > 0.f) || g <= L;
-              const bool pass_u = !(L > 0.f) || (u >= -L && u <= L);
-              const float sg = sigmoid_clamped(gc);
-              const float silu = gc * sg;
-              const float dsilu = sg * (1.0f + gc * (1.0f - sg));
-              const float dh = w * acc;
-              const float dg = pass_g ? dh * uc * dsilu : 0.f;
-              const float du = pass_u ? dh * silu : 0.f;
-              const __half hg = __float2half_rn(dg);
-              const __half hu = __float2half_rn(du);
-              overflow |= (__hisinf(hg) | __hisinf(hu)) != 0;
-              p.out_h[row * (2 * p.inter) + i] = *reinterpret_cast<const uint16_t*>(&hg);
-              p.out_h[row * (2 * p.inter) + p.inter + i] = *reinterpret_cast<const uint16_t*>(&hu);
-              prod = acc * silu * uc;
+              const float h = gc * sigmoid_clamped(gc) * uc;
+              const __half hh = __float2half_rn(h);
+              overflow |= __hisinf(hh) != 0;
+              p.out_a[o] = g;
+              p.out_b[o] = u;
+              p.out_h[o] = *reinterpret_cast<const uint16_t*>(&hh);
             }
-            red[lane * 33 + c] = prod;
+          }
+          if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
+        } else if constexpr (MODE == kModeDown || MODE == kModeGateUpT) {
+          float wl = 1.0f;
+          if constexpr (MODE == kModeDown) wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int n = c0 + c;
+            const float w = __shfl_sync(0xffffffffu, wl, c);
+            if (n < n_rows) {
+              const int64_t row = p0 + n;
+              float a = __uint_as_float(v0[c]);
+              float b = __uint_as_float(v1[c]);
+              if constexpr (MODE == kModeDown) {
+                a *= w;
+                b *= w;
+              }
+              p.out_a[row * p.ld_out + f0 + m] = a;
+              if (two) p.out_a[row * p.ld_out + f0 + 128 + m] = b;
+            }
+          }
+        } else {  // kModeDownT
+          // Per half: the accumulators of 32 tokens, then the saved G/U of
+          // 8 tokens at a time, loaded together ahead of their use.
+          const float L = p.limit;
+          float* red = epi + q * 32 * 33;
+          float* red2 = epi + 4 * 32 * 33;
+          bool overflow = false;
+          const float wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
+          for (int hf = 0; hf < (two ? 2 : 1); ++hf) {
+            tmem_ld32((hf ? d1 : d0) + lane_base + (uint32_t)c0, v0);
+            const int i = f0 + 128 * hf + m;
+#pragma unroll
+            for (int cb = 0; cb < 32; cb += 8) {
+              float g8[8], u8[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int64_t row = p0 + min(c0 + cb + c, n_rows - 1);
+                g8[c] = __ldg(p.in_g + row * p.ld_out + i);
+                u8[c] = __ldg(p.in_u + row * p.ld_out + i);
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int n = c0 + cb + c;
+                const float w = __shfl_sync(0xffffffffu, wl, cb + c);
+                float prod = 0.f;
+                if (n < n_rows) {
+                  const int64_t row = p0 + n;
+                  const float acc_v = __uint_as_float(v0[cb + c]);
+                  const float g = g8[c];
+                  const float u = u8[c];
+                  const float gc = L > 0.f ? fminf(g, L) : g;
+                  const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
+                  const bool pass_g = !(L > 0.f) || g <= L;
+                  const bool pass_u = !(L > 0.f) || (u >= -L && u <= L);
+                  const float sg = sigmoid_clamped(gc);
+                  const float silu = gc * sg;
+                  const float dsilu = sg * (1.0f + gc * (1.0f - sg));
+                  const float dh = w * acc_v;
+                  const float dg = pass_g ? dh * uc * dsilu : 0.f;
+                  const float du = pass_u ? dh * silu : 0.f;
+                  const __half hg = __float2half_rn(dg);
+                  const __half hu = __float2half_rn(du);
+                  overflow |= (__hisinf(hg) | __hisinf(hu)) != 0;
+                  p.out_h[row * (2 * p.inter) + i] = *reinterpret_cast<const uint16_t*>(&hg);
+                  p.out_h[row * (2 * p.inter) + p.inter + i] = *reinterpret_cast<const uint16_t*>(&hu);
+                  prod = acc_v * silu * uc;
+                }
+                float* slot = red + lane * 33 + cb + c;
+                *slot = hf ? *slot + prod : prod;
+              }
+            }
           }
           if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
           __syncwarp();
@@ -440,7 +559,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) {
+        if (wide) {
+          mbar_arrive(&acc_empty[0]);
+          mbar_arrive(&acc_empty[1]);
+        } else {
+          mbar_arrive(&acc_empty[acc.next]);
+        }
+      }
+      acc.retire(wide);
     }
   } else if (warp >= kDecWarp0) {
     // --------------------------------------------------------------- decoders
@@ -450,38 +577,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int rb = tile % n_rowblk;
       const int e = tt.x;
-      uint32_t lora_w[16];
+      uint32_t lora_w[32];
       lora_values<MODE>(p, e, rb, dt, lora_w);
       // group scales of the next four stages, loaded well before their use
-      uint16_t sq0 = n_main > 0 ? load_scale<MODE>(p, e, rb, 0, dt) : 0;
-      uint16_t sq1 = n_main > 1 ? load_scale<MODE>(p, e, rb, 1, dt) : 0;
-      uint16_t sq2 = n_main > 2 ? load_scale<MODE>(p, e, rb, 2, dt) : 0;
-      uint16_t sq3 = n_main > 3 ? load_scale<MODE>(p, e, rb, 3, dt) : 0;
+      uint32_t sq0 = n_main > 0 ? load_scales<MODE>(p, e, rb, 0, dt) : 0u;
+      uint32_t sq1 = n_main > 1 ? load_scales<MODE>(p, e, rb, 1, dt) : 0u;
+      uint32_t sq2 = n_main > 2 ? load_scales<MODE>(p, e, rb, 2, dt) : 0u;
+      uint32_t sq3 = n_main > 3 ? load_scales<MODE>(p, e, rb, 3, dt) : 0u;
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
         uint8_t* A = sA + ra.stage * kABytes;
         if (s < n_main) {
-          const uint16_t scale = sq0;
+          const uint32_t sc = sq0;
           sq0 = sq1;
           sq1 = sq2;
           sq2 = sq3;
-          sq3 = (s + 4 < n_main) ? load_scale<MODE>(p, e, rb, s + 4, dt) : 0;
+          sq3 = (s + 4 < n_main) ? load_scales<MODE>(p, e, rb, s + 4, dt) : 0u;
           if (!wait_all(&p_full[rp.stage], rp.phase, abort_flag, status)) goto done;
-          const uint4 qv = *reinterpret_cast<const uint4*>(sP + rp.stage * kPBytes + dt * 16);
+          uint4 q0, q1;
+          packed_pair<MODE>(sP + rp.stage * kPBytes, dt, q0, q1);
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
           rp.advance(kStagesP);
-          uint32_t w[16];
-          decode_group32(qv, bf16_scale_to_h2(scale), w);
+          uint32_t w0[16], w1[16];
+          decode_group32(q0, bf16_scale_to_h2((uint16_t)(sc & 0xFFFFu)), w0);
+          decode_group32(q1, bf16_scale_to_h2((uint16_t)(sc >> 16)), w1);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
-                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          for (int c = 0; c < 4; ++c) {
+            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, c)) =
+                make_uint4(w0[4 * c], w0[4 * c + 1], w0[4 * c + 2], w0[4 * c + 3]);
+            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, 4 + c)) =
+                make_uint4(w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+          }
         } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
-                make_uint4(lora_w[4 * j], lora_w[4 * j + 1], lora_w[4 * j + 2], lora_w[4 * j + 3]);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, c)) =
+                make_uint4(lora_w[4 * c], lora_w[4 * c + 1], lora_w[4 * c + 2], lora_w[4 * c + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

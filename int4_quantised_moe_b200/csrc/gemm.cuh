@@ -3,9 +3,10 @@
 
 namespace r4 {
 
-// The four dequant-fused grouped GEMMs of the layer. All put 128 weight rows
-// (output features) on the UMMA M side and up to 256 permuted tokens of one
-// expert on the N side: D[m, n] = sum_k A[m, k] * B[n, k].
+// The four dequant-fused grouped GEMMs of the layer. A work item puts 256
+// weight rows (output features; gate/up: 128 features of each) on the UMMA M
+// side as two M=128 MMAs that share every B tile, and up to 256 permuted
+// tokens of one expert on the N side: D[m, n] = sum_k A[m, k] * B[n, k].
 enum GemmMode : int {
   kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
   kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
@@ -14,10 +15,10 @@ enum GemmMode : int {
 };
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
-constexpr int kRowsM = 128;        // UMMA M
-constexpr int kStagesA = 3;        // decoded FP16 A tiles (16 KB each)
-constexpr int kStagesB = 4;        // TMA-loaded B tiles (32 KB each)
-constexpr int kStagesP = 6;        // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kRowsM = 256;        // weight rows per work item (two UMMAs of M = 128)
+constexpr int kStagesA = 2;        // decoded FP16 A tiles (32 KB each)
+constexpr int kStagesB = 3;        // TMA-loaded B tiles (32 KB each)
+constexpr int kStagesP = 4;        // TMA-loaded packed int4 tiles (8 KB each)
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
@@ -28,15 +29,16 @@ struct GemmParams {
   const int4* tok_tiles;     // {expert, first permuted row, rows, 0}
   const WsHeader* hdr;       // n_tok_tiles
   uint32_t* status;
-  int n_rowblk;              // output row blocks per token tile
+  int n_rowblk;              // output feature blocks per token tile
+  int feat;                  // output features of the mode (the last block may hold only 128)
   int n_main;                // main reduction stages (K / 64)
   int need_saved;            // backward: run only when a saved forward is pending
-  // frozen base (packed, scales) of projection 0 and 1
+  // frozen base scales of projection 0 and 1 (bf16)
   const uint16_t* s0;
   const uint16_t* s1;
   int64_t s_expert;          // scale elements per expert
   int s_row;                 // scales per stored row
-  int stored_rows;           // stored rows per expert of one projection (GU_T: I)
+  int stored_rows;           // stored rows per expert of one projection
   // LoRA operand of the extra reduction stage (bf16 LoRA tensors)
   const uint16_t* lx0;
   const uint16_t* lx1;
