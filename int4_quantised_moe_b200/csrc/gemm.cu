@@ -43,7 +43,7 @@ constexpr int kOffBar = kOffP + kStagesP * kPBytes;
 constexpr int kNumBars = 2 * kStagesP + 2 * kStagesA + 2 * kStagesB + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
-constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;
+constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // route-gradient partials: per-warp tables, per-warp sums
 constexpr int kSmemBytes = kOffEpi + kEpiFloats * 4 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {  // kModeDownT
           // Per half: the accumulators of 32 tokens, then the saved G/U of
-          // 8 tokens at a time, loaded together ahead of their use.
+          // 4 tokens at a time, loaded together ahead of their use.
           const float L = p.limit;
           float* red = epi + q * 32 * 33;
           float* red2 = epi + 4 * 32 * 33;
@@ -500,24 +500,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32((hf ? d1 : d0) + lane_base + (uint32_t)c0, v0);
             const int i = f0 + 128 * hf + m;
 #pragma unroll
-            for (int cb = 0; cb < 32; cb += 8) {
-              float g8[8], u8[8];
+            for (int cb = 0; cb < 32; cb += 4) {
+              float gq[4], uq[4];
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
+              for (int c = 0; c < 4; ++c) {
                 const int64_t row = p0 + min(c0 + cb + c, n_rows - 1);
-                g8[c] = __ldg(p.in_g + row * p.ld_out + i);
-                u8[c] = __ldg(p.in_u + row * p.ld_out + i);
+                gq[c] = __ldg(p.in_g + row * p.ld_out + i);
+                uq[c] = __ldg(p.in_u + row * p.ld_out + i);
               }
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
+              for (int c = 0; c < 4; ++c) {
                 const int n = c0 + cb + c;
                 const float w = __shfl_sync(0xffffffffu, wl, cb + c);
-                float prod = 0.f;
+                float pr = 0.f;
                 if (n < n_rows) {
                   const int64_t row = p0 + n;
                   const float acc_v = __uint_as_float(v0[cb + c]);
-                  const float g = g8[c];
-                  const float u = u8[c];
+                  const float g = gq[c];
+                  const float u = uq[c];
                   const float gc = L > 0.f ? fminf(g, L) : g;
                   const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
                   const bool pass_g = !(L > 0.f) || g <= L;
@@ -533,10 +533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                   overflow |= (__hisinf(hg) | __hisinf(hu)) != 0;
                   p.out_h[row * (2 * p.inter) + i] = *reinterpret_cast<const uint16_t*>(&hg);
                   p.out_h[row * (2 * p.inter) + p.inter + i] = *reinterpret_cast<const uint16_t*>(&hu);
-                  prod = acc_v * silu * uc;
+                  pr = acc_v * silu * uc;
                 }
                 float* slot = red + lane * 33 + cb + c;
-                *slot = hf ? *slot + prod : prod;
+                *slot = hf ? *slot + pr : pr;
               }
             }
           }
@@ -587,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
         uint8_t* A = sA + ra.stage * kABytes;
+        int p_release = -1;  // packed stage to hand back once its bytes are consumed
         if (s < n_main) {
           const uint32_t sc = sq0;
           sq0 = sq1;
@@ -596,8 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_all(&p_full[rp.stage], rp.phase, abort_flag, status)) goto done;
           uint4 q0, q1;
           packed_pair<MODE>(sP + rp.stage * kPBytes, dt, q0, q1);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+          p_release = rp.stage;
           rp.advance(kStagesP);
           uint32_t w0[16], w1[16];
           decode_group32(q0, bf16_scale_to_h2((uint16_t)(sc & 0xFFFFu)), w0);
@@ -617,7 +617,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[ra.stage]);
+        if (lane == 0) {
+          // The packed stage is released only here, after the decoded values
+          // that consume its bytes were stored: an arrive issued right after
+          // the shared loads can overtake them, and the refill of the stage
+          // then lands under loads still in flight.
+          if (p_release >= 0) mbar_arrive(&p_empty[p_release]);
+          mbar_arrive(&a_full[ra.stage]);
+        }
         ra.advance(kStagesA);
       }
     }

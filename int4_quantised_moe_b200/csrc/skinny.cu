@@ -63,25 +63,53 @@ __device__ __forceinline__ void grad_store(uint16_t* out, int64_t o, float v, in
   out[o] = bf16_bits_rn(v);
 }
 
-// One (feature p, rank j) gradient element of job `jb` for expert e.
-__device__ __forceinline__ void grad_element(const SkJob& jb, int rank, int rpad, int e, int p, int j, const float* D,
-                                             float gs, int accumulate, bool zero) {
-  uint16_t* out = jb.out_lo;
-  int pp = p, dj = j;
-  if (jb.split == kSplitFeature) {
-    const int half = jb.P / 2;
-    if (p >= half) {
-      out = jb.out_hi;
-      pp = p - half;
-      dj = rpad + j;
-    }
+__device__ __forceinline__ uint32_t grad_pair(uint32_t old, float a, float b, int accumulate) {
+  if (accumulate) {
+    a += __uint_as_float(old << 16);
+    b += __uint_as_float(old & 0xFFFF0000u);
   }
-  auto put = [&](uint16_t* buf, int jj, int dcol) {
-    const int64_t o = jb.transposed ? ((int64_t)e * rank + jj) * jb.pout + pp : ((int64_t)e * jb.pout + pp) * rank + jj;
-    grad_store(buf, o, zero ? 0.f : gs * D[dcol], zero ? 0 : accumulate);
-  };
-  put(out, j, dj);
-  if (jb.split == kSplitRank) put(jb.out_hi, j, rpad + j);
+  return (uint32_t)bf16_bits_rn(a) | ((uint32_t)bf16_bits_rn(b) << 16);
+}
+
+// The `rank` gradient values of feature pp of expert e in one output buffer:
+// buf = (accumulate ? buf : 0) + gs * D[j], D read from the accumulator
+// columns in `v` (all zero when `zero`). [E, pout, r] rows are contiguous and
+// go out as 16-byte vectors when r is a multiple of 8 and the buffer is
+// 16-byte aligned; [E, r, pout] columns are written one element per rank
+// index, contiguous across the warp's lanes.
+__device__ __forceinline__ void grad_row(uint16_t* buf, const SkJob& jb, int rank, int e, int pp, const uint32_t (&v)[32],
+                                         float gs, int accumulate, bool zero) {
+  if (zero) accumulate = 0;
+  if (!jb.transposed) {
+    uint16_t* dst = buf + ((int64_t)e * jb.pout + pp) * rank;
+    if ((rank & 7) == 0 && (reinterpret_cast<uintptr_t>(buf) & 15u) == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (8 * c < rank) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 8 * c);
+          const uint4 old = accumulate ? *d4 : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+          uint32_t nw[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float a = zero ? 0.f : gs * __uint_as_float(v[8 * c + 2 * t]);
+            const float b = zero ? 0.f : gs * __uint_as_float(v[8 * c + 2 * t + 1]);
+            nw[t] = grad_pair(ow[t], a, b, accumulate);
+          }
+          *d4 = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < rank) grad_store(dst, j, zero ? 0.f : gs * __uint_as_float(v[j]), accumulate);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < rank)
+        grad_store(buf, ((int64_t)e * rank + j) * jb.pout + pp, zero ? 0.f : gs * __uint_as_float(v[j]), accumulate);
+  }
 }
 
 template <int MODE>
@@ -292,29 +320,44 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const SkJob& jb = p.job[g.job];
         const int rows = p.offsets[g.e + 1] - p.offsets[g.e];
         const int pf = 128 * g.fb + 32 * q + lane;  // feature of this lane
-        float D[64];
+        // outputs of this item: the low rank block -> out_lo, except the
+        // second feature half of a feature split (high block -> out_hi); the
+        // rank split writes both blocks
+        uint16_t* out0 = jb.out_lo;
+        uint32_t col0 = 0;
+        int pbase = 0;
+        if (jb.split == kSplitFeature && 128 * g.fb >= jb.P / 2) {
+          out0 = jb.out_hi;
+          col0 = (uint32_t)p.rpad;
+          pbase = jb.P / 2;
+        }
+        const bool both = jb.split == kSplitRank;
+        const bool live = pf < jb.P;
+        uint32_t v0[32], v1[32];
         if (rows == 0) {
           // no rows of this expert in the call: cleared, or kept when accumulating
-          if (!p.accumulate && pf < jb.P)
-            for (int j = 0; j < p.rank; ++j) grad_element(jb, p.rank, p.rpad, g.e, pf, j, D, 0.f, 0, true);
+          if (!p.accumulate && live) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v0[j] = 0u;
+            grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, 0.f, 0, true);
+            if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v0, 0.f, 0, true);
+          }
           continue;
         }
         const int ab = it & 1;
         if (!wait_all(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status)) goto done;
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128), v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) D[j] = __uint_as_float(v[j]);
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128 + 32), v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) D[32 + j] = __uint_as_float(v[j]);
+        const uint32_t t0 = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128);
+        tmem_ld32(t0 + col0, v0);
+        if (both) tmem_ld32(t0 + (uint32_t)p.rpad, v1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
         ++it;
-        if (pf < jb.P)
-          for (int j = 0; j < p.rank; ++j) grad_element(jb, p.rank, p.rpad, g.e, pf, j, D, p.grad_scale, p.accumulate, false);
+        if (live) {
+          grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, p.grad_scale, p.accumulate, false);
+          if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v1, p.grad_scale, p.accumulate, false);
+        }
       }
     }
   }
