@@ -38,6 +38,13 @@ UNIT = "routed tokens/s"
 
 # ----------------------------------------------------------------- helpers
 
+def gemm_source_hash():
+    import hashlib
+    d = os.path.join(ROOT, "int4_quantised_moe_b200", "csrc")
+    src = b"".join(open(os.path.join(d, f), "rb").read() for f in ("gemm.cu", "gemm.cuh", "common.cuh"))
+    return hashlib.sha256(src).hexdigest()[:16]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -207,11 +214,12 @@ def main():
         pg = dist
 
     from int4_quantised_moe_b200 import binding as B
+    from int4_quantised_moe_b200 import dp
 
     # layer (same on every rank) and this rank's batch
     wl = make_workload(cfg, device=dev)
     if rank > 0:
-        x, ids, w, g = make_batch(cfg, seed=20261001 + 7919 * rank, device=dev)
+        x, ids, w, g = make_batch(cfg, seed=dp.rank_batch_seed(rank), device=dev)
         wl.x, wl.expert_ids, wl.route_weights, wl.grad_out = x, ids, w, g
     counts = expert_counts(wl.expert_ids, cfg.experts)
     nbytes, flops, R, hit = algorithmic(cfg, counts)
@@ -227,19 +235,14 @@ def main():
         layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=True)
         layer.backward(wl.grad_out, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
         if pg is not None:
-            for n in LORA_NAMES:
-                pg.all_reduce(grads[n])
+            dp.allreduce_lora_grads(grads)
 
     def barrier():
         if pg is not None:
             pg.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if pg is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return dp.max_over_ranks(v, device=dev)
 
     for _ in range(args.warmup):
         step()
@@ -281,9 +284,11 @@ def main():
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
+        # DRAM bytes of one launch from an ncu capture; void once the GEMM
+        # sources differ from the ones the counters were taken on
         tj = json.load(open(tfile))
-        if tj.get("kernel") == dom and tj.get("config") == args.config:
-            traffic = tj.get("dram_bytes_per_launch")
+        if tj.get("config") == args.config and tj.get("source_sha256_16") == gemm_source_hash():
+            traffic = tj.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2), "peak": pk["tflops_sustained"],
                 "unit": "TFLOP/s", "frac": round(achieved / pk["tflops_sustained"], 4), "traffic": traffic,
                 "peak_source": f"{pk['source']} bf16 sustained (fp16 dense rate equals bf16)"}
@@ -316,8 +321,7 @@ def main():
         layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
         layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
         if pg is not None:
-            for n in LORA_NAMES:
-                pg.all_reduce(grads[n])
+            dp.allreduce_lora_grads(grads)
         h_out.copy_(out, non_blocking=True)
         h_gin.copy_(gin, non_blocking=True)
         h_gr.copy_(groute, non_blocking=True)
@@ -357,10 +361,7 @@ def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_na
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": {"workload": workload_name, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "global_batch_tokens": cfg.qlen * world, "routed_rows_per_gpu": R,
-                       "l2": "inputs larger than L2: every step streams all hit experts' packed weights "
-                             f"({2 * hit * 3 * cfg.hidden * cfg.inter * (0.5 + 1 / 16) / 1e9:.1f} GB)"},
+            "config": arm_config(cfg, world, workload_name, R, hit),
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": len(launches), "clocks": clocks, "device_status": st,
             "kernels": {n: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 4), "share": round(v["share"], 4)}
@@ -371,6 +372,14 @@ def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_na
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: int) -> dict:
+    """The `config` object of the JSON line, shared by both arms."""
+    return {"workload": workload_name, "parallelism": f"dp{world}" if world > 1 else "single",
+            "global_batch_tokens": cfg.qlen * world, "routed_rows_per_gpu": R,
+            "l2": "inputs larger than L2: every step streams all hit experts' packed weights "
+                  f"({2 * hit * 3 * cfg.hidden * cfg.inter * (0.5 + 1 / 16) / 1e9:.1f} GB)"}
 
 
 def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:
@@ -385,11 +394,13 @@ def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:
         rows_t += rows
         secs_t += secs
     value = rows_t / secs_t
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    _, _, R, hit = algorithmic(cfg, expert_counts(wl.expert_ids, cfg.experts))
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_t / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_name},
+        "config": arm_config(cfg, world, workload_name, R, hit),
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                          "sample": f"each step: float64 NumPy oracle fwd+bwd of whole experts for about {per_step:.1f} s"},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
