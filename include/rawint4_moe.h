@@ -96,6 +96,8 @@ typedef struct rawint4_moe_cfg {
  * down_q:       uint8 [E, H, I/2]; down_s:       bf16 [E, H, I/32]
  * Layout of one projection: rawint4_sft_reference.py, _validate_rawint4_layout
  * (packed uint8 [N_out, K_in/2], scales bf16 [N_out, K_in/32]). */
+/* Every base and LoRA pointer must be 16-byte aligned (RAWINT4_INVALID_ARGUMENT
+ * otherwise): the kernels read them with TMA and 16-byte vector loads. */
 typedef struct rawint4_moe_base {
   const uint8_t *gate_q, *up_q, *down_q;
   const uint16_t *gate_s, *up_s, *down_s;

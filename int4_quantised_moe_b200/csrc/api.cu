@@ -63,7 +63,7 @@ Layout make_layout(const rawint4_moe_cfg& c) {
   L.gdw = take(rows * kLoraPad * 2);
   L.dgu = take(rows * 2 * I * 2);
   L.gb = take(rows * kLoraPad * 2);
-  L.dpart = take(rows * ((I + 255) / 256) * 4);
+  L.dpart = take(rows * 2 * ((I + 255) / 256) * 4);
   L.rpad = (c.rank + 15) / 16 * 16;
   const int64_t rp = L.rpad;
   L.gu16 = take(E * 2 * rp * H * 2);
@@ -89,11 +89,14 @@ bool cfg_ok(const rawint4_moe_cfg* c) {
   return true;
 }
 
+// Base and LoRA tensors are read by TMA and by 16-byte vector loads: their
+// starting addresses must be 16-byte aligned.
+bool a16(const void* p) { return p && reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 bool base_ok(const rawint4_moe_base* b) {
-  return b && b->gate_q && b->up_q && b->down_q && b->gate_s && b->up_s && b->down_s;
+  return b && a16(b->gate_q) && a16(b->up_q) && a16(b->down_q) && a16(b->gate_s) && a16(b->up_s) && a16(b->down_s);
 }
 bool lora_ok(const rawint4_moe_lora* l) {
-  return l && l->gate_a && l->gate_b && l->up_a && l->up_b && l->down_a && l->down_b;
+  return l && a16(l->gate_a) && a16(l->gate_b) && a16(l->up_a) && a16(l->up_b) && a16(l->down_a) && a16(l->down_b);
 }
 bool grads_ok(const rawint4_moe_lora_grads* g) {
   return g && g->gate_a && g->gate_b && g->up_a && g->up_b && g->down_a && g->down_b;
@@ -141,7 +144,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1};
-// 128-byte swizzling for the 128-byte-wide boxes the transposed modes read
+// the 64-byte-wide boxes of the transposed modes are loaded with 64-byte
+// swizzling (conflict-free reads by the decoders)
 bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -150,7 +154,7 @@ bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, in
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -205,6 +209,21 @@ int common_checks(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base, cons
 int grid_for_tiles(int sms, int max_tiles, int rowblk) {
   const int64_t t = (int64_t)max_tiles * rowblk;
   return (int)(t < sms ? (t > 0 ? t : 1) : sms);
+}
+
+// CTA pairs for a GEMM launch: all that fit at once, or fewer for a small
+// problem (work items = token tiles x feature blocks).
+int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
+  static int cached[64][4];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev][mode] <= 0) {
+    const int n = gemm_max_clusters(mode);
+    cached[dev][mode] = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
+  }
+  const int fit = cached[dev][mode];
+  const int64_t items = (int64_t)max_tiles * rowblk;
+  return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }
 
 #define R4_TRY(x)                                \
@@ -325,7 +344,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 128) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 128) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = I / 128;
@@ -346,7 +365,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_gate_up", st);
-    R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeGateUp, gp, mp, gemm_clusters(kModeGateUp, sms, max_tiles, gp.n_rowblk), st));
   }
 
   // ha = c * h A_d^T and hw = w * ha
@@ -363,7 +382,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 256) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 256) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -382,7 +401,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_down", st);
-    R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeDown, gp, mp, gemm_clusters(kModeDown, sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_out", st);
@@ -472,7 +491,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 128, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 128, 64) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (I + 255) / 256;
@@ -494,7 +513,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_down_t", st);
-    R4_TRY(launch_gemm(kModeDownT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
   }
 
   // gb = c * [dG B_g, dU B_u]: gate in columns [0, r), up in [rp, rp + r)
@@ -515,7 +534,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 128, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 128, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -537,7 +556,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_gate_up_t", st);
-    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, gemm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_dx", st);
@@ -545,7 +564,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
   if (grad_route) {
     R4_PROF("combine_route", st);
-    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), (I + 255) / 256, at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ,
+    R4_TRY(launch_combine_route(at<float>(ws, L.dpart), 2 * ((I + 255) / 256), at<int32_t>(ws, L.inv), k, hdr, grad_route, maxQ,
                                 st));
   }
 

@@ -187,14 +187,16 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Instruction descriptor, kind::f16: FP16 A/B, FP32 D, M = 128.
-__host__ __device__ constexpr uint32_t make_idesc_f16(uint32_t n, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor, kind::f16: FP16 A/B, FP32 D, M = 128 (or 256 for
+// a CTA-pair MMA).
+__host__ __device__ constexpr uint32_t make_idesc_f16(uint32_t n, bool a_mn_major, bool b_mn_major,
+                                                      uint32_t m = 128) {
   return (1u << 4)                          // D format: F32
          | (0u << 7) | (0u << 10)           // A, B format: F16
          | ((a_mn_major ? 1u : 0u) << 15)   // A major
          | ((b_mn_major ? 1u : 0u) << 16)   // B major
          | ((n >> 3) << 17)                 // N / 8
-         | ((128u >> 4) << 24);             // M / 16
+         | ((m >> 4) << 24);                // M / 16
 }
 
 // Shared-memory matrix descriptor with 128-byte swizzling.
@@ -231,6 +233,136 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------- cp.async with mbarrier
+// Small asynchronous global->shared copies whose completion is counted on an
+// mbarrier: the issuing thread never waits for them (unlike ordinary loads,
+// which a later release-arrive of the same thread would have to wait for).
+// `src_bytes` 0 fills the destination with zeros without reading.
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_8(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once all cp.async of this thread issued so far have landed
+// (the barrier's expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ------------------------------------------------------ CTA pairs (2 SMs)
+// A cluster of two CTAs on one SM pair: rank 0 (the leader) issues the
+// pair-wide MMAs; every other wrapper runs in both CTAs.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// All threads of both CTAs (each warp converged).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier given by its shared::cluster address (either CTA),
+// with the default (CTA-scope release) semantics: the operand data the
+// arrival announces lives in the arriving CTA's own shared memory and is
+// made visible to that SM's tensor-core (async) proxy by a proxy fence
+// before the arrival. A cluster-scope release here costs a full memory
+// barrier per arrival (about 0.7 us measured) and is not needed for that.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// try_wait for phases completed by the peer CTA or by pair-wide tensor-core
+// commits (default acquire semantics, as for local phases).
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             uint32_t* status) {
+  if (mbar_try_wait_cl(bar, parity, 0u)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_cl(bar, parity, 1000000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      raise_status(status, RAWINT4_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool wait_all_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            uint32_t* status) {
+  const bool ok = mbar_wait_cl(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+// Tiled TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (shared::cluster address). No
+// multicast: each CTA loads only its own tile.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t c0,
+                                                 int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Pair-wide D[tmem] (+)= A * B^T: M = 256 (rows 0-127 from the leader's A
+// tile, 128-255 from the peer's at the same offset), N columns of B split
+// between the two CTAs (first half in the leader), FP16 in, FP32 accumulate;
+// each CTA's TMEM receives its own 128 rows. Issued by one leader thread.
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on `bar` (same offset) in every CTA of `cta_mask` when all MMAs
+// this thread issued so far have finished.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 // ------------------------------------------------------------------ decode

@@ -3,10 +3,13 @@
 
 namespace r4 {
 
-// The four dequant-fused grouped GEMMs of the layer. A work item puts 256
-// weight rows (output features; gate/up: 128 features of each) on the UMMA M
-// side as two M=128 MMAs that share every B tile, and up to 256 permuted
-// tokens of one expert on the N side: D[m, n] = sum_k A[m, k] * B[n, k].
+// The four dequant-fused grouped GEMMs of the layer, run by clusters of two
+// CTAs on an SM pair. A work item puts 256 weight rows (output features;
+// gate/up: 128 features of each) on the UMMA M side, 128 rows in each CTA's
+// shared memory, and up to 256 permuted tokens of one expert on the N side,
+// half of them in each CTA: D[m, n] = sum_k A[m, k] * B[n, k]. One leader
+// thread issues the pair-wide MMA (M = 256); each CTA's TMEM holds its 128
+// rows of the accumulator.
 enum GemmMode : int {
   kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
   kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
@@ -15,10 +18,11 @@ enum GemmMode : int {
 };
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
-constexpr int kRowsM = 256;        // weight rows per work item (two UMMAs of M = 128)
-constexpr int kStagesA = 2;        // decoded FP16 A tiles (32 KB each)
-constexpr int kStagesB = 3;        // TMA-loaded B tiles (32 KB each)
-constexpr int kStagesP = 4;        // TMA-loaded packed int4 tiles (8 KB each)
+constexpr int kRowsM = 128;        // weight rows per CTA (256 per CTA pair)
+constexpr int kStagesA = 4;        // decoded FP16 A tiles (16 KB each)
+constexpr int kStagesB = 6;        // TMA-loaded B tiles (up to 128 tokens, 16 KB each)
+constexpr int kStagesP = 8;        // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kStagesS = 16;       // group scales of one stage (512 B each)
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
@@ -29,7 +33,7 @@ struct GemmParams {
   const int4* tok_tiles;     // {expert, first permuted row, rows, 0}
   const WsHeader* hdr;       // n_tok_tiles
   uint32_t* status;
-  int n_rowblk;              // output feature blocks per token tile
+  int n_rowblk;              // output feature blocks (of a CTA pair) per token tile
   int feat;                  // output features of the mode (the last block may hold only 128)
   int n_main;                // main reduction stages (K / 64)
   int need_saved;            // backward: run only when a saved forward is pending
@@ -53,7 +57,7 @@ struct GemmParams {
   uint16_t* out_h;           // GU: h (fp16); DOWN_T: dG|dU (fp16)
   const float* in_g;         // DOWN_T: saved G
   const float* in_u;         // DOWN_T: saved U
-  float* droute_part;        // DOWN_T: [rows, n_rowblk]
+  float* droute_part;        // DOWN_T: [rows, 2 n_rowblk] (one partial per CTA)
   int ld_out;                // row length of out_a / out_b / out_h / in_*
   int inter;
   float limit;
@@ -67,6 +71,9 @@ struct GemmMaps {
 };
 
 size_t gemm_smem_bytes();
-cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t stream);
+// Launches `clusters` CTA pairs (at most the number that fit at once).
+cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
+// CTA pairs of the mode's kernel resident at once on this device (0 on error).
+int gemm_max_clusters(int mode);
 
 }  // namespace r4
