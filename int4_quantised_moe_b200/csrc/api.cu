@@ -144,8 +144,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1};
-// the 64-byte-wide boxes of the transposed modes are loaded with 64-byte
-// swizzling (conflict-free reads by the decoders)
+// the 128- and 64-byte-wide boxes of the transposed modes are loaded with the
+// matching swizzle (conflict-free reads by the decoders)
 bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -154,7 +154,7 @@ bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, in
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (box_x == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -211,14 +211,14 @@ int grid_for_tiles(int sms, int max_tiles, int rowblk) {
   return (int)(t < sms ? (t > 0 ? t : 1) : sms);
 }
 
-// CTA pairs for a GEMM launch: all that fit at once, or fewer for a small
+// CTA pairs for a pair-kernel launch: all that fit at once, or fewer for a small
 // problem (work items = token tiles x feature blocks).
 int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
   static int cached[64][4];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   if (cached[dev][mode] <= 0) {
-    const int n = gemm_max_clusters(mode);
+    const int n = gemm_pair_max_clusters(mode);
     cached[dev][mode] = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
   }
   const int fit = cached[dev][mode];
@@ -344,7 +344,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 128) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 128) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = I / 128;
@@ -365,7 +365,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_gate_up", st);
-    R4_TRY(launch_gemm(kModeGateUp, gp, mp, gemm_clusters(kModeGateUp, sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
 
   // ha = c * h A_d^T and hw = w * ha
@@ -382,7 +382,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 128) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 128) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 256) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 256) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -401,7 +401,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_down", st);
-    R4_TRY(launch_gemm(kModeDown, gp, mp, gemm_clusters(kModeDown, sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_out", st);
@@ -510,10 +510,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.in_g = at<float>(ws, L.g);
   gp.in_u = at<float>(ws, L.u);
   gp.droute_part = at<float>(ws, L.dpart);
+  gp.n_parts = 2 * gp.n_rowblk;
   gp.ld_out = I;
   {
     R4_PROF("gemm_down_t", st);
-    R4_TRY(launch_gemm(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm_pair(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
   }
 
   // gb = c * [dG B_g, dU B_u]: gate in columns [0, r), up in [rp, rp + r)
@@ -534,7 +535,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 128, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -556,7 +557,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_gate_up_t", st);
-    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, gemm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_dx", st);

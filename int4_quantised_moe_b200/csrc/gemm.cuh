@@ -3,13 +3,16 @@
 
 namespace r4 {
 
-// The four dequant-fused grouped GEMMs of the layer, run by clusters of two
-// CTAs on an SM pair. A work item puts 256 weight rows (output features;
-// gate/up: 128 features of each) on the UMMA M side, 128 rows in each CTA's
-// shared memory, and up to 256 permuted tokens of one expert on the N side,
-// half of them in each CTA: D[m, n] = sum_k A[m, k] * B[n, k]. One leader
-// thread issues the pair-wide MMA (M = 256); each CTA's TMEM holds its 128
-// rows of the accumulator.
+// The four dequant-fused grouped GEMMs of the layer. Weight rows (output
+// features) sit on the UMMA M side and up to 256 permuted tokens of one expert
+// on the N side: D[m, n] = sum_k A[m, k] * B[n, k]. Two kernels implement
+// them (both take the same parameters):
+//   gemm.cu       one CTA per SM, 256 weight rows per work item as two
+//                 M = 128 MMAs sharing every B tile (gate/up, down, gate/up^T)
+//   gemm_pair.cu  CTA pairs on SM pairs (tcgen05 cta_group::2), 256 weight
+//                 rows per item as one M = 256 pair MMA; each SM's TMEM holds
+//                 only 128 rows, so 256-token accumulators double-buffer and
+//                 a heavy epilogue overlaps the next item (down^T)
 enum GemmMode : int {
   kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
   kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
@@ -18,22 +21,13 @@ enum GemmMode : int {
 };
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
-constexpr int kRowsM = 128;        // weight rows per CTA (256 per CTA pair)
-constexpr int kStagesA = 4;        // decoded FP16 A tiles (16 KB each)
-constexpr int kStagesB = 6;        // TMA-loaded B tiles (up to 128 tokens, 16 KB each)
-constexpr int kStagesP = 8;        // TMA-loaded packed int4 tiles (4 KB each)
-constexpr int kStagesS = 16;       // group scales of one stage (512 B each)
-constexpr int kThreads = 512;      // 16 warps
-constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
-constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
-constexpr int kDecThreads = 256;
 constexpr int kLoraPad = 64;       // width of the LoRA side matrices (>= 2 * rank)
 
 struct GemmParams {
   const int4* tok_tiles;     // {expert, first permuted row, rows, 0}
   const WsHeader* hdr;       // n_tok_tiles
   uint32_t* status;
-  int n_rowblk;              // output feature blocks (of a CTA pair) per token tile
+  int n_rowblk;              // output feature blocks (work items) per token tile
   int feat;                  // output features of the mode (the last block may hold only 128)
   int n_main;                // main reduction stages (K / 64)
   int need_saved;            // backward: run only when a saved forward is pending
@@ -57,7 +51,8 @@ struct GemmParams {
   uint16_t* out_h;           // GU: h (fp16); DOWN_T: dG|dU (fp16)
   const float* in_g;         // DOWN_T: saved G
   const float* in_u;         // DOWN_T: saved U
-  float* droute_part;        // DOWN_T: [rows, 2 n_rowblk] (one partial per CTA)
+  float* droute_part;        // DOWN_T: [rows, n_parts] route-gradient partial sums
+  int n_parts;               // DOWN_T: partials per row (one per CTA and feature block)
   int ld_out;                // row length of out_a / out_b / out_h / in_*
   int inter;
   float limit;
@@ -70,10 +65,11 @@ struct GemmMaps {
   CUtensorMap bx[4];  // B LoRA: 2D fp16 {64, rows}, 128B swizzle, boxes {64, 16 << i}
 };
 
-size_t gemm_smem_bytes();
-// Launches `clusters` CTA pairs (at most the number that fit at once).
-cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
-// CTA pairs of the mode's kernel resident at once on this device (0 on error).
-int gemm_max_clusters(int mode);
+// One CTA per SM; `grid` CTAs (at most one per SM).
+cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t stream);
+// CTA pairs; `clusters` pairs (at most the number resident at once).
+cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
+// CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
+int gemm_pair_max_clusters(int mode);
 
 }  // namespace r4
