@@ -10,29 +10,36 @@ namespace {
 __device__ __forceinline__ bool bwd_enabled(const WsHeader* hdr) { return hdr->saved == 1u; }
 
 // ------------------------------------------------------------------ gather
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm, int top_k,
-                                   const WsHeader* hdr, uint4* __restrict__ dst, int vecs_per_row, uint32_t* status,
-                                   int need_saved) {
+// One warp per permuted row: the source token is looked up once, then the
+// row is converted 8 elements per lane and step with 16-byte loads/stores.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
+                                                          int top_k, const WsHeader* hdr, uint4* __restrict__ dst,
+                                                          int vecs_per_row, uint32_t* status, int need_saved) {
   if (need_saved && !bwd_enabled(hdr)) return;
   const int64_t rows = hdr->routed;
-  const int64_t total = rows * vecs_per_row;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   bool overflow = false;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = idx / vecs_per_row;
-    const int c = (int)(idx - row * vecs_per_row);
+  for (int64_t row = warp0; row < rows; row += nwarps) {
     const int32_t t = perm[row] / top_k;
-    const uint4 v = __ldg(src + (int64_t)t * vecs_per_row + c);
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
+    const uint4* s = src + (int64_t)t * vecs_per_row;
+    uint4* d = dst + row * vecs_per_row;
+#pragma unroll 4
+    for (int c = lane; c < vecs_per_row; c += 32) {
+      const uint4 v = __ldg(s + c);
+      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+      uint32_t out[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = __uint_as_float(in[j] << 16);
-      const float hi = __uint_as_float(in[j] & 0xFFFF0000u);
-      __half2 h = __floats2half2_rn(lo, hi);
-      overflow |= (__hisinf(__low2half(h)) | __hisinf(__high2half(h))) != 0 && isfinite(lo) && isfinite(hi);
-      out[j] = *reinterpret_cast<uint32_t*>(&h);
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(in[j] << 16);
+        const float hi = __uint_as_float(in[j] & 0xFFFF0000u);
+        __half2 h = __floats2half2_rn(lo, hi);
+        overflow |= (__hisinf(__low2half(h)) | __hisinf(__high2half(h))) != 0 && isfinite(lo) && isfinite(hi);
+        out[j] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      d[c] = make_uint4(out[0], out[1], out[2], out[3]);
     }
-    dst[idx] = make_uint4(out[0], out[1], out[2], out[3]);
   }
   if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
 }
@@ -136,7 +143,7 @@ cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, in
                                uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved,
                                cudaStream_t stream) {
   const int vecs = H / 8;
-  gather_rows_kernel<<<grid_for((int64_t)max_rows * vecs, 256), 256, 0, stream>>>(
+  gather_rows_kernel<<<grid_for((int64_t)max_rows * 32, 256), 256, 0, stream>>>(
       reinterpret_cast<const uint4*>(src_bf16), perm, top_k, hdr, reinterpret_cast<uint4*>(dst_f16), vecs, status,
       need_saved);
   return cudaGetLastError();

@@ -382,38 +382,71 @@ cudaError_t launch_sk(const SkParams& p, const SkMaps& m, int grid, cudaStream_t
 }
 
 // ---------------------------------------------------------- LoRA to FP16
-__global__ void lora_convert_kernel(LoraCvt j0, LoraCvt j1, LoraCvt j2) {
-  const LoraCvt jb = blockIdx.z == 0 ? j0 : (blockIdx.z == 1 ? j1 : j2);
+__device__ __forceinline__ uint32_t bf16x2_to_h2(uint32_t v) {
+  __half2 h = __floats2half2_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// One job per blockIdx.y. Copies: 8 elements per thread and step (16-byte
+// loads and stores; K is a multiple of 128). Transposes: tiles of 64 columns
+// of one expert; the tile's 64 source rows of r elements are one contiguous,
+// 16-byte aligned run of 128 r bytes, loaded as 16-byte vectors, turned
+// around in shared memory and stored as rows of 64 fp16.
+__global__ void __launch_bounds__(256) lora_convert_kernel(LoraCvt j0, LoraCvt j1, LoraCvt j2, int experts) {
+  const LoraCvt jb = blockIdx.y == 0 ? j0 : (blockIdx.y == 1 ? j1 : j2);
   if (!jb.dst) return;
-  const int e = blockIdx.y;
-  const int r = jb.rank;
-  const int rows_out = jb.rpad * jb.nsrc;
-  const int c0 = blockIdx.x * 64;
-  if (c0 >= jb.cols) return;
-  uint16_t* dst = jb.dst + (int64_t)e * rows_out * jb.cols;
+  const int r = jb.rank, rp = jb.rpad, cols = jb.cols;
   if (!jb.transpose) {
-    for (int idx = threadIdx.x; idx < rows_out * 64; idx += blockDim.x) {
-      const int row = idx >> 6, c = c0 + (idx & 63);
-      if (c >= jb.cols) continue;
-      const int blk = row / jb.rpad, j = row - blk * jb.rpad;
-      float v = 0.f;
+    const int rows_out = rp * jb.nsrc;
+    const int vpr = cols / 8;
+    const int64_t total = (int64_t)experts * rows_out * vpr;
+    uint4* dst = reinterpret_cast<uint4*>(jb.dst);
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+      const int64_t row_g = idx / vpr;
+      const int v = (int)(idx - row_g * vpr);
+      const int e = (int)(row_g / rows_out);
+      const int row = (int)(row_g - (int64_t)e * rows_out);
+      const int blk = row / rp, j = row - blk * rp;
+      uint4 out = make_uint4(0u, 0u, 0u, 0u);
       if (j < r) {
-        const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * jb.cols;
-        v = bf16_bits_to_float(src[c]);
+        const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * cols;
+        const uint4 in = __ldg(reinterpret_cast<const uint4*>(src) + v);
+        out = make_uint4(bf16x2_to_h2(in.x), bf16x2_to_h2(in.y), bf16x2_to_h2(in.z), bf16x2_to_h2(in.w));
       }
-      dst[(int64_t)row * jb.cols + c] = f16_bits_rn(v);
+      dst[idx] = out;
     }
   } else {
     __shared__ float tile[64][33];
-    const uint16_t* src = jb.src0 + (int64_t)e * jb.cols * r;  // [cols, r]
-    for (int idx = threadIdx.x; idx < 64 * r; idx += blockDim.x) {
-      const int c = idx / r, j = idx % r;
-      tile[c][j] = (c0 + c < jb.cols) ? bf16_bits_to_float(src[(int64_t)(c0 + c) * r + j]) : 0.f;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < 64 * jb.rpad; idx += blockDim.x) {
-      const int j = idx >> 6, c = idx & 63;
-      if (c0 + c < jb.cols) dst[(int64_t)j * jb.cols + c0 + c] = f16_bits_rn(j < r ? tile[c][j] : 0.f);
+    const int tiles_per_e = cols / 64;
+    for (int t = blockIdx.x; t < experts * tiles_per_e; t += gridDim.x) {
+      const int e = t / tiles_per_e;
+      const int c0 = (t - e * tiles_per_e) * 64;
+      const uint4* src = reinterpret_cast<const uint4*>(jb.src0 + ((int64_t)e * cols + c0) * r);  // [64][r], contiguous
+      for (int v = threadIdx.x; v < 8 * r; v += blockDim.x) {
+        const uint4 in = __ldg(src + v);
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int flat = 8 * v + u;
+          const int c = flat / r, j = flat - c * r;
+          const uint32_t bits = (w[u >> 1] >> (16 * (u & 1))) & 0xFFFFu;
+          tile[c][j] = __uint_as_float(bits << 16);
+        }
+      }
+      __syncthreads();
+      for (int o = threadIdx.x; o < rp * 8; o += blockDim.x) {
+        const int j = o >> 3, v = o & 7;
+        uint32_t h[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float a = j < r ? tile[8 * v + 2 * u][j] : 0.f;
+          const float b = j < r ? tile[8 * v + 2 * u + 1][j] : 0.f;
+          h[u] = (uint32_t)f16_bits_rn(a) | ((uint32_t)f16_bits_rn(b) << 16);
+        }
+        *reinterpret_cast<uint4*>(jb.dst + ((int64_t)e * rp + j) * cols + c0 + 8 * v) = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+      __syncthreads();
     }
   }
 }
@@ -427,11 +460,9 @@ cudaError_t launch_skinny(int mode, const SkParams& p, const SkMaps& m, int grid
 cudaError_t launch_lora_convert(const LoraCvt* jobs, int njobs, int experts, cudaStream_t stream) {
   LoraCvt z{};
   LoraCvt j[3] = {njobs > 0 ? jobs[0] : z, njobs > 1 ? jobs[1] : z, njobs > 2 ? jobs[2] : z};
-  int cols = 0;
-  for (int i = 0; i < njobs && i < 3; ++i) cols = j[i].cols > cols ? j[i].cols : cols;
-  if (cols == 0) return cudaSuccess;
-  dim3 grid((cols + 63) / 64, experts, 3);
-  lora_convert_kernel<<<grid, 256, 0, stream>>>(j[0], j[1], j[2]);
+  if (njobs <= 0) return cudaSuccess;
+  dim3 grid(148 * 4, njobs > 3 ? 3 : njobs, 1);
+  lora_convert_kernel<<<grid, 256, 0, stream>>>(j[0], j[1], j[2], experts);
   return cudaGetLastError();
 }
 
