@@ -67,7 +67,7 @@ struct GemmMaps {
 
 // One CTA per SM; `grid` CTAs (at most one per SM).
 cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t stream);
-// CTA pairs; `clusters` pairs (at most the number resident at once).
+// CTA pairs (down^T only); `clusters` pairs (at most the number resident at once).
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
 // CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
 int gemm_pair_max_clusters(int mode);

@@ -702,26 +702,20 @@ int max_clusters_mode() {
 
 }  // namespace pairk
 
+// The library runs only the down^T GEMM on CTA pairs (its epilogue is the
+// one that needs double-buffered 256-token accumulators); the kernel itself
+// is written for every mode.
+// The library runs only the down^T GEMM on CTA pairs (its epilogue is the
+// one that needs double-buffered 256-token accumulators); the kernel itself
+// is written for every mode.
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
-  using namespace pairk;
-  switch (mode) {
-    case kModeGateUp: return launch_mode<kModeGateUp>(p, maps, clusters, stream);
-    case kModeDown: return launch_mode<kModeDown>(p, maps, clusters, stream);
-    case kModeDownT: return launch_mode<kModeDownT>(p, maps, clusters, stream);
-    case kModeGateUpT: return launch_mode<kModeGateUpT>(p, maps, clusters, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (mode != kModeDownT) return cudaErrorInvalidValue;
+  return pairk::launch_mode<kModeDownT>(p, maps, clusters, stream);
 }
 
 int gemm_pair_max_clusters(int mode) {
-  using namespace pairk;
-  switch (mode) {
-    case kModeGateUp: return max_clusters_mode<kModeGateUp>();
-    case kModeDown: return max_clusters_mode<kModeDown>();
-    case kModeDownT: return max_clusters_mode<kModeDownT>();
-    case kModeGateUpT: return max_clusters_mode<kModeGateUpT>();
-    default: return 0;
-  }
+  if (mode != kModeDownT) return 0;
+  return pairk::max_clusters_mode<kModeDownT>();
 }
 
 }  // namespace r4
