@@ -1,5 +1,7 @@
 // Dequant-fused grouped GEMMs of the routed RAWINT4 MoE-LoRA layer on
-// sm_100a tensor cores (tcgen05, TMEM accumulators, TMA-fed operands).
+// sm_100a tensor cores (tcgen05, TMEM accumulators, TMA-fed operands), one
+// CTA per SM: gate/up (forward), down (forward) and gate/up^T (backward dX).
+// The down^T GEMM runs on CTA pairs (gemm_pair.cu).
 //
 // One persistent CTA per SM walks (token tile, feature block) work items. A
 // token tile is up to 256 permuted rows of one expert; a feature block is 256
@@ -8,6 +10,7 @@
 // B tile, so every activation tile read from L2 feeds 256 weight rows.
 // Warp roles:
 //   warp 0      TMA producer of packed int4 weight tiles   (ring of kStagesP)
+//   warp 3      loader of the group scales (cp.async, ring of kStagesS)
 //   warp 2      TMA producer of B tiles (activations)      (ring of kStagesB)
 //   warps 8-15  decoders: int4 -> fp16 into the UMMA A layout (ring of kStagesA)
 //   warp 1      UMMA issuer (one elected lane) and TMEM owner
@@ -22,7 +25,7 @@
 // of the expert (loaded into registers at the start of the item and stored
 // by the decoders), its B operand the precomputed c-scaled rank-r side matrix.
 //
-// The backward modes read the packed base along its stored output dimension
+// The gate/up^T mode reads the packed base along its stored output dimension
 // (transpose-free dX, rawint4_sft_reference.py transpose_free_rawint4_dx):
 // the decoders write the same packed bytes into an MN-major A tile, so no
 // transposed or dense copy of any base weight ever exists.
@@ -54,9 +57,7 @@ constexpr int kOffS = kOffP + kStagesP * kPBytes;
 constexpr int kOffBar = kOffS + kStagesS * kSBytes;
 constexpr int kNumBars = 2 * kStagesP + 2 * kStagesA + 2 * kStagesB + 2 * kStagesS + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
-constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // route-gradient partials: per-warp tables, per-warp sums
-constexpr int kSmemBytes = kOffEpi + kEpiFloats * 4 + 1024;  // + alignment slack
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 template <int MODE>
@@ -277,6 +278,7 @@ struct AccTrack {
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  static_assert(MODE != kModeDownT, "down^T runs on the CTA-pair kernel (gemm_pair.cu)");
   const CUtensorMap& tq0 = maps.q0;
   const CUtensorMap& tq1 = maps.q1;
   extern __shared__ uint8_t smem_raw[];
@@ -298,7 +300,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  float* epi = reinterpret_cast<float*>(smem + kOffEpi);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = (uint32_t)(32 * q) << 16;
       for (int c0 = 0; c0 < n_mma; c0 += 32) {
         uint32_t v0[32], v1[32];
-        if constexpr (MODE != kModeDownT) {
+        {
           tmem_ld32(d0 + lane_base + (uint32_t)c0, v0);
           if (two) {
             tmem_ld32(d1 + lane_base + (uint32_t)c0, v1);
@@ -561,73 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (two) p.out_a[row * p.ld_out + f0 + 128 + m] = b;
             }
           }
-        } else {  // kModeDownT
-          // Per half: the accumulators of 32 tokens, then the saved G/U of
-          // 4 tokens at a time, loaded together ahead of their use.
-          const float L = p.limit;
-          float* red = epi + q * 32 * 33;
-          float* red2 = epi + 4 * 32 * 33;
-          bool overflow = false;
-          const float wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
-          for (int hf = 0; hf < (two ? 2 : 1); ++hf) {
-            tmem_ld32((hf ? d1 : d0) + lane_base + (uint32_t)c0, v0);
-            const int i = f0 + 128 * hf + m;
-#pragma unroll
-            for (int cb = 0; cb < 32; cb += 4) {
-              float gq[4], uq[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int64_t row = p0 + min(c0 + cb + c, n_rows - 1);
-                gq[c] = __ldg(p.in_g + row * p.ld_out + i);
-                uq[c] = __ldg(p.in_u + row * p.ld_out + i);
-              }
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int n = c0 + cb + c;
-                const float w = __shfl_sync(0xffffffffu, wl, cb + c);
-                float pr = 0.f;
-                if (n < n_rows) {
-                  const int64_t row = p0 + n;
-                  const float acc_v = __uint_as_float(v0[cb + c]);
-                  const float g = gq[c];
-                  const float u = uq[c];
-                  const float gc = L > 0.f ? fminf(g, L) : g;
-                  const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
-                  const bool pass_g = !(L > 0.f) || g <= L;
-                  const bool pass_u = !(L > 0.f) || (u >= -L && u <= L);
-                  const float sg = sigmoid_clamped(gc);
-                  const float silu = gc * sg;
-                  const float dsilu = sg * (1.0f + gc * (1.0f - sg));
-                  const float dh = w * acc_v;
-                  const float dg = pass_g ? dh * uc * dsilu : 0.f;
-                  const float du = pass_u ? dh * silu : 0.f;
-                  const __half hg = __float2half_rn(dg);
-                  const __half hu = __float2half_rn(du);
-                  overflow |= (__hisinf(hg) | __hisinf(hu)) != 0;
-                  p.out_h[row * (2 * p.inter) + i] = *reinterpret_cast<const uint16_t*>(&hg);
-                  p.out_h[row * (2 * p.inter) + p.inter + i] = *reinterpret_cast<const uint16_t*>(&hu);
-                  pr = acc_v * silu * uc;
-                }
-                float* slot = red + lane * 33 + cb + c;
-                *slot = hf ? *slot + pr : pr;
-              }
-            }
-          }
-          if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
-          __syncwarp();
-          float colsum = 0.f;
-#pragma unroll 8
-          for (int r2 = 0; r2 < 32; ++r2) colsum += red[r2 * 33 + lane];
-          red2[q * 32 + lane] = colsum;
-          named_bar_sync(3, 128);
-          if (q == 0) {
-            const int n = c0 + lane;
-            if (n < n_rows) {
-              const float sum = red2[lane] + red2[32 + lane] + red2[64 + lane] + red2[96 + lane];
-              p.droute_part[(int64_t)(p0 + n) * p.n_parts + rb] = sum;
-            }
-          }
-          named_bar_sync(3, 128);
         }
       }
       tc_fence_before();
@@ -726,7 +660,6 @@ cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int
   switch (mode) {
     case kModeGateUp: return launch_mode<kModeGateUp>(p, maps, grid, stream);
     case kModeDown: return launch_mode<kModeDown>(p, maps, grid, stream);
-    case kModeDownT: return launch_mode<kModeDownT>(p, maps, grid, stream);
     case kModeGateUpT: return launch_mode<kModeGateUpT>(p, maps, grid, stream);
     default: return cudaErrorInvalidValue;
   }
