@@ -110,7 +110,8 @@ typedef struct rawint4_moe_lora {
   const uint16_t *gate_a, *gate_b, *up_a, *up_b, *down_a, *down_b;
 } rawint4_moe_lora;
 
-/* LoRA gradient buffers (device, bf16), same shapes as rawint4_moe_lora. */
+/* LoRA gradient buffers (device, bf16), same shapes as rawint4_moe_lora;
+ * 16-byte aligned (RAWINT4_INVALID_ARGUMENT otherwise). */
 typedef struct rawint4_moe_lora_grads {
   uint16_t *gate_a, *gate_b, *up_a, *up_b, *down_a, *down_b;
 } rawint4_moe_lora_grads;

@@ -99,7 +99,7 @@ bool lora_ok(const rawint4_moe_lora* l) {
   return l && a16(l->gate_a) && a16(l->gate_b) && a16(l->up_a) && a16(l->up_b) && a16(l->down_a) && a16(l->down_b);
 }
 bool grads_ok(const rawint4_moe_lora_grads* g) {
-  return g && g->gate_a && g->gate_b && g->up_a && g->up_b && g->down_a && g->down_b;
+  return g && a16(g->gate_a) && a16(g->gate_b) && a16(g->up_a) && a16(g->up_b) && a16(g->down_a) && a16(g->down_b);
 }
 
 // --------------------------------------------------------------- device

@@ -16,7 +16,10 @@ constexpr int kSkStage = kSkA + kSkB;
 constexpr int kSkOffBar = kSkStages * kSkStage;
 constexpr int kSkNumBars = 2 * kSkStages + 4;
 constexpr int kSkOffMisc = kSkOffBar + kSkNumBars * 8;
-constexpr int kSkSmem = kSkOffMisc + 16 + 1024;
+// gradient staging of the transposed outputs: [2 outputs][32 rank][128 features] fp32
+constexpr int kSkOffStage = (kSkOffMisc + 16 + 15) / 16 * 16;
+constexpr int kSkStageFloats = 2 * 32 * 128;
+constexpr int kSkSmem = kSkOffStage + kSkStageFloats * 4 + 1024;
 static_assert(kSkSmem <= 232448, "shared memory budget");
 constexpr uint32_t kSkTmemCols = 256;
 
@@ -112,6 +115,40 @@ __device__ __forceinline__ void grad_row(uint16_t* buf, const SkJob& jb, int ran
   }
 }
 
+// The [E, r, pout] outputs of one 128-feature block (two for the rank split):
+// the four epilogue warps write their features' gradients into shared memory,
+// then store whole 256-byte rows (8 features per thread and step) with the
+// authoritative-window rule (accumulate: add the old value, round once).
+// All 128 epilogue threads take part (named barrier 1).
+__device__ __forceinline__ void grad_block_transposed(const SkJob& jb, int rank, int e, int p0, uint16_t* out0, bool both,
+                                                      const uint32_t (&v0)[32], const uint32_t (&v1)[32], float gs,
+                                                      int accumulate, bool zero, float* st, int c, int tid) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j < rank) {
+      st[j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v0[j]);
+      if (both) st[4096 + j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v1[j]);
+    }
+  }
+  named_bar_sync(1, 128);
+  const int nout = both ? 2 : 1;
+  for (int idx = tid; idx < nout * rank * 16; idx += 128) {
+    const int o = idx / (rank * 16);
+    const int rem = idx - o * rank * 16;
+    const int j = rem >> 4, v8 = rem & 15;
+    const float* src = st + o * 4096 + j * 128 + 8 * v8;
+    uint16_t* buf = o ? jb.out_hi : out0;
+    uint4* dst = reinterpret_cast<uint4*>(buf + ((int64_t)e * rank + j) * jb.pout + p0 + 8 * v8);
+    const uint4 old = accumulate ? *dst : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+    uint32_t nw[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) nw[t] = grad_pair(ow[t], src[2 * t], src[2 * t + 1], accumulate);
+    *dst = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+  }
+  named_bar_sync(1, 128);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kSkThreads, 1)
     skinny_kernel(const __grid_constant__ SkParams p, const __grid_constant__ SkMaps maps) {
@@ -124,6 +161,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSkOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkOffMisc + 4);
+  float* gstage = reinterpret_cast<float*>(smem + kSkOffStage);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -336,9 +374,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         uint32_t v0[32], v1[32];
         if (rows == 0) {
           // no rows of this expert in the call: cleared, or kept when accumulating
-          if (!p.accumulate && live) {
+          if (p.accumulate) continue;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v0[j] = 0u;
+          for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
+          if (jb.transposed) {
+            grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, 0.f, 0, true, gstage,
+                                  32 * q + lane, threadIdx.x - 64);
+          } else if (live) {
             grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, 0.f, 0, true);
             if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v0, 0.f, 0, true);
           }
@@ -354,7 +396,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
         ++it;
-        if (live) {
+        if (jb.transposed) {
+          grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, p.grad_scale, p.accumulate,
+                                false, gstage, 32 * q + lane, threadIdx.x - 64);
+        } else if (live) {
           grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, p.grad_scale, p.accumulate, false);
           if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v1, p.grad_scale, p.accumulate, false);
         }
