@@ -11,9 +11,25 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/rawint4_moe.h"
 
 namespace r4 {
+
+// Host: whether a one-time per-device setting (a kernel's shared-memory
+// opt-in) was applied on the current device; the caller sets the bit after
+// applying it. Per device, so a process that drives several GPUs applies it
+// on each.
+inline bool device_flag_test(std::atomic<unsigned long long>& mask, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  *dev_out = dev;
+  return dev < 64 && (mask.load() & (1ull << dev)) != 0;
+}
+inline void device_flag_set(std::atomic<unsigned long long>& mask, int dev) {
+  if (dev < 64) mask.fetch_or(1ull << dev);
+}
 
 // ------------------------------------------------------------------ status
 // Workspace header shared by all kernels of one layer call. Lives at the

@@ -644,11 +644,12 @@ done:
 
 template <int MODE>
 cudaError_t launch_mode(const GemmParams& p, const GemmMaps& m, int grid, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (!device_flag_test(attr_set, &dev)) {
     cudaError_t err = cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    attr_set = true;
+    device_flag_set(attr_set, dev);
   }
   gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, stream>>>(p, m);
   return cudaGetLastError();

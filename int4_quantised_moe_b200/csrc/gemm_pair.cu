@@ -665,11 +665,12 @@ done:
 
 template <int MODE>
 bool set_smem_attr() {
-  static bool done = false;
-  if (!done) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  if (!device_flag_test(done, &dev)) {
     if (cudaFuncSetAttribute(gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
       return false;
-    done = true;
+    device_flag_set(done, dev);
   }
   return true;
 }

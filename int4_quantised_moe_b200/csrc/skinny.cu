@@ -416,11 +416,12 @@ done:
 
 template <int MODE>
 cudaError_t launch_sk(const SkParams& p, const SkMaps& m, int grid, cudaStream_t stream) {
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<unsigned long long> attr{0};
+  int dev = 0;
+  if (!device_flag_test(attr, &dev)) {
     cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmem);
     if (e != cudaSuccess) return e;
-    attr = true;
+    device_flag_set(attr, dev);
   }
   skinny_kernel<MODE><<<grid, kSkThreads, kSkSmem, stream>>>(p, m);
   return cudaGetLastError();
