@@ -587,7 +587,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e = tt.x;
       uint32_t lora_w[32];
       lora_values<MODE>(p, e, rb, dt, lora_w);
-      // group scales of the next four stages, loaded well before their use
       for (int s = 0; s <= n_main; ++s) {
         if (!wait_all(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
         uint8_t* A = sA + ra.stage * kABytes;
