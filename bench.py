@@ -6,11 +6,14 @@ combine; backward gather, down^T, gate/up^T, combine, six LoRA gradients)
 over one synthetic batch. Default workload: the largest layer (E=384, top-8,
 H=7168, I=2048, rank 32, alpha 64, 8192 tokens, no clamp) on one B200.
 
-    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--config C]
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--config C] [--mode infer]
 
 Prints one JSON line (rank 0). Under torchrun each rank runs a data-parallel
 replica on its own batch (weak scaling) and the six LoRA gradient buffers are
 summed over ranks with NCCL after every backward.
+
+--mode infer times the frozen-base inference forward instead (no LoRA, no
+saved context; routing, gather, gate/up, down, combine) on the same workload.
 """
 
 from __future__ import annotations
@@ -33,6 +36,7 @@ import torch  # noqa: E402
 from workloads import CONFIGS, LORA_NAMES, LayerConfig, expert_counts, lora_shapes, make_batch, make_workload  # noqa: E402
 
 METRIC = "routed tokens/s per MoE layer (fwd+bwd) and % of HBM/tensor roofline, 1×B200"
+METRIC_INFER = "routed tokens/s per MoE layer (frozen-base inference forward) and % of HBM/tensor roofline, 1×B200"
 UNIT = "routed tokens/s"
 
 
@@ -54,22 +58,25 @@ def peaks():
     return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def algorithmic(cfg: LayerConfig, counts: torch.Tensor):
+def algorithmic(cfg: LayerConfig, counts: torch.Tensor, infer: bool = False):
     """Algorithmic bytes and FLOPs of one fwd+bwd (weights of hit experts read
     in fwd and bwd, LoRA params read twice and grads written, x/out/dY/grad_in
-    and a second read of x in bf16; saved activations not counted)."""
+    and a second read of x in bf16; saved activations not counted), or of one
+    base-only forward (weights of hit experts once, x and out)."""
     Q, k, H, I, r = cfg.qlen, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank
     R = int(counts.sum())
     hit = int((counts > 0).sum())
-    flops = 12 * R * H * I + 18 * R * r * (H + I) + 2 * R * I
     w_e = 3 * H * I * (0.5 + 1.0 / 16.0)
+    if infer:
+        return w_e * hit + 4 * Q * H, 6 * R * H * I + 2 * R * I, R, hit
+    flops = 12 * R * H * I + 18 * R * r * (H + I) + 2 * R * I
     l_e = 2 * r * (3 * H + 3 * I)
     nbytes = 2 * w_e * hit + 3 * l_e * hit + 10 * Q * H
     return nbytes, flops, R, hit
 
 
-def gemm_flops(name: str, R: int, cfg: LayerConfig) -> float:
-    H, I, r = cfg.hidden, cfg.inter, cfg.rank
+def gemm_flops(name: str, R: int, cfg: LayerConfig, lora: bool = True) -> float:
+    H, I, r = cfg.hidden, cfg.inter, (cfg.rank if lora else 0)
     return {
         "gemm_gate_up": 2 * R * H * 2 * I + 2 * R * 2 * I * r,
         "gemm_down": 2 * R * I * H + 2 * R * H * r,
@@ -123,9 +130,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample(wl, target_s: float):
+def oracle_sample(wl, target_s: float, infer: bool = False):
     """Time the float64 oracle on whole experts of the workload until about
-    `target_s` seconds of CPU work; returns (routed rows, seconds, experts)."""
+    `target_s` seconds of CPU work; returns (routed rows, seconds, experts).
+    infer: the base-only forward (LoRA B zeroed, no backward)."""
     import numpy as np
     from oracle import moe as omoe
     from oracle import rawint4 as orq
@@ -147,14 +155,16 @@ def oracle_sample(wl, target_s: float):
             gate_q=wl.gate_q[e:e + 1].cpu().numpy(), gate_s=bits(wl.gate_s[e:e + 1]),
             up_q=wl.up_q[e:e + 1].cpu().numpy(), up_s=bits(wl.up_s[e:e + 1]),
             down_q=wl.down_q[e:e + 1].cpu().numpy(), down_s=bits(wl.down_s[e:e + 1]),
-            lora={n: orq.bf16_bits_to_f64(bits(wl.lora[n][e:e + 1])) for n in LORA_NAMES},
+            lora={n: (0.0 if infer and n.endswith("_b") else 1.0) * orq.bf16_bits_to_f64(bits(wl.lora[n][e:e + 1]))
+                  for n in LORA_NAMES},
             alpha=wl.cfg.alpha, swiglu_limit=wl.cfg.swiglu_limit)
         x = orq.bf16_bits_to_f64(bits(wl.x[torch.as_tensor(sel, device=wl.x.device)]))
         dy = orq.bf16_bits_to_f64(bits(wl.grad_out[torch.as_tensor(sel, device=wl.x.device)]))
         rw = wl.route_weights.cpu().numpy()[sel].astype(np.float64)
         t0 = time.perf_counter()
         _, ctx = omoe.forward(layer, x, sub_ids, rw)
-        omoe.backward(layer, ctx, dy)
+        if not infer:
+            omoe.backward(layer, ctx, dy)
         spent += time.perf_counter() - t0
         rows += int(counts[e])
         used.append(e)
@@ -184,7 +194,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--experts", type=int, default=None, help="override the expert count (profiling cases)")
     ap.add_argument("--qlen", type=int, default=None, help="override the token count (profiling cases)")
+    ap.add_argument("--mode", default="train", choices=["train", "infer"],
+                    help="train: fwd+bwd step (default); infer: frozen-base inference forward")
     args = ap.parse_args()
+    infer = args.mode == "infer"
     if args.warmup < 3:
         args.warmup = 3
 
@@ -222,7 +235,7 @@ def main():
         x, ids, w, g = make_batch(cfg, seed=dp.rank_batch_seed(rank), device=dev)
         wl.x, wl.expert_ids, wl.route_weights, wl.grad_out = x, ids, w, g
     counts = expert_counts(wl.expert_ids, cfg.experts)
-    nbytes, flops, R, hit = algorithmic(cfg, counts)
+    nbytes, flops, R, hit = algorithmic(cfg, counts, infer)
     layer = B.Layer.create(cfg.experts, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank, cfg.alpha, cfg.swiglu_limit,
                            cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora)
     grads = {n: torch.zeros(s, dtype=torch.bfloat16, device=dev) for n, s in lora_shapes(cfg).items()}
@@ -232,6 +245,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        if infer:
+            layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=False, use_lora=False)
+            return
         layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=True)
         layer.backward(wl.grad_out, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
         if pg is not None:
@@ -279,7 +295,7 @@ def main():
             for n, v in per.items()}
     pk = peaks()
     dom = max((n for n in kern if n.startswith("gemm_")), key=lambda n: kern[n]["avg_ms"] * kern[n]["launches"])
-    dom_flops = gemm_flops(dom, R, cfg)
+    dom_flops = gemm_flops(dom, R, cfg, lora=not infer)
     achieved = dom_flops / (kern[dom]["avg_ms"] / 1e3) / 1e12
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
@@ -287,7 +303,7 @@ def main():
         # DRAM bytes of one launch from an ncu capture; void once the GEMM
         # sources differ from the ones the counters were taken on
         tj = json.load(open(tfile))
-        if tj.get("config") == args.config and tj.get("source_sha256_16") == gemm_source_hash():
+        if not infer and tj.get("config") == args.config and tj.get("source_sha256_16") == gemm_source_hash():
             traffic = tj.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2), "peak": pk["tflops_sustained"],
                 "unit": "TFLOP/s", "frac": round(achieved / pk["tflops_sustained"], 4), "traffic": traffic,
@@ -317,6 +333,10 @@ def main():
         d_x.copy_(h_x, non_blocking=True)
         d_ids.copy_(h_ids, non_blocking=True)
         d_w.copy_(h_w, non_blocking=True)
+        if infer:
+            layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=False, use_lora=False)
+            h_out.copy_(out, non_blocking=True)
+            return
         d_g.copy_(h_g, non_blocking=True)
         layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
         layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
@@ -338,8 +358,8 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
-    h2d = sum(t.numel() * t.element_size() for t in (h_x, h_ids, h_w, h_g))
-    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_gin, h_gr))
+    h2d = sum(t.numel() * t.element_size() for t in ((h_x, h_ids, h_w) if infer else (h_x, h_ids, h_w, h_g)))
+    d2h = sum(t.numel() * t.element_size() for t in ((h_out,) if infer else (h_out, h_gin, h_gr)))
     e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e_ms, 4),
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     return finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline,
@@ -350,15 +370,18 @@ def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_na
            launches, clocks, kern, hit):
     st = layer.status()
     cpu = None
+    infer = args.mode == "infer"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows, secs, used = oracle_sample(wl, args.cpu_seconds)
+        rows, secs, used = oracle_sample(wl, args.cpu_seconds, infer)
+        what = "base-only fwd" if infer else "fwd+bwd"
         cpu = {"value": round(rows / secs, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"float64 NumPy oracle fwd+bwd of {len(used)} whole expert(s) of this workload "
+               "sample": f"float64 NumPy oracle {what} of {len(used)} whole expert(s) of this workload "
                          f"({rows} routed rows, {secs:.1f} s)"}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_INFER if infer else METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": arm_config(cfg, world, workload_name, R, hit),
@@ -385,24 +408,27 @@ def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: in
 def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:
     """The oracle as it stands on the host cores; each step a bounded sample."""
     wl = make_workload(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+    infer = args.mode == "infer"
     per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(wl, per_step)
+        oracle_sample(wl, per_step, infer)
     rows_t, secs_t = 0, 0.0
     for _ in range(args.steps):
-        rows, secs, used = oracle_sample(wl, per_step)
+        rows, secs, used = oracle_sample(wl, per_step, infer)
         rows_t += rows
         secs_t += secs
     value = rows_t / secs_t
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    _, _, R, hit = algorithmic(cfg, expert_counts(wl.expert_ids, cfg.experts))
+    _, _, R, hit = algorithmic(cfg, expert_counts(wl.expert_ids, cfg.experts), infer)
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "impl": "reference", "metric": METRIC_INFER if infer else METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_t / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": arm_config(cfg, world, workload_name, R, hit),
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                         "sample": f"each step: float64 NumPy oracle fwd+bwd of whole experts for about {per_step:.1f} s"},
+                         "sample": f"each step: float64 NumPy oracle {'base-only fwd' if infer else 'fwd+bwd'} of whole "
+                                   f"experts for about {per_step:.1f} s"},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -138,6 +138,13 @@ RAWINT4_API int rawint4_moe_lora_workspace_size(const rawint4_moe_cfg* cfg, size
  *                 is invalidated (the scratch is shared).
  *   workspace     device buffer of at least rawint4_moe_lora_workspace_size
  *                 bytes, 256-byte aligned; ws_bytes is its size.
+ *   lora          may be NULL: frozen-base inference forward, out = the
+ *                 base-only layer (the LoRA terms are absent, as with zero
+ *                 LoRA B). It saves no context, so save_for_backward must be
+ *                 0 (RAWINT4_INVALID_ARGUMENT otherwise). This is the
+ *                 frozen-base inference kernel of the contract test
+ *                 (test_rawint4_sft_numerical.py, _run_inference_regression:
+ *                 checked against the routed reference with zero LoRA).
  * The base, LoRA and input buffers must stay valid until the enqueued work
  * completes. */
 RAWINT4_API int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base,
@@ -149,7 +156,7 @@ RAWINT4_API int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_m
  * contract test's backward(dY, dX, 6 LoRA grads, dRoute, 3 base grads,
  * accumulate, grad_scale)). It consumes the saved context: exactly one
  * backward per saving forward. cfg, base and lora must be the ones the
- * forward used.
+ * forward used; lora must not be NULL (RAWINT4_INVALID_ARGUMENT).
  *   grad_out    bf16 [Q, H] (Q of the saved forward)
  *   grad_in     bf16 [Q, H] (overwritten) = d(sum grad_out*out)/dx
  *   grad_route  fp32 [Q, k] (overwritten; may be NULL) = <grad_out[t], y_{t,s}>

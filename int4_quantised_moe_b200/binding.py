@@ -163,9 +163,11 @@ def make_grads(grads: Dict[str, torch.Tensor]) -> LoraGrads:
                                                 "down_lora_a", "down_lora_b")])
 
 
-def rawint4_moe_lora_fwd(cfg: Cfg, base: Base, lora: Lora, qlen: int, expert_ids, route_weights, x, out,
+def rawint4_moe_lora_fwd(cfg: Cfg, base: Base, lora: Optional[Lora], qlen: int, expert_ids, route_weights, x, out,
                          save_for_backward: bool, workspace: torch.Tensor, stream=None) -> None:
-    rc = _lib.rawint4_moe_lora_fwd(ctypes.byref(cfg), ctypes.byref(base), ctypes.byref(lora), int(qlen),
+    """lora=None: frozen-base inference forward (save_for_backward must be False)."""
+    lora_ref = ctypes.byref(lora) if lora is not None else None
+    rc = _lib.rawint4_moe_lora_fwd(ctypes.byref(cfg), ctypes.byref(base), lora_ref, int(qlen),
                                    _ptr(expert_ids), _ptr(route_weights), _ptr(x), _ptr(out),
                                    1 if save_for_backward else 0, _ptr(workspace), workspace.numel(),
                                    _stream(stream))
@@ -241,12 +243,13 @@ class Layer:
         lo = make_lora(lora)
         return cls(cfg, base, lo, ws, (gate_q, gate_s, up_q, up_s, down_q, down_s, dict(lora)))
 
-    def forward(self, expert_ids, route_weights, x, out=None, save_for_backward=True, stream=None):
+    def forward(self, expert_ids, route_weights, x, out=None, save_for_backward=True, stream=None, use_lora=True):
+        """use_lora=False: frozen-base inference forward (no LoRA terms, nothing saved)."""
         q = x.shape[0]
         if out is None:
             out = torch.empty_like(x)
-        rawint4_moe_lora_fwd(self.cfg, self.base, self.lora, q, expert_ids, route_weights, x, out,
-                             save_for_backward, self.workspace, stream)
+        rawint4_moe_lora_fwd(self.cfg, self.base, self.lora if use_lora else None, q, expert_ids, route_weights, x,
+                             out, save_for_backward, self.workspace, stream)
         return out
 
     def backward(self, grad_out, grads: Dict[str, torch.Tensor], accumulate=False, grad_scale=1.0, grad_in=None,

@@ -199,7 +199,8 @@ T* at(void* ws, size_t off) {
 
 int common_checks(const rawint4_moe_cfg* cfg, const rawint4_moe_base* base, const rawint4_moe_lora* lora,
                   void* workspace, size_t ws_bytes, Layout* L) {
-  if (!cfg_ok(cfg) || !base_ok(base) || !lora_ok(lora) || !workspace) return RAWINT4_INVALID_ARGUMENT;
+  // lora may be NULL (base-only forward); the entry points check where that is allowed
+  if (!cfg_ok(cfg) || !base_ok(base) || (lora && !lora_ok(lora)) || !workspace) return RAWINT4_INVALID_ARGUMENT;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return RAWINT4_INVALID_ARGUMENT;
   *L = make_layout(*cfg);
   if (ws_bytes < L->total) return RAWINT4_INVALID_ARGUMENT;
@@ -269,6 +270,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   if (rc != RAWINT4_OK) return rc;
   if (qlen < 0 || qlen > cfg->max_tokens) return RAWINT4_INVALID_ARGUMENT;
   if (qlen > 0 && (!expert_ids || !route_weights || !x || !out)) return RAWINT4_INVALID_ARGUMENT;
+  // Without LoRA the call is a frozen-base inference forward: it saves no
+  // context, so there is nothing a backward could consume.
+  const bool has_lora = lora != nullptr;
+  if (!has_lora && save_for_backward) return RAWINT4_INVALID_ARGUMENT;
   int sms = 0;
   rc = check_device(&sms);
   if (rc != RAWINT4_OK) return rc;
@@ -297,12 +302,16 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0,
                               st));
   }
-  {
+  if (has_lora) {
     R4_PROF("lora_convert", st);
     LoraCvt cv[2] = {{lora->gate_a, lora->up_a, at<uint16_t>(ws, L.gu16), r, rp, H, 0, 2},
                      {lora->down_a, nullptr, at<uint16_t>(ws, L.ad16), r, rp, I, 0, 1}};
     R4_TRY(launch_lora_convert(cv, 2, E, st));
   }
+  // Base-only forward: the GEMMs' rank stage multiplies zero side rows by a
+  // zero B operand (every row of it read from the first elements of the
+  // zeroed xa buffer), which adds exact zeros to the accumulators.
+  const uint16_t* zero_rows = at<uint16_t>(ws, L.xa);
 
   SkParams sp{};
   sp.tok_tiles = at<int4>(ws, L.tiles);
@@ -326,9 +335,12 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   sp.sw = 2 * rp;
   sp.out0 = at<uint16_t>(ws, L.xa);
   sp.out1 = nullptr;
-  {
+  if (has_lora) {
     R4_PROF("lora_xa", st);
     R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
+  } else {
+    R4_PROF("zero_xa", st);
+    R4_TRY(launch_fill_u16(at<uint16_t>(ws, L.xa), L.rows * kLoraPad, 0, st));
   }
 
   GemmMaps mp;
@@ -355,10 +367,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.s_expert = (int64_t)I * (H / 32);
   gp.s_row = H / 32;
   gp.stored_rows = I;
-  gp.lx0 = lora->gate_b;
-  gp.lx1 = lora->up_b;
-  gp.lx_expert = (int64_t)I * r;
-  gp.lx_ld = r;
+  gp.lx0 = has_lora ? lora->gate_b : zero_rows;
+  gp.lx1 = has_lora ? lora->up_b : zero_rows;
+  gp.lx_expert = has_lora ? (int64_t)I * r : 0;
+  gp.lx_ld = has_lora ? r : 0;
   gp.out_a = at<float>(ws, L.g);
   gp.out_b = at<float>(ws, L.u);
   gp.out_h = at<uint16_t>(ws, L.h);
@@ -369,16 +381,19 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // ha = c * h A_d^T and hw = w * ha
-  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.h), L.rows, I, 128) ||
-      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.ad16), E, rp, I))
-    return RAWINT4_CUDA_ERROR;
-  sp.nk = I / 64;
-  sp.sw = rp;
-  sp.out0 = at<uint16_t>(ws, L.ha);
-  sp.out1 = at<uint16_t>(ws, L.hw);
-  {
+  if (has_lora) {
+    if (!map_act(&sm.a[0], at<uint16_t>(ws, L.h), L.rows, I, 128) ||
+        !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.ad16), E, rp, I))
+      return RAWINT4_CUDA_ERROR;
+    sp.nk = I / 64;
+    sp.sw = rp;
+    sp.out0 = at<uint16_t>(ws, L.ha);
+    sp.out1 = at<uint16_t>(ws, L.hw);
     R4_PROF("lora_ha", st);
     R4_TRY(launch_skinny(kSkRows, sp, sm, rows_grid, st));
+  } else {
+    R4_PROF("zero_ha", st);
+    R4_TRY(launch_fill_u16(at<uint16_t>(ws, L.ha), L.rows * kLoraPad, 0, st));
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
@@ -392,9 +407,9 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.s_expert = (int64_t)H * (I / 32);
   gp.s_row = I / 32;
   gp.stored_rows = H;
-  gp.lx0 = gp.lx1 = lora->down_b;
-  gp.lx_expert = (int64_t)H * r;
-  gp.lx_ld = r;
+  gp.lx0 = gp.lx1 = has_lora ? lora->down_b : zero_rows;
+  gp.lx_expert = has_lora ? (int64_t)H * r : 0;
+  gp.lx_ld = has_lora ? r : 0;
   gp.out_a = at<float>(ws, L.y);
   gp.out_b = nullptr;
   gp.out_h = nullptr;
@@ -417,6 +432,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
                          void* stream_) {
   // The base is frozen: refuse any base-gradient buffer before touching anything.
   if (base_grad_gate || base_grad_up || base_grad_down) return RAWINT4_FROZEN_BASE;
+  if (!lora) return RAWINT4_INVALID_ARGUMENT;  // the backward trains the LoRA adapters
   Layout L;
   int rc = common_checks(cfg, base, lora, workspace, ws_bytes, &L);
   if (rc != RAWINT4_OK) return rc;

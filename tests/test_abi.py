@@ -91,3 +91,22 @@ def test_host_argument_errors(lib):
     assert cdll.rawint4_moe_permute_workspace_size(5, 0, 4, ctypes.byref(n)) == lib.INVALID_ARGUMENT
     for code in range(0, 9):
         assert lib.strerror(code) != "unknown status code"
+
+
+def test_base_only_forward_cannot_save(lib):
+    """lora = NULL selects the frozen-base inference forward, which saves no
+    context: save_for_backward = 1 is an argument error, and so is a backward
+    without LoRA. Both are caught on the host before anything is enqueued, so
+    the placeholder pointers are never dereferenced."""
+    cdll = lib.library()
+    cfg = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 32)
+    nbytes = lib.rawint4_moe_lora_workspace_size(cfg)
+    fake = 4096  # aligned, never dereferenced
+    base = lib.Base(*([fake] * 6))
+    rc = cdll.rawint4_moe_lora_fwd(ctypes.byref(cfg), ctypes.byref(base), None, 5, fake, fake, fake, fake, 1, fake,
+                                   nbytes, None)
+    assert rc == lib.INVALID_ARGUMENT
+    grads = lib.LoraGrads(*([fake] * 6))
+    rc = cdll.rawint4_moe_lora_bwd(ctypes.byref(cfg), ctypes.byref(base), None, fake, fake, None, ctypes.byref(grads),
+                                   None, None, None, 0, 1.0, fake, nbytes, None)
+    assert rc == lib.INVALID_ARGUMENT

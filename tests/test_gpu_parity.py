@@ -5,8 +5,8 @@ lifecycle (test_rawint4_sft_numerical.py: GAS1 overwrite with sentinel
 buffers, accumulation, the lazy clear of a new window, checkpoint-recompute
 cache replacement, frozen-base fail-fast, base bytes unchanged), the
 clamp-boundary fixture, the rectangular multiblock variant, the inference
-regression with zero LoRA, bad expert ids, qlen = 0 and a missing saved
-forward.
+regression with zero LoRA, the base-only (lora = NULL) inference forward, bad
+expert ids, qlen = 0 and a missing saved forward.
 """
 
 import hashlib
@@ -239,6 +239,32 @@ def test_inference_regression_zero_lora():
     layer = make_layer(g)
     out = layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False)
     close("inference.out", out, out_r, TOL_OUT)
+
+
+def test_base_only_inference_forward():
+    """lora = NULL: the frozen-base inference forward. Its output equals, bit
+    for bit, the LoRA forward with every LoRA B zeroed (the rank stage then adds
+    exact zeros to the accumulators), is close to the oracle's base-only layer,
+    leaves the base bytes unchanged, and refuses to save a context."""
+    from tests._gpu import B
+    wl = make_workload(CONFIGS[1])
+    zero_b = {n: (torch.zeros_like(t) if n.endswith("_b") else t) for n, t in wl.lora.items()}
+    zb = Workload(wl.cfg, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, zero_b, wl.x,
+                  wl.expert_ids, wl.route_weights, wl.grad_out)
+    out_r, _ = omoe.forward(oracle_layer(zb), f64(zb.x), zb.expert_ids.numpy(), f64(zb.route_weights))
+    g = on_gpu(wl)
+    before = base_hash(g)
+    layer = make_layer(g)
+    out = layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False, use_lora=False)
+    assert layer.status() == 0
+    close("base_only.out", out, out_r, TOL_OUT)
+    gz = on_gpu(zb)
+    out_z = make_layer(gz).forward(gz.expert_ids, gz.route_weights, gz.x, save_for_backward=False)
+    assert torch.equal(out.view(torch.int16), out_z.view(torch.int16))
+    with pytest.raises(B.RawInt4Error) as ei:
+        layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=True, use_lora=False)
+    assert ei.value.code == B.INVALID_ARGUMENT
+    assert base_hash(g) == before
 
 
 def test_bad_expert_id_and_status():
