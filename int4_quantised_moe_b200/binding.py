@@ -223,6 +223,32 @@ def rawint4_moe_permute_static_max_bytes() -> int:
 # and one workspace together and calls the two entry points.
 # ---------------------------------------------------------------------------
 
+def _expect(t, name: str, dtype: torch.dtype, shape: tuple, device: Optional[torch.device] = None) -> None:
+    """Host-side argument check: the C ABI sees raw pointers only, so a wrong
+    dtype, shape, device or layout is caught here with a readable message."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected a tensor on {device}, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: tensors passed to the layer must be contiguous")
+
+
+LORA_TENSOR_NAMES = ("gate_lora_a", "gate_lora_b", "up_lora_a", "up_lora_b", "down_lora_a", "down_lora_b")
+
+
+def lora_tensor_shapes(experts: int, hidden: int, inter: int, rank: int) -> Dict[str, tuple]:
+    """Shapes of the six LoRA tensors (and of their gradient buffers)."""
+    E, H, I, r = experts, hidden, inter, rank
+    return {"gate_lora_a": (E, r, H), "gate_lora_b": (E, I, r), "up_lora_a": (E, r, H), "up_lora_b": (E, I, r),
+            "down_lora_a": (E, r, I), "down_lora_b": (E, H, r)}
+
 @dataclass
 class Layer:
     cfg: Cfg
@@ -235,8 +261,20 @@ class Layer:
     def create(cls, experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens, gate_q, gate_s, up_q, up_s,
                down_q, down_s, lora: Dict[str, torch.Tensor], device=None):
         cfg = make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens)
-        nbytes = rawint4_moe_lora_workspace_size(cfg)
+        nbytes = rawint4_moe_lora_workspace_size(cfg)  # validates the configuration
         dev = device if device is not None else gate_q.device
+        E, H, I = int(experts), int(hidden), int(inter)
+        for name, t, dt, shape in (("gate_q", gate_q, torch.uint8, (E, I, H // 2)),
+                                   ("up_q", up_q, torch.uint8, (E, I, H // 2)),
+                                   ("down_q", down_q, torch.uint8, (E, H, I // 2)),
+                                   ("gate_s", gate_s, torch.bfloat16, (E, I, H // 32)),
+                                   ("up_s", up_s, torch.bfloat16, (E, I, H // 32)),
+                                   ("down_s", down_s, torch.bfloat16, (E, H, I // 32))):
+            _expect(t, name, dt, shape, gate_q.device)
+        for name, shape in lora_tensor_shapes(E, H, I, int(rank)).items():
+            if name not in lora:
+                raise KeyError(f"lora: missing {name}")
+            _expect(lora[name], name, torch.bfloat16, shape, gate_q.device)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         ws[:256].zero_()
         base = make_base(gate_q, gate_s, up_q, up_s, down_q, down_s)
@@ -245,17 +283,33 @@ class Layer:
 
     def forward(self, expert_ids, route_weights, x, out=None, save_for_backward=True, stream=None, use_lora=True):
         """use_lora=False: frozen-base inference forward (no LoRA terms, nothing saved)."""
-        q = x.shape[0]
+        q, k, H = x.shape[0] if x.dim() == 2 else -1, self.cfg.top_k, self.cfg.hidden
+        dev = self.workspace.device
+        _expect(x, "x", torch.bfloat16, (q, H), dev)
+        _expect(expert_ids, "expert_ids", torch.int64, (q, k), dev)
+        _expect(route_weights, "route_weights", torch.float32, (q, k), dev)
         if out is None:
             out = torch.empty_like(x)
+        _expect(out, "out", torch.bfloat16, (q, H), dev)
         rawint4_moe_lora_fwd(self.cfg, self.base, self.lora if use_lora else None, q, expert_ids, route_weights, x,
                              out, save_for_backward, self.workspace, stream)
         return out
 
     def backward(self, grad_out, grads: Dict[str, torch.Tensor], accumulate=False, grad_scale=1.0, grad_in=None,
                  grad_route=None, stream=None, **base_grads):
+        dev = self.workspace.device
+        q, k, H = grad_out.shape[0] if grad_out.dim() == 2 else -1, self.cfg.top_k, self.cfg.hidden
+        _expect(grad_out, "grad_out", torch.bfloat16, (q, H), dev)
         if grad_in is None:
             grad_in = torch.empty_like(grad_out)
+        _expect(grad_in, "grad_in", torch.bfloat16, (q, H), dev)
+        if grad_route is not None:
+            _expect(grad_route, "grad_route", torch.float32, (q, k), dev)
+        c = self.cfg
+        for name, shape in lora_tensor_shapes(c.experts, c.hidden, c.inter, c.rank).items():
+            if name not in grads:
+                raise KeyError(f"grads: missing {name}")
+            _expect(grads[name], f"grads[{name}]", torch.bfloat16, shape, dev)
         rawint4_moe_lora_bwd(self.cfg, self.base, self.lora, grad_out, grad_in, grad_route, make_grads(grads),
                              accumulate, grad_scale, self.workspace, stream, **base_grads)
         return grad_in

@@ -110,3 +110,31 @@ def test_base_only_forward_cannot_save(lib):
     rc = cdll.rawint4_moe_lora_bwd(ctypes.byref(cfg), ctypes.byref(base), None, fake, fake, None, ctypes.byref(grads),
                                    None, None, None, 0, 1.0, fake, nbytes, None)
     assert rc == lib.INVALID_ARGUMENT
+
+
+def test_binding_rejects_wrong_tensors(lib):
+    """The binding checks dtype, shape, device and layout before any C call,
+    so a wrong tensor fails with a readable message instead of reaching the
+    kernels as a raw pointer. Runs on CPU: every case fails before the
+    workspace is allocated."""
+    E, k, H, I, r = 4, 2, 256, 256, 8
+    shapes = lib.lora_tensor_shapes(E, H, I, r)
+    lora = {n: torch.zeros(s, dtype=torch.bfloat16) for n, s in shapes.items()}
+    q = dict(gate_q=torch.zeros((E, I, H // 2), dtype=torch.uint8), gate_s=torch.zeros((E, I, H // 32), dtype=torch.bfloat16),
+             up_q=torch.zeros((E, I, H // 2), dtype=torch.uint8), up_s=torch.zeros((E, I, H // 32), dtype=torch.bfloat16),
+             down_q=torch.zeros((E, H, I // 2), dtype=torch.uint8), down_s=torch.zeros((E, H, I // 32), dtype=torch.bfloat16))
+
+    def create(**over):
+        a = dict(q, **over)
+        return lib.Layer.create(E, k, H, I, r, 16.0, 0.0, 8, a["gate_q"], a["gate_s"], a["up_q"], a["up_s"],
+                                a["down_q"], a["down_s"], over.get("lora", lora))
+
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        create()
+    # the first tensor checked is gate_q: dtype, then shape, then device
+    with pytest.raises(TypeError, match="dtype"):
+        create(gate_q=torch.zeros((E, I, H // 2), dtype=torch.int8))
+    with pytest.raises(ValueError, match="shape"):
+        create(gate_q=torch.zeros((E, I, H // 4), dtype=torch.uint8))
+    with pytest.raises(lib.RawInt4Error):
+        lib.Layer.create(E, k, 200, I, r, 16.0, 0.0, 8, *q.values(), lora)  # H not a multiple of 128
