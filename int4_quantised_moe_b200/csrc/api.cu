@@ -4,6 +4,7 @@
 // (test_rawint4_sft_numerical.py, _forward and _backward).
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "aux.cuh"
@@ -215,14 +216,15 @@ int grid_for_tiles(int sms, int max_tiles, int rowblk) {
 // CTA pairs for a pair-kernel launch: all that fit at once, or fewer for a small
 // problem (work items = token tiles x feature blocks).
 int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
-  static int cached[64][4];
+  static std::atomic<int> cached[64][4];  // per device and mode; 0 = not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (cached[dev][mode] <= 0) {
+  int fit = cached[dev][mode].load();
+  if (fit <= 0) {
     const int n = gemm_pair_max_clusters(mode);
-    cached[dev][mode] = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
+    fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
+    cached[dev][mode].store(fit);
   }
-  const int fit = cached[dev][mode];
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }

@@ -16,4 +16,8 @@ struct ProfScope {
 
 }  // namespace r4
 
-#define R4_PROF(name, stream) ::r4::ProfScope r4_prof_scope_##__LINE__(name, stream)
+// One scope object per use, named after the line (two-level paste so that
+// __LINE__ expands before it is pasted).
+#define R4_PROF_CAT2(a, b) a##b
+#define R4_PROF_CAT(a, b) R4_PROF_CAT2(a, b)
+#define R4_PROF(name, stream) ::r4::ProfScope R4_PROF_CAT(r4_prof_scope_, __LINE__)(name, stream)
