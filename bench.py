@@ -85,6 +85,31 @@ def gemm_flops(name: str, R: int, cfg: LayerConfig, lora: bool = True) -> float:
     }.get(name, 0.0)
 
 
+def phase_times(launches, steps: int) -> dict:
+    """Kernel time per step of the forward and of the backward launches (the
+    per-launch CUDA events, in issue order): a step's backward runs from its
+    header_bwd launch up to the next header_fwd."""
+    fwd = bwd = 0.0
+    in_bwd = False
+    for name, ms in launches:
+        if name == "header_fwd":
+            in_bwd = False
+        elif name == "header_bwd":
+            in_bwd = True
+        if in_bwd:
+            bwd += ms
+        else:
+            fwd += ms
+    n = max(1, steps)
+    return {"fwd_kernel_ms": round(fwd / n, 4), "bwd_kernel_ms": round(bwd / n, 4)}
+
+
+def count_stats(counts: torch.Tensor) -> dict:
+    """Realised routed rows per expert: min, median, max and empty experts."""
+    c = counts.to(torch.int64)
+    return {"min": int(c.min()), "median": float(c.double().median()), "max": int(c.max()), "empty": int((c == 0).sum())}
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
 
@@ -384,9 +409,10 @@ def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_na
             "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": arm_config(cfg, world, workload_name, R, hit),
+            "config": arm_config(cfg, world, workload_name, R, hit, expert_counts(wl.expert_ids, cfg.experts)),
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": len(launches), "clocks": clocks, "device_status": st,
+            "gpu_launches": len(launches), "phases": phase_times(launches, args.steps), "clocks": clocks,
+            "device_status": st,
             "kernels": {n: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 4), "share": round(v["share"], 4)}
                         for n, v in sorted(kern.items(), key=lambda kv: -kv[1]["share"])},
         }
@@ -397,10 +423,11 @@ def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_na
     return 0
 
 
-def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: int) -> dict:
+def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: int, counts: torch.Tensor) -> dict:
     """The `config` object of the JSON line, shared by both arms."""
     return {"workload": workload_name, "parallelism": f"dp{world}" if world > 1 else "single",
             "global_batch_tokens": cfg.qlen * world, "routed_rows_per_gpu": R,
+            "expert_rows": count_stats(counts),
             "l2": "inputs larger than L2: every step streams all hit experts' packed weights "
                   f"({2 * hit * 3 * cfg.hidden * cfg.inter * (0.5 + 1 / 16) / 1e9:.1f} GB)"}
 
@@ -419,13 +446,14 @@ def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:
         secs_t += secs
     value = rows_t / secs_t
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    _, _, R, hit = algorithmic(cfg, expert_counts(wl.expert_ids, cfg.experts), infer)
+    counts = expert_counts(wl.expert_ids, cfg.experts)
+    _, _, R, hit = algorithmic(cfg, counts, infer)
     line = {
         "impl": "reference", "metric": METRIC_INFER if infer else METRIC, "value": round(value, 2), "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_t / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": arm_config(cfg, world, workload_name, R, hit),
+        "config": arm_config(cfg, world, workload_name, R, hit, counts),
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                          "sample": f"each step: float64 NumPy oracle {'base-only fwd' if infer else 'fwd+bwd'} of whole "
                                    f"experts for about {per_step:.1f} s"},

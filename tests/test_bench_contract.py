@@ -39,3 +39,23 @@ def test_reference_arm_line(mode):
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_reports_expert_rows():
+    d = _run()
+    er = d["config"]["expert_rows"]
+    assert set(er) == {"min", "median", "max", "empty"}
+    assert 0 <= er["min"] <= er["median"] <= er["max"] and 0 <= er["empty"] <= 4
+
+
+def test_phase_split_of_launches():
+    """Forward and backward kernel time per step from the launch list in issue order."""
+    sys.path.insert(0, ROOT)
+    import bench
+    step = [("header_fwd", 0.01), ("route", 0.05), ("gemm_gate_up", 5.0), ("gemm_down", 3.0), ("combine_out", 0.3),
+            ("header_bwd", 0.01), ("gemm_down_t", 3.5), ("gemm_gate_up_t", 5.0), ("lora_grads", 1.0),
+            ("header_end", 0.01)]
+    ph = bench.phase_times(step * 2, 2)
+    assert ph == {"fwd_kernel_ms": 8.36, "bwd_kernel_ms": 9.52}
+    inf = [("header_fwd", 0.01), ("gemm_gate_up", 5.0), ("gemm_down", 3.0)] * 3
+    assert bench.phase_times(inf, 3) == {"fwd_kernel_ms": 8.01, "bwd_kernel_ms": 0.0}
