@@ -59,3 +59,26 @@ def test_phase_split_of_launches():
     assert ph == {"fwd_kernel_ms": 8.36, "bwd_kernel_ms": 9.52}
     inf = [("header_fwd", 0.01), ("gemm_gate_up", 5.0), ("gemm_down", 3.0)] * 3
     assert bench.phase_times(inf, 3) == {"fwd_kernel_ms": 8.01, "bwd_kernel_ms": 0.0}
+
+
+def test_reference_arm_under_torchrun():
+    """Launched the way the driver launches N > 1 (torchrun, one process per
+    rank): rank 0 alone runs the oracle and prints the line, with n_gpus = N;
+    the other ranks exit 0 without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.join(ROOT, "bench.py"),
+           "--gpus", "2", "--impl", "reference", "--config", "0", "--steps", "1", "--warmup", "3", "--cpu-seconds", "0.2"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="1")
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
