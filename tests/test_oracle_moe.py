@@ -294,3 +294,29 @@ def test_config0_runs_and_has_signal():
     gin, groute, grads = omoe.backward(layer, ctx, f64(wl.grad_out))
     for arr in [out, gin, groute] + list(grads.values()):
         assert np.all(np.isfinite(arr)) and np.count_nonzero(arr)
+
+
+def test_duplicate_expert_slots_are_independent():
+    """A token routed twice to the same expert (top-k never does this, the
+    layer accepts it): the forward is linear in the route weights, so slots
+    (e, w1), (e, w2) give the output of one slot (e, w1 + w2) next to a
+    zero-weight slot; both duplicate slots see the same dRoute = <dY, y_e>,
+    and the LoRA gradients are those of the merged slot."""
+    wl = _tiny(seed=11)
+    layer = oracle_layer(wl)
+    Q = wl.cfg.qlen
+    x, dy = f64(wl.x), f64(wl.grad_out)
+    dup = np.array([[t % 4, t % 4] for t in range(Q)], dtype=np.int64)
+    w = np.stack([np.linspace(0.2, 0.7, Q), np.linspace(0.5, 0.1, Q)], 1)
+    merged = np.array([[t % 4, (t + 1) % 4] for t in range(Q)], dtype=np.int64)
+    wm = np.stack([w[:, 0] + w[:, 1], np.zeros(Q)], 1)
+    out_d, ctx_d = omoe.forward(layer, x, dup, w)
+    out_m, ctx_m = omoe.forward(layer, x, merged, wm)
+    np.testing.assert_allclose(out_d, out_m, rtol=1e-12, atol=1e-12)
+    gin_d, gr_d, gd = omoe.backward(layer, ctx_d, dy)
+    gin_m, gr_m, gm = omoe.backward(layer, ctx_m, dy)
+    np.testing.assert_allclose(gin_d, gin_m, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(gr_d[:, 0], gr_d[:, 1], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gr_d[:, 0], gr_m[:, 0], rtol=1e-12, atol=1e-12)
+    for n in LORA_NAMES:
+        np.testing.assert_allclose(gd[n], gm[n], rtol=1e-11, atol=1e-11)
