@@ -338,8 +338,8 @@ __device__ __forceinline__ bool wait_all_cl(uint64_t* bar, uint32_t parity, vola
   return __all_sync(0xffffffffu, ok);
 }
 // Tiled TMA load into this CTA's shared memory whose completion is counted on
-// an mbarrier of either CTA of the pair (shared::cluster address). No
-// multicast: each CTA loads only its own tile.
+// an mbarrier of either CTA of the pair (shared::cluster address). Each CTA
+// loads only its own tile, from this GPU's memory, into its own shared memory.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t c0,
                                                  int32_t c1) {
   asm volatile(
