@@ -207,6 +207,94 @@ def cpu_cores() -> int:
 
 # --------------------------------------------------------------------- main
 
+def peak_basis(clocks: dict) -> str:
+    """Which measured tensor peak a kernel timed in this run is compared with:
+    the burst figure when the SM clock held within 5 % of its maximum during the
+    timed region, the sustained (power-capped) figure otherwise."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm is None or mx is None or mx <= 0:
+        return "burst"
+    return "burst" if sm >= 0.95 * mx else "sustained"
+
+
+def rooflines(kern: dict, R: int, cfg: LayerConfig, infer: bool, nbytes: float, flops: float, ms_step: float,
+              clocks: dict, config_index: int):
+    """Dominant-GEMM roofline and whole-step roofline against the measured peaks."""
+    pk = peaks()
+    basis = peak_basis(clocks)
+    p_t = pk["tflops"] if basis == "burst" else pk["tflops_sustained"]
+    dom = max((n for n in kern if n.startswith("gemm_")), key=lambda n: kern[n]["avg_ms"] * kern[n]["launches"])
+    dom_flops = gemm_flops(dom, R, cfg, lora=not infer)
+    achieved = dom_flops / (kern[dom]["avg_ms"] / 1e3) / 1e12
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        # DRAM bytes of one launch from an ncu capture; void once the GEMM
+        # sources differ from the ones the counters were taken on
+        tj = json.load(open(tfile))
+        if not infer and tj.get("config") == config_index and tj.get("source_sha256_16") == gemm_source_hash():
+            traffic = tj.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2), "peak": p_t, "unit": "TFLOP/s",
+                "frac": round(achieved / p_t, 4), "traffic": traffic,
+                "frac_burst": round(achieved / pk["tflops"], 4),
+                "frac_sustained": round(achieved / pk["tflops_sustained"], 4),
+                "peak_source": f"{pk['source']} bf16 {basis} (SM clock median {clocks.get('sm_mhz')} of "
+                               f"{clocks.get('sm_max_mhz')} MHz; fp16 dense rate equals bf16)"}
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9) * 1e3
+    t_tc = flops / (p_t * 1e12) * 1e3
+    t_roof = max(t_hbm, t_tc)
+    step = {"bound": "tensor" if t_tc > t_hbm else "hbm", "t_roof_ms": round(t_roof, 4),
+            "frac": round(t_roof / ms_step, 4), "peak_basis": basis,
+            "frac_burst": round(max(t_hbm, flops / (pk["tflops"] * 1e12) * 1e3) / ms_step, 4),
+            "frac_sustained": round(max(t_hbm, flops / (pk["tflops_sustained"] * 1e12) * 1e3) / ms_step, 4),
+            "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
+            "achieved_hbm_gbs": round(nbytes / (ms_step / 1e3) / 1e9, 1),
+            "hbm_frac": round(nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+            "routed_rows": R}
+    return roofline, step
+
+
+def kernel_table(launches) -> dict:
+    per = {}
+    for name, ms in launches:
+        per.setdefault(name, []).append(ms)
+    tot = max(1e-9, sum(sum(v) for v in per.values()))
+    return {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "share": sum(v) / tot} for n, v in per.items()}
+
+
+def kernel_summary(kern: dict) -> dict:
+    return {n: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 4), "share": round(v["share"], 4)}
+            for n, v in sorted(kern.items(), key=lambda kv: -kv[1]["share"])}
+
+
+def device_timed(step, steps: int, warmup: int, layer, B, dev, stream, barrier, max_over_ranks):
+    """W warm-up steps, then K steps between CUDA events on the launching
+    stream, with the library's per-launch events and the sampled SM clocks."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = layer.status()
+    if st:
+        raise RuntimeError(f"device status after warm-up: {st:#x}")
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index or 0)
+    time.sleep(0.3)
+    B.profile_begin(64 * steps)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = B.profile_end(64 * steps)
+    clocks = sampler.stop()
+    barrier()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    return ms_total / steps, launches, clocks
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -217,6 +305,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the extra measurements of the memory-bound and skewed layers")
     ap.add_argument("--experts", type=int, default=None, help="override the expert count (profiling cases)")
     ap.add_argument("--qlen", type=int, default=None, help="override the token count (profiling cases)")
     ap.add_argument("--mode", default="train", choices=["train", "infer"],
@@ -234,8 +324,7 @@ def main():
         import dataclasses
         cfg = dataclasses.replace(cfg, name=cfg.name + "_override", experts=args.experts or cfg.experts,
                                   qlen=args.qlen or cfg.qlen)
-    workload_name = (f"{cfg.name}: E={cfg.experts} top_k={cfg.top_k} H={cfg.hidden} I={cfg.inter} r={cfg.rank} "
-                     f"alpha={cfg.alpha:g} qlen={cfg.qlen} swiglu_limit={cfg.swiglu_limit:g} routing={cfg.routing}")
+    workload_name = describe(cfg)
 
     if args.impl == "reference":
         if rank != 0:
@@ -253,6 +342,13 @@ def main():
 
     from int4_quantised_moe_b200 import binding as B
     from int4_quantised_moe_b200 import dp
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        return dp.max_over_ranks(v, device=dev)
 
     # layer (same on every rank) and this rank's batch
     wl = make_workload(cfg, device=dev)
@@ -278,149 +374,131 @@ def main():
         if pg is not None:
             dp.allreduce_lora_grads(grads)
 
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        return dp.max_over_ranks(v, device=dev)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    st = layer.status()
-    if st:
-        raise RuntimeError(f"device status after warm-up: {st:#x}")
-
     # ---- device-timed region (inputs resident in HBM) with per-launch events
-    barrier()
-    torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local)
-    time.sleep(0.3)
-    B.profile_begin(64 * args.steps)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for _ in range(args.steps):
-        step()
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    launches = B.profile_end(64 * args.steps)
-    clocks = sampler.stop()
-    barrier()
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
-    ms_step = ms_total / args.steps
+    ms_step, launches, clocks = device_timed(step, args.steps, args.warmup, layer, B, dev, stream, barrier,
+                                             max_over_ranks)
     value = cfg.qlen * cfg.top_k * world / (ms_step / 1e3)
-
-    # per-kernel averages and the dominant kernel's roofline
-    per = {}
-    for name, ms in launches:
-        per.setdefault(name, []).append(ms)
-    kern = {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "share": sum(v) / max(1e-9, sum(sum(x) for x in per.values()))}
-            for n, v in per.items()}
-    pk = peaks()
-    dom = max((n for n in kern if n.startswith("gemm_")), key=lambda n: kern[n]["avg_ms"] * kern[n]["launches"])
-    dom_flops = gemm_flops(dom, R, cfg, lora=not infer)
-    achieved = dom_flops / (kern[dom]["avg_ms"] / 1e3) / 1e12
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tfile):
-        # DRAM bytes of one launch from an ncu capture; void once the GEMM
-        # sources differ from the ones the counters were taken on
-        tj = json.load(open(tfile))
-        if not infer and tj.get("config") == args.config and tj.get("source_sha256_16") == gemm_source_hash():
-            traffic = tj.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2), "peak": pk["tflops_sustained"],
-                "unit": "TFLOP/s", "frac": round(achieved / pk["tflops_sustained"], 4), "traffic": traffic,
-                "peak_source": f"{pk['source']} bf16 sustained (fp16 dense rate equals bf16)"}
-    t_roof = max(nbytes / (pk["hbm_gbs"] * 1e9), flops / (pk["tflops_sustained"] * 1e12)) * 1e3
-    step_roofline = {"bound": "tensor" if flops / pk["tflops_sustained"] / 1e12 > nbytes / pk["hbm_gbs"] / 1e9 else "hbm",
-                     "t_roof_ms": round(t_roof, 4), "frac": round(t_roof / ms_step, 4),
-                     "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
-                     "routed_rows": R, "experts_hit": hit}
+    kern = kernel_table(launches)
+    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, args.config)
+    step_roofline["experts_hit"] = hit
 
     # ---- end to end through the public API from pinned host buffers
     e2e = None
-    if args.no_e2e:
-        return finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline,
-                      e2e, launches, clocks, kern, hit)
-    h_x = wl.x.cpu().pin_memory()
-    h_ids = wl.expert_ids.cpu().pin_memory()
-    h_w = wl.route_weights.cpu().pin_memory()
-    h_g = wl.grad_out.cpu().pin_memory()
-    h_out = torch.empty_like(h_x).pin_memory()
-    h_gin = torch.empty_like(h_x).pin_memory()
-    h_gr = torch.empty(groute.shape, dtype=torch.float32).pin_memory()
-    d_x, d_ids, d_w, d_g = torch.empty_like(wl.x), torch.empty_like(wl.expert_ids), torch.empty_like(
-        wl.route_weights), torch.empty_like(wl.grad_out)
+    if not args.no_e2e:
+        h_x = wl.x.cpu().pin_memory()
+        h_ids = wl.expert_ids.cpu().pin_memory()
+        h_w = wl.route_weights.cpu().pin_memory()
+        h_g = wl.grad_out.cpu().pin_memory()
+        h_out = torch.empty_like(h_x).pin_memory()
+        h_gin = torch.empty_like(h_x).pin_memory()
+        h_gr = torch.empty(groute.shape, dtype=torch.float32).pin_memory()
+        d_x, d_ids, d_w, d_g = torch.empty_like(wl.x), torch.empty_like(wl.expert_ids), torch.empty_like(
+            wl.route_weights), torch.empty_like(wl.grad_out)
 
-    def e2e_step():
-        d_x.copy_(h_x, non_blocking=True)
-        d_ids.copy_(h_ids, non_blocking=True)
-        d_w.copy_(h_w, non_blocking=True)
-        if infer:
-            layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=False, use_lora=False)
+        def e2e_step():
+            d_x.copy_(h_x, non_blocking=True)
+            d_ids.copy_(h_ids, non_blocking=True)
+            d_w.copy_(h_w, non_blocking=True)
+            if infer:
+                layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=False, use_lora=False)
+                h_out.copy_(out, non_blocking=True)
+                return
+            d_g.copy_(h_g, non_blocking=True)
+            layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
+            layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
+            if pg is not None:
+                dp.allreduce_lora_grads(grads)
             h_out.copy_(out, non_blocking=True)
-            return
-        d_g.copy_(h_g, non_blocking=True)
-        layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
-        layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
-        if pg is not None:
-            dp.allreduce_lora_grads(grads)
-        h_out.copy_(out, non_blocking=True)
-        h_gin.copy_(gin, non_blocking=True)
-        h_gr.copy_(groute, non_blocking=True)
+            h_gin.copy_(gin, non_blocking=True)
+            h_gr.copy_(groute, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(args.steps):
         e2e_step()
-    e_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
-    h2d = sum(t.numel() * t.element_size() for t in ((h_x, h_ids, h_w) if infer else (h_x, h_ids, h_w, h_g)))
-    d2h = sum(t.numel() * t.element_size() for t in ((h_out,) if infer else (h_out, h_gin, h_gr)))
-    e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e_ms, 4),
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    return finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline,
-                  e2e, launches, clocks, kern, hit)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_end = torch.cuda.Event(enable_timing=True)
+        e_start.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
+        h2d = sum(t.numel() * t.element_size() for t in ((h_x, h_ids, h_w) if infer else (h_x, h_ids, h_w, h_g)))
+        d2h = sum(t.numel() * t.element_size() for t in ((h_out,) if infer else (h_out, h_gin, h_gr)))
+        e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT,
+               "ms_per_step": round(e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-
-def finish(args, cfg, world, rank, pg, layer, wl, value, ms_step, R, workload_name, roofline, step_roofline, e2e,
-           launches, clocks, kern, hit):
     st = layer.status()
     cpu = None
-    infer = args.mode == "infer"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows, secs, used = oracle_sample(wl, args.cpu_seconds, infer)
         what = "base-only fwd" if infer else "fwd+bwd"
         cpu = {"value": round(rows / secs, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                "sample": f"float64 NumPy oracle {what} of {len(used)} whole expert(s) of this workload "
                          f"({rows} routed rows, {secs:.1f} s)"}
+    cfg_obj = arm_config(cfg, world, workload_name, R, hit, counts)
+    del layer, wl, grads, out, gin, groute
+    torch.cuda.empty_cache()
+
+    # ---- the memory-bound and the skewed layer, and the base-only forward of
+    # the memory-bound one (one GPU, default workload only)
+    others = None
+    if world == 1 and args.config == 4 and args.experts is None and args.qlen is None and not args.no_other_configs:
+        others = [other_config(c, m, B, dev, stream) for c, m in ((2, "train"), (3, "train"), (2, "infer"))]
 
     if rank == 0:
         line = {
             "metric": METRIC_INFER if infer else METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": arm_config(cfg, world, workload_name, R, hit, expert_counts(wl.expert_ids, cfg.experts)),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": cfg_obj,
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": len(launches), "phases": phase_times(launches, args.steps), "clocks": clocks,
-            "device_status": st,
-            "kernels": {n: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 4), "share": round(v["share"], 4)}
-                        for n, v in sorted(kern.items(), key=lambda kv: -kv[1]["share"])},
+            "device_status": st, "kernels": kernel_summary(kern), "other_configs": others,
         }
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def describe(cfg: LayerConfig) -> str:
+    return (f"{cfg.name}: E={cfg.experts} top_k={cfg.top_k} H={cfg.hidden} I={cfg.inter} r={cfg.rank} "
+            f"alpha={cfg.alpha:g} qlen={cfg.qlen} swiglu_limit={cfg.swiglu_limit:g} routing={cfg.routing}")
+
+
+def other_config(index: int, mode: str, B, dev, stream, steps: int = 10, warmup: int = 3) -> dict:
+    """Device-timed steps of another workload (no e2e pass, no CPU baseline)."""
+    cfg = CONFIGS[index]
+    infer = mode == "infer"
+    wl = make_workload(cfg, device=dev)
+    counts = expert_counts(wl.expert_ids, cfg.experts)
+    nbytes, flops, R, hit = algorithmic(cfg, counts, infer)
+    layer = B.Layer.create(cfg.experts, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank, cfg.alpha, cfg.swiglu_limit,
+                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora)
+    grads = {n: torch.zeros(s, dtype=torch.bfloat16, device=dev) for n, s in lora_shapes(cfg).items()}
+    out = torch.empty_like(wl.x)
+    gin = torch.empty_like(wl.x)
+    groute = torch.empty(wl.expert_ids.shape, dtype=torch.float32, device=dev)
+
+    def step():
+        if infer:
+            layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=False, use_lora=False)
+            return
+        layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=True)
+        layer.backward(wl.grad_out, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
+
+    ms_step, launches, clocks = device_timed(step, steps, warmup, layer, B, dev, stream, lambda: None, lambda v: v)
+    kern = kernel_table(launches)
+    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, index)
+    res = {"workload": describe(cfg), "mode": mode, "steps": steps, "warmup": warmup,
+           "ms_per_step": round(ms_step, 4), "value": round(cfg.qlen * cfg.top_k / (ms_step / 1e3), 1), "unit": UNIT,
+           "expert_rows": count_stats(counts), "experts_hit": hit, "step_roofline": step_roofline,
+           "roofline": roofline, "clocks": clocks, "device_status": layer.status(), "kernels": kernel_summary(kern)}
+    del layer, wl, grads, out, gin, groute
+    torch.cuda.empty_cache()
+    return res
 
 
 def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: int, counts: torch.Tensor) -> dict:

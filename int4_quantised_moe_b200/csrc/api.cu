@@ -103,10 +103,14 @@ bool grads_ok(const rawint4_moe_lora_grads* g) {
   return g && a16(g->gate_a) && a16(g->gate_b) && a16(g->up_a) && a16(g->up_b) && a16(g->down_a) && a16(g->down_b);
 }
 
+}  // namespace
+
 // --------------------------------------------------------------- device
+namespace {
 std::mutex g_mu;
 int g_checked_device = -1;
 int g_sm_count = 0;
+}  // namespace
 
 int check_device(int* sms) {
   int dev = 0;
@@ -125,6 +129,8 @@ int check_device(int* sms) {
   *sms = g_sm_count;
   return RAWINT4_OK;
 }
+
+namespace {
 
 // ------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

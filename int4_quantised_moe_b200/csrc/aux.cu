@@ -35,7 +35,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
         const float lo = __uint_as_float(in[j] << 16);
         const float hi = __uint_as_float(in[j] & 0xFFFF0000u);
         __half2 h = __floats2half2_rn(lo, hi);
-        overflow |= (__hisinf(__low2half(h)) | __hisinf(__high2half(h))) != 0 && isfinite(lo) && isfinite(hi);
+        // each half on its own: a finite value that became inf (an inf or NaN
+        // input is not an overflow of the conversion)
+        overflow |= (__hisinf(__low2half(h)) != 0 && isfinite(lo)) || (__hisinf(__high2half(h)) != 0 && isfinite(hi));
         out[j] = *reinterpret_cast<uint32_t*>(&h);
       }
       d[c] = make_uint4(out[0], out[1], out[2], out[3]);

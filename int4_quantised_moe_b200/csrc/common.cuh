@@ -31,6 +31,10 @@ inline void device_flag_set(std::atomic<unsigned long long>& mask, int dev) {
   if (dev < 64) mask.fetch_or(1ull << dev);
 }
 
+// Host: the current device is an sm_100 part (RAWINT4_UNSUPPORTED otherwise,
+// RAWINT4_CUDA_ERROR when a query fails); *sms receives its SM count.
+int check_device(int* sms);
+
 // ------------------------------------------------------------------ status
 // Workspace header shared by all kernels of one layer call. Lives at the
 // start of the caller's workspace.

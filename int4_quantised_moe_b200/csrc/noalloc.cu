@@ -35,7 +35,10 @@ int scratch_address(void** out) {
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) return RAWINT4_CUDA_ERROR;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();  // leave no sticky error for the next library call to report
+      return RAWINT4_CUDA_ERROR;
+    }
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -62,8 +65,11 @@ RAWINT4_API int rawint4_moe_permute_static(const int64_t* ids, int32_t qlen, int
   const size_t need = hdr_bytes + tile_bytes + route_scratch_bytes(slots, experts);
   if (need > kStaticScratchBytes) return RAWINT4_STATIC_SCRATCH_TOO_SMALL;
 
+  int sms = 0;
+  int rc = check_device(&sms);  // a device without sm_100 code is UNSUPPORTED, not a CUDA error
+  if (rc != RAWINT4_OK) return rc;
   void* base = nullptr;
-  int rc = scratch_address(&base);
+  rc = scratch_address(&base);
   if (rc != RAWINT4_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream_);
   uint8_t* b = static_cast<uint8_t*>(base);

@@ -95,9 +95,9 @@ def pack_rawint4_codes(codes: np.ndarray) -> np.ndarray:
     """Codes in [0, 15] -> bytes, keeping the low-nibble-first order."""
     codes = np.asarray(codes)
     if codes.ndim < 1 or codes.shape[-1] % 2:
-        raise ValueError("RAWINT4 code count must be even")
+        raise ValueError("an odd number of codes cannot be packed two per byte")
     if codes.size and (codes.min() < 0 or codes.max() > 15):
-        raise ValueError("RAWINT4 codes must be in [0, 15]")
+        raise ValueError("a code outside 0..15 does not fit in one nibble")
     c = codes.astype(np.uint8)
     return np.ascontiguousarray(c[..., 0::2] | (c[..., 1::2] << 4))
 
