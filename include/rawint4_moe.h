@@ -216,7 +216,7 @@ RAWINT4_API int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t to
  *   ids, qlen, top_k, experts, offsets, perm, inv: as rawint4_moe_permute
  *   (device pointers, caller-owned outputs).
  * The scratch (header, tile list, per-block histograms: about
- * 512 + 16*(E + ceil(Q*k/256)) + 4*E*ceil(Q*k/1024) bytes) lives in a fixed
+ * 512 + 16*(E + ceil(Q*k/192)) + 4*E*ceil(Q*k/1024) bytes) lives in a fixed
  * device array of rawint4_moe_permute_static_max_bytes() bytes (1 MiB)
  * inside the library; every GPU that loads the library holds it until the
  * process exits. Larger problems are rejected with
@@ -240,6 +240,18 @@ RAWINT4_API size_t rawint4_moe_permute_static_max_bytes(void);
  * concurrent use from several threads. */
 RAWINT4_API int rawint4_moe_profile_begin(int max_launches);
 RAWINT4_API int rawint4_moe_profile_end(int max_out, int* n_out, const char** names, float* ms);
+
+/* Test export (no counterpart in the method): the bound, in nanoseconds, on
+ * every pipeline wait of the dequant GEMM kernels launched after this call
+ * (default 4e9 ns; ns = 0 restores it). When a wait runs past the bound, the
+ * kernel raises RAWINT4_DEV_TIMEOUT in the device status, every warp of the
+ * kernel leaves at its next wait once the copies and tensor-core operations
+ * it issued have landed, the tensor memory is released, and that call's
+ * outputs are invalid; the next call with a normal bound is unaffected. A
+ * bound far below a normal wait (1 ns, say) sends a call down that path on
+ * purpose, which is how the path is tested. Process-wide; do not change it
+ * while another host thread launches layer calls. */
+RAWINT4_API int rawint4_moe_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

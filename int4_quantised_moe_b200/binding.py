@@ -46,6 +46,7 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_profile_end",
     "rawint4_moe_permute_static",
     "rawint4_moe_permute_static_max_bytes",
+    "rawint4_moe_set_wait_limit_ns",
 )
 
 
@@ -97,6 +98,7 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_permute.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
     lib.rawint4_moe_permute_static.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     lib.rawint4_moe_permute_static_max_bytes.argtypes = []
+    lib.rawint4_moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
@@ -321,6 +323,12 @@ class Layer:
 # ---------------------------------------------------------------------------
 # Timing hook (measurement only)
 # ---------------------------------------------------------------------------
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound on every pipeline wait of the GEMM kernels launched from now on
+    (0 restores the default of 4 s); see include/rawint4_moe.h."""
+    _check(_lib.rawint4_moe_set_wait_limit_ns(int(ns)), "rawint4_moe_set_wait_limit_ns")
+
 
 def profile_begin(max_launches: int = 4096) -> None:
     _lib.rawint4_moe_profile_begin.argtypes = [ctypes.c_int]

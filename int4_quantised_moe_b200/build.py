@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librawint4_moe.so")
-SOURCES = ["api.cu", "gemm.cu", "gemm_pair.cu", "skinny.cu", "route.cu", "aux.cu", "prof.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "gemm.cu", "gemm_pair.cu", "gemm_tm.cu", "skinny.cu", "route.cu", "aux.cu", "prof.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "gemm.cuh", "skinny.cuh", "route.cuh", "aux.cuh", "prof.cuh"]
 
 NVCC_FLAGS = [
@@ -43,14 +43,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
+    from concurrent.futures import ThreadPoolExecutor
+
+    def compile_one(src: str) -> str:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         cmd = [_nvcc(), *NVCC_FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-        objs.append(obj)
+        return obj
+
+    # independent translation units compile in parallel
+    with ThreadPoolExecutor(max_workers=max(1, min(len(SOURCES), os.cpu_count() or 1))) as pool:
+        objs = list(pool.map(compile_one, SOURCES))
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     subprocess.run(cmd, check=True)

@@ -153,16 +153,21 @@ EncodeTiledFn encode_fn() {
 // packed projection [E, rows, kbytes] uint8; box {box_x bytes, box_y rows, 1};
 // the 128- and 64-byte-wide boxes of the transposed modes are loaded with the
 // matching swizzle (conflict-free reads by the decoders)
-bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y) {
+bool map_packed(CUtensorMap* m, const uint8_t* base, int64_t E, int64_t rows, int64_t kbytes, int box_x, int box_y,
+                bool swizzle32 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kbytes, (cuuint64_t)rows, (cuuint64_t)E};
   cuuint64_t strides[2] = {(cuuint64_t)kbytes, (cuuint64_t)(kbytes * rows)};
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
   cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = box_x == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_x == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, box_x == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (box_x == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // fp16 row-major [rows, cols]; box {64, box_rows}, 128-byte swizzle (UMMA
@@ -234,6 +239,36 @@ int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }
+
+// CTA pairs for a launch of the tensor-memory GEMM (gemm_tm.cu).
+int tm_clusters(int mode, int sms, int max_tiles, int rowblk) {
+  static std::atomic<int> cached[64][4];  // per device and mode; 0 = not queried yet
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int fit = cached[dev][mode].load();
+  if (fit <= 0) {
+    const int n = gemm_tm_max_clusters(mode);
+    fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);
+    cached[dev][mode].store(fit);
+  }
+  const int64_t items = (int64_t)max_tiles * rowblk;
+  return (int)(items < fit ? (items > 0 ? items : 1) : fit);
+}
+
+// Which GEMM kernels run: the tensor-memory pair kernels (gemm_tm.cu) when
+// the environment selects them (RAWINT4_GEMM=tm), the shared-memory operand
+// kernels (gemm.cu, gemm_pair.cu) otherwise.
+bool use_tm_forward() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("RAWINT4_GEMM");
+    v = (e && strcmp(e, "tm") == 0) ? 1 : 0;
+  }
+  return v == 1;
+}
+
+// Bound on any pipeline wait of the GEMM kernels (test export can shorten it).
+std::atomic<unsigned long long> g_wait_ns{4000000000ull};
 
 #define R4_TRY(x)                                \
   do {                                           \
@@ -307,7 +342,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   const int max_tiles = max_tok_tiles(maxR, E);
   {
     R4_PROF("gather_x", st);
-    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0,
+    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, 0,
                               st));
   }
   if (has_lora) {
@@ -364,10 +399,13 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, 128) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, 128) ||
+  const bool tm = use_tm_forward();
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, tm ? 64 : 128, tm) ||
+      !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, tm ? 64 : 128, tm) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
-  gp.n_rowblk = I / 128;
+  gp.wait_ns = g_wait_ns.load();
+  gp.n_rowblk = (I + 127) / 128;
   gp.feat = I;
   gp.n_main = H / kBlockK;
   gp.s0 = base->gate_s;
@@ -385,7 +423,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_gate_up", st);
-    R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    if (tm)
+      R4_TRY(launch_gemm_tm(kModeGateUp, gp, mp, tm_clusters(kModeGateUp, sms, max_tiles, gp.n_rowblk), st));
+    else
+      R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
 
   // ha = c * h A_d^T and hw = w * ha
@@ -405,7 +446,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, 256) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, 256) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, tm ? 64 : 256, tm) ||
+      !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, tm ? 64 : 256, tm) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -424,11 +466,14 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_down", st);
-    R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    if (tm)
+      R4_TRY(launch_gemm_tm(kModeDown, gp, mp, tm_clusters(kModeDown, sms, max_tiles, gp.n_rowblk), st));
+    else
+      R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_out", st);
-    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, st));
+    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, out, H, qlen, 0, 0, st));
   }
   return RAWINT4_OK;
 }
@@ -462,10 +507,16 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("header_bwd", st);
     R4_TRY(launch_header_check_bwd(hdr, st));
   }
+  // grad_out enters the fp16 operands scaled by an exact power of two chosen
+  // from its largest magnitude; the combines and the gradient epilogue undo it
+  {
+    R4_PROF("absmax_dy", st);
+    R4_TRY(launch_absmax_rows(grad_out, hdr, H, maxQ, st));
+  }
   {
     R4_PROF("gather_dy", st);
     R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR,
-                              &hdr->status, 1, st));
+                              &hdr->status, 1, 1, st));
   }
   {
     R4_PROF("lora_convert", st);
@@ -513,8 +564,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.w_perm = at<float>(ws, L.w_perm);
   gp.inter = I;
   gp.limit = c.swiglu_limit;
+  gp.wait_ns = g_wait_ns.load();
 
   // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
+  const bool tm = use_tm_forward();
   if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
@@ -538,7 +591,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_down_t", st);
-    R4_TRY(launch_gemm_pair(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
+    if (tm)
+      R4_TRY(launch_gemm_tm(kModeDownT, gp, mp, tm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
+    else
+      R4_TRY(launch_gemm_pair(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
   }
 
   // gb = c * [dG B_g, dU B_u]: gate in columns [0, r), up in [rp, rp + r)
@@ -559,7 +615,8 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 128, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 128, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, tm ? 64 : 128, 64) ||
+      !map_packed(&mp.q1, base->up_q, E, I, H / 2, tm ? 64 : 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -581,11 +638,14 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_gate_up_t", st);
-    R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    if (tm)
+      R4_TRY(launch_gemm_tm(kModeGateUpT, gp, mp, tm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
+    else
+      R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_dx", st);
-    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, st));
+    R4_TRY(launch_combine_rows(at<float>(ws, L.y), at<int32_t>(ws, L.inv), k, hdr, grad_in, H, maxQ, 1, 1, st));
   }
   if (grad_route) {
     R4_PROF("combine_route", st);
@@ -629,6 +689,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("header_end", st);
     R4_TRY(launch_header_end_bwd(hdr, st));
   }
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? 4000000000ull : (unsigned long long)ns);
   return RAWINT4_OK;
 }
 

@@ -12,11 +12,20 @@ __device__ __forceinline__ bool bwd_enabled(const WsHeader* hdr) { return hdr->s
 // ------------------------------------------------------------------ gather
 // One warp per permuted row: the source token is looked up once, then the
 // row is converted 8 elements per lane and step with 16-byte loads/stores.
+// scale_dy (grad_out): every value is multiplied by 2^s first, s from the
+// largest magnitude found by absmax_rows_kernel (exact: a power of two).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
-                                                          int top_k, const WsHeader* hdr, uint4* __restrict__ dst,
-                                                          int vecs_per_row, uint32_t* status, int need_saved) {
+                                                          int top_k, WsHeader* hdr, uint4* __restrict__ dst,
+                                                          int vecs_per_row, uint32_t* status, int need_saved,
+                                                          int scale_dy) {
   if (need_saved && !bwd_enabled(hdr)) return;
   const int64_t rows = hdr->routed;
+  float sc = 1.0f;
+  if (scale_dy) {
+    const int e = dy_scale_exponent(hdr->dy_amax);
+    sc = ldexpf(1.0f, e);
+    if (blockIdx.x == 0 && threadIdx.x == 0) hdr->dy_exp = e;
+  }
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -32,8 +41,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
       uint32_t out[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float lo = __uint_as_float(in[j] << 16);
-        const float hi = __uint_as_float(in[j] & 0xFFFF0000u);
+        const float lo = sc * __uint_as_float(in[j] << 16);
+        const float hi = sc * __uint_as_float(in[j] & 0xFFFF0000u);
         __half2 h = __floats2half2_rn(lo, hi);
         // each half on its own: a finite value that became inf (an inf or NaN
         // input is not an overflow of the conversion)
@@ -46,11 +55,33 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
 }
 
+// Largest |v| over the first hdr->qlen rows of a bf16 [rows, 8 * vecs] matrix,
+// as bf16 magnitude bits, folded into hdr->dy_amax (reset by the backward's
+// header check). Magnitude bits of finite values order like the values.
+__global__ void __launch_bounds__(256) absmax_rows_kernel(const uint4* __restrict__ src, int vecs_per_row, WsHeader* hdr) {
+  if (!bwd_enabled(hdr)) return;
+  const int64_t total = (int64_t)hdr->qlen * vecs_per_row;
+  uint32_t m = 0u;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(src + i);
+    m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+  }
+  m = max(m & 0xFFFFu, m >> 16);
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(&hdr->dy_amax, m);
+}
+
 // ----------------------------------------------------------------- combine
+// unscale_dy: the rows carry grad_out's power-of-two scale; multiply by 2^-s.
 __global__ void combine_rows_kernel(const float4* __restrict__ src, const int32_t* __restrict__ inv, int top_k,
-                                    const WsHeader* hdr, uint2* __restrict__ out, int vecs_per_row, int need_saved) {
+                                    const WsHeader* hdr, uint2* __restrict__ out, int vecs_per_row, int need_saved,
+                                    int unscale_dy) {
   if (need_saved && !bwd_enabled(hdr)) return;
   const int64_t total = (int64_t)hdr->qlen * vecs_per_row;
+  const float sc = unscale_dy ? ldexpf(1.0f, -hdr->dy_exp) : 1.0f;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = idx / vecs_per_row;
     const int c = (int)(idx - t * vecs_per_row);
@@ -65,8 +96,8 @@ __global__ void combine_rows_kernel(const float4* __restrict__ src, const int32_
         acc.w += v.w;
       }
     }
-    const uint32_t lo = (uint32_t)bf16_bits_rn(acc.x) | ((uint32_t)bf16_bits_rn(acc.y) << 16);
-    const uint32_t hi = (uint32_t)bf16_bits_rn(acc.z) | ((uint32_t)bf16_bits_rn(acc.w) << 16);
+    const uint32_t lo = (uint32_t)bf16_bits_rn(sc * acc.x) | ((uint32_t)bf16_bits_rn(sc * acc.y) << 16);
+    const uint32_t hi = (uint32_t)bf16_bits_rn(sc * acc.z) | ((uint32_t)bf16_bits_rn(sc * acc.w) << 16);
     out[idx] = make_uint2(lo, hi);
   }
 }
@@ -75,12 +106,13 @@ __global__ void combine_route_kernel(const float* __restrict__ part, int nparts,
                                      int top_k, const WsHeader* hdr, float* __restrict__ grad_route) {
   if (!bwd_enabled(hdr)) return;
   const int64_t total = (int64_t)hdr->qlen * top_k;
+  const float sc = ldexpf(1.0f, -hdr->dy_exp);  // the partials carry grad_out's scale
   for (int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f < total; f += (int64_t)gridDim.x * blockDim.x) {
     const int32_t p = inv[f];
     float acc = 0.f;
     if (p >= 0)
       for (int b = 0; b < nparts; ++b) acc += part[(int64_t)p * nparts + b];
-    grad_route[f] = acc;
+    grad_route[f] = sc * acc;
   }
 }
 
@@ -90,6 +122,8 @@ __global__ void header_begin_fwd_kernel(WsHeader* hdr, int save) {
   hdr->saved = save ? 1u : 0u;
 }
 __global__ void header_check_bwd_kernel(WsHeader* hdr) {
+  hdr->dy_amax = 0u;
+  hdr->dy_exp = 0;
   if (hdr->magic != kWsMagic || hdr->saved != 1u) {
     hdr->saved = 0u;
     atomicOr(&hdr->status, (uint32_t)RAWINT4_DEV_NO_SAVED_FORWARD);
@@ -141,21 +175,29 @@ int grid_for(int64_t work, int threads) {
 
 }  // namespace
 
-cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, const WsHeader* hdr,
-                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved,
+cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, WsHeader* hdr,
+                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved, int scale_dy,
                                cudaStream_t stream) {
   const int vecs = H / 8;
   gather_rows_kernel<<<grid_for((int64_t)max_rows * 32, 256), 256, 0, stream>>>(
       reinterpret_cast<const uint4*>(src_bf16), perm, top_k, hdr, reinterpret_cast<uint4*>(dst_f16), vecs, status,
-      need_saved);
+      need_saved, scale_dy);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_absmax_rows(const uint16_t* src_bf16, WsHeader* hdr, int H, int max_tokens, cudaStream_t stream) {
+  const int vecs = H / 8;
+  absmax_rows_kernel<<<grid_for((int64_t)max_tokens * vecs, 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src_bf16), vecs, hdr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine_rows(const float* src, const int32_t* inv, int top_k, const WsHeader* hdr, uint16_t* out_bf16,
-                                int H, int max_tokens, int need_saved, cudaStream_t stream) {
+                                int H, int max_tokens, int need_saved, int unscale_dy, cudaStream_t stream) {
   const int vecs = H / 4;
   combine_rows_kernel<<<grid_for((int64_t)max_tokens * vecs, 256), 256, 0, stream>>>(
-      reinterpret_cast<const float4*>(src), inv, top_k, hdr, reinterpret_cast<uint2*>(out_bf16), vecs, need_saved);
+      reinterpret_cast<const float4*>(src), inv, top_k, hdr, reinterpret_cast<uint2*>(out_bf16), vecs, need_saved,
+      unscale_dy);
   return cudaGetLastError();
 }
 

@@ -5,15 +5,23 @@ namespace r4 {
 
 // dst[p, :] = fp16(src[perm[p] / top_k, :]) for p < hdr->routed (bf16 src [Q, H]).
 // need_saved: the kernel does nothing unless the header holds a pending saved forward (backward use).
-cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, const WsHeader* hdr,
-                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved,
+// scale_dy: grad_out; values are multiplied by 2^s (dy_scale_exponent of hdr->dy_amax) and s is
+// recorded in hdr->dy_exp.
+cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, WsHeader* hdr,
+                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved, int scale_dy,
                                cudaStream_t stream);
 
-// out[t, :] = bf16(sum_s src[inv[t*k+s], :]) in slot order, t < hdr->qlen (fp32 src [R, H]).
-cudaError_t launch_combine_rows(const float* src, const int32_t* inv, int top_k, const WsHeader* hdr,
-                                uint16_t* out_bf16, int H, int max_tokens, int need_saved, cudaStream_t stream);
+// hdr->dy_amax = max(hdr->dy_amax, largest |v| of the first hdr->qlen rows of bf16 src [*, H]);
+// runs only with a pending saved forward (backward use).
+cudaError_t launch_absmax_rows(const uint16_t* src_bf16, WsHeader* hdr, int H, int max_tokens, cudaStream_t stream);
 
-// grad_route[t, s] = sum_b part[inv[f], b] (0 for dropped slots), f = t*k+s < hdr->qlen*k.
+// out[t, :] = bf16(sum_s src[inv[t*k+s], :]) in slot order, t < hdr->qlen (fp32 src [R, H]);
+// unscale_dy: the sum is multiplied by 2^-hdr->dy_exp before rounding.
+cudaError_t launch_combine_rows(const float* src, const int32_t* inv, int top_k, const WsHeader* hdr,
+                                uint16_t* out_bf16, int H, int max_tokens, int need_saved, int unscale_dy,
+                                cudaStream_t stream);
+
+// grad_route[t, s] = 2^-hdr->dy_exp sum_b part[inv[f], b] (0 for dropped slots), f = t*k+s < hdr->qlen*k.
 cudaError_t launch_combine_route(const float* part, int nparts, const int32_t* inv, int top_k, const WsHeader* hdr,
                                  float* grad_route, int max_tokens, cudaStream_t stream);
 

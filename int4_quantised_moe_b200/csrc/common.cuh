@@ -45,8 +45,25 @@ struct WsHeader {
   int32_t routed;        // valid permuted rows (ids in [0, E))
   uint32_t status;       // OR of RAWINT4_DEV_* bits
   int32_t n_tok_tiles;   // entries of the token-tile list
-  int32_t pad[10];
+  uint32_t dy_amax;      // backward: largest |grad_out| element, as its bf16 magnitude bits
+  int32_t dy_exp;        // backward: grad_out enters the fp16 operands scaled by 2^dy_exp
+  int32_t pad[8];
 };
+static_assert(sizeof(WsHeader) == 64, "workspace header layout");
+
+// Exponent s of the power-of-two scale applied to grad_out before it is
+// converted to fp16 operands: the largest magnitude times 2^s lies in [1, 2),
+// so every element keeps fp16's full relative precision unless it is more
+// than 2^14 times smaller than the largest one, and nothing overflows. The
+// backward is linear in grad_out (the clamp masks depend only on the saved
+// forward), so every output is exact after multiplying by 2^-s in fp32. An
+// all-zero or non-finite grad_out takes s = 0.
+__device__ __forceinline__ int dy_scale_exponent(uint32_t amax_bits16) {
+  if (amax_bits16 == 0u || amax_bits16 >= 0x7F80u) return 0;
+  int e = 0;
+  frexpf(__uint_as_float(amax_bits16 << 16), &e);  // |max| = f 2^e, f in [0.5, 1)
+  return min(120, max(-120, 1 - e));
+}
 constexpr uint32_t kWsMagic = 0x52344d45u;  // "R4ME"
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s bound on any spin
@@ -74,6 +91,18 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ANDs a predicate over the participating threads:
+// every participant gets the same result.
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.b32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -244,6 +273,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Registers into 32 lanes x 16 consecutive 32-bit columns of TMEM (thread i
+// of the warp writes lane base + i); tmem_wait_st waits for this thread's
+// stores to complete.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // 32 lanes x 16 consecutive 32-bit columns of TMEM into registers.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -373,6 +415,18 @@ __device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, 
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Pair-wide D[tmem] (+)= A[tmem] * B^T: as umma_f16_pair, but the A operand
+// (128 rows x 16 fp16 per CTA, K-major, two elements per 32-bit column) is
+// read from each CTA's tensor memory at the same address instead of shared
+// memory.
+__device__ __forceinline__ void umma_f16_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive once on `bar` (same offset) in every CTA of `cta_mask` when all MMAs

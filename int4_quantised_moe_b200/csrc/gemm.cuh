@@ -21,6 +21,7 @@ enum GemmMode : int {
 };
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
+constexpr int kTmAccCols = 192;    // gemm_tm.cu: columns of one TMEM accumulator = max token-tile rows
 constexpr int kLoraPad = 64;       // width of the LoRA side matrices (>= 2 * rank)
 
 struct GemmParams {
@@ -56,6 +57,7 @@ struct GemmParams {
   int ld_out;                // row length of out_a / out_b / out_h / in_*
   int inter;
   float limit;
+  unsigned long long wait_ns;  // bound on any pipeline wait (gemm_tm.cu)
 };
 
 struct GemmMaps {
@@ -71,5 +73,8 @@ cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
 // CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
 int gemm_pair_max_clusters(int mode);
+// CTA pairs with the decoded weights in tensor memory (gemm_tm.cu): gate/up and down.
+cudaError_t launch_gemm_tm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
+int gemm_tm_max_clusters(int mode);
 
 }  // namespace r4

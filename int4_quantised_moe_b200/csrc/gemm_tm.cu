@@ -1,0 +1,871 @@
+// Dequant-fused grouped GEMMs of the routed RAWINT4 MoE-LoRA layer on
+// sm_100a tensor cores with the decoded weight operand in tensor memory.
+//
+// Clusters of two CTAs on an SM pair walk (token tile, feature block) work
+// items, as the CTA-pair kernel of gemm_pair.cu does: 256 weight rows per item
+// (128 per CTA), one pair-wide M = 256 UMMA per 16-wide reduction step, each
+// CTA loading its half of the token tile. The difference is where the decoded
+// weights go: the decoder warps store them with tcgen05.st into a ring of A
+// stages in each CTA's tensor memory, and the UMMA reads A from there
+// (tcgen05.mma [d], [a-tmem], b-desc). Shared memory then holds only the TMA
+// rings of packed weights, group scales and activation tiles, which can be
+// made several times deeper than with decoded tiles in shared memory, and the
+// tensor cores read only the activation tiles from it.
+//
+// Tensor memory of each CTA (512 columns x 128 lanes):
+//   [0, 2 kAccCols)                 two accumulators of up to kAccCols token columns
+//   [2 kAccCols, + 32 kAStages)     A stages: 128 weight rows x 64 reduction fp16
+// so a token tile has at most kAccCols rows (the tile list is cut to that).
+//
+// Warp roles, in each CTA:
+//   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP)
+//   warp 1      leader CTA: pair-wide UMMA issuer; both CTAs: TMEM allocation
+//   warp 2      TMA producer of this CTA's half of the token tile (ring of kStagesB)
+//   warp 3      loader of the group scales (cp.async, ring of kStagesS)
+//   warps 4-7   epilogue: this CTA's TMEM rows -> fused math -> global
+//   warps 8-15  decoders: int4 -> fp16 -> tensor memory (two warps per lane quarter)
+//
+// K-major modes (gate/up and down forward): decoder warp (q, g) owns TMEM
+// lanes 32q..32q+31 (weight rows) and the 32-wide reduction group g of each
+// 64-wide stage; a thread decodes the 16 packed bytes of its row and group
+// and stores the 32 fp16 values as 16 columns of its lane.
+//
+// MN-major modes (the transpose-free backward, rawint4_sft_reference.py
+// transpose_free_rawint4_dx: down^T and gate/up^T): the packed base is read
+// along its stored output dimension, so one stored row holds one reduction
+// index for many weight rows. Decoder warp (q, g) loads the 32 stored rows of
+// group g (lane i: row i, the 16 bytes of the warp's 32 weight rows), turns
+// that 32 x 32 nibble block around across the warp with five shuffle and
+// byte-permute steps (lane m then holds the 32 reduction values of weight row
+// m), decodes with the per-row group scales and stores to its TMEM lane as in
+// the K-major modes. No transposed or dense copy of a base weight is made.
+//
+// The LoRA side product of each projection runs as one extra 64-wide
+// reduction stage in the same accumulators: its A operand is the LoRA tensor
+// of the expert (loaded into registers at the start of the item and stored by
+// the decoders), its B operand the precomputed c-scaled rank-r side matrix.
+#include "gemm.cuh"
+
+namespace r4 {
+
+namespace tmk {
+
+constexpr int kRowsM = 128;                       // weight rows per CTA (256 per pair)
+constexpr int kAStages = 4;                       // A stages in tensor memory (32 columns each)
+constexpr uint32_t kACol0 = 2 * kTmAccCols;       // first A column
+static_assert(kACol0 + 32 * kAStages <= 512, "tensor memory columns");
+constexpr int kStagesB = 10;                      // TMA-loaded B half tiles
+constexpr int kStagesP = 16;                      // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kStagesS = 16;                      // group scales of one stage (512 B each)
+constexpr int kThreads = 512;                     // 16 warps
+constexpr int kEpiWarp0 = 4;                      // warps 4..7: epilogue
+constexpr int kDecWarp0 = 8;                      // warps 8..15: decoders
+constexpr int kDecWarps = 8;
+
+constexpr int kBBytes = (kTmAccCols / 2) * kBlockK * 2;  // this CTA's half of <= kTmAccCols tokens
+constexpr int kPBytes = kRowsM * kBlockK / 2;            // 4 KB
+constexpr int kSBytes = 512;                             // 256 bf16 group scales
+constexpr int kOffB = 0;
+constexpr int kOffP = kOffB + kStagesB * kBBytes;
+constexpr int kOffS = kOffP + kStagesP * kPBytes;
+constexpr int kOffBar = kOffS + kStagesS * kSBytes;
+constexpr int kNumBars = 2 * kStagesP + 2 * kAStages + 2 * kStagesB + 2 * kStagesS + 4 + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
+constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // down^T dRoute partials; gate/up exchange uses 2 * 32 * 33
+constexpr int kTabBytes = 8 * 64;                 // MN-major: one 16-pair scale table per decoder warp
+constexpr int kOffScaleTab = kOffEpi + kEpiFloats * 4;
+constexpr int kSmemBytes = kOffScaleTab + kTabBytes + 1024;  // + alignment slack
+static_assert(kBBytes % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte aligned stages");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+constexpr uint16_t kPairMask = 3;
+constexpr uint64_t kDrainNs = 20000000ull;       // bound on the drains of an aborted call (20 ms)
+
+template <int MODE>
+constexpr bool kAMnMajor = (MODE == kModeDownT || MODE == kModeGateUpT);
+
+template <int MODE>
+__device__ __forceinline__ int kext_steps(int rpad) {
+  const int kext = (MODE == kModeGateUp || MODE == kModeGateUpT) ? 2 * rpad : rpad;
+  return kext / 16;
+}
+
+// First output feature of CTA `cta`'s 128 rows of block rb (gate/up: 64
+// features, TMEM lanes 0-63 gate and 64-127 up).
+template <int MODE>
+__device__ __forceinline__ int cta_f0(int rb, int cta) {
+  return MODE == kModeGateUp ? rb * 128 + 64 * cta : rb * 256 + 128 * cta;
+}
+
+// UMMA N of a token tile: rounded up to 32 so each CTA's half is a whole
+// number of 16-row boxes.
+__device__ __forceinline__ int pair_n(int rows) { return max(32, (rows + 31) & ~31); }
+
+// ------------------------------------------------------------ bounded waits
+// Sets this CTA's abort flag and the peer's (distributed shared memory), so
+// that every role of the pair leaves at its next wait.
+__device__ __forceinline__ void abort_pair(volatile int* abort_flag) {
+  *abort_flag = 1;
+  const uint32_t peer = cluster_addr((const void*)abort_flag, cluster_ctarank() ^ 1u);
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ bool wait_lim(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                         uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      raise_status(status, RAWINT4_DEV_TIMEOUT);
+      abort_pair(abort_flag);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                          uint64_t limit_ns) {
+  const bool ok = wait_lim(bar, parity, abort_flag, status, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Waits (bounded) for the fills of the last `n` (at most `stages`) stages a
+// producer issued into `full`: a call that aborts must not leave with copies
+// still landing in its shared memory.
+__device__ __forceinline__ void drain_ring(uint64_t* full, Ring r, int issued, int stages) {
+  const int n = issued < stages ? issued : stages;
+  const uint64_t t0 = globaltimer();
+  for (int j = 0; j < n; ++j) {
+    // step back to the previous issue
+    if (r.stage == 0) {
+      r.stage = stages - 1;
+      r.phase ^= 1u;
+    } else {
+      --r.stage;
+    }
+    while (!mbar_try_wait(&full[r.stage], r.phase)) {
+      if (globaltimer() - t0 > kDrainNs) return;
+    }
+  }
+}
+// Copies whose completion is counted on the leader's barrier cannot be
+// observed by the peer: it waits a grace period that any issued copy ends in.
+__device__ __forceinline__ void grace_wait() {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+}
+
+// ----------------------------------------------------------- K-major decode
+// Scale slot of one stage: [128 rows][2] bf16 (the two groups of the stage's
+// 64 reduction elements of each weight row).
+template <int MODE>
+__device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, int fc, int s, int ln, uint8_t* S) {
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int row = ln + 32 * t;
+    const uint16_t* sp = p.s0;
+    int f;
+    if constexpr (MODE == kModeGateUp) {
+      sp = row < 64 ? p.s0 : p.s1;
+      f = fc + (row & 63);
+    } else {
+      f = fc + row;
+    }
+    const bool ok = f < p.feat;
+    const uint16_t* src = ok ? sp + (int64_t)e * p.s_expert + (int64_t)f * p.s_row + 2 * s : p.s0;
+    cp_async_4(S + row * 4, src, ok ? 4u : 0u);
+  }
+}
+
+// MN-major scale slot: [64 stored rows][4] bf16, the group scales of this
+// CTA's 128 weight rows (4 groups of 32) at each stored row of the stage.
+template <int MODE>
+__device__ __forceinline__ void load_stage_scales_mn(const GemmParams& p, int e, int fc, int s, int ln, uint8_t* S) {
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int kr = ln + 32 * t;
+    int row = s * kBlockK + kr;
+    const uint16_t* sp = p.s0;
+    if (MODE == kModeGateUpT && row >= p.stored_rows) {
+      row -= p.stored_rows;
+      sp = p.s1;
+    }
+    // groups past the features are zero (a zero scale decodes every code to
+    // 0); features come in multiples of 64, so the two 4-byte halves suffice
+    const uint16_t* src = sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + fc / 32;
+    const bool ok0 = fc < p.feat, ok1 = fc + 64 < p.feat;
+    cp_async_4(S + kr * 8, ok0 ? src : p.s0, ok0 ? 4u : 0u);
+    cp_async_4(S + kr * 8 + 4, ok1 ? src + 2 : p.s0, ok1 ? 4u : 0u);
+  }
+}
+
+// 32 x 32 transpose of 4-bit values across a warp. On entry lane i holds row
+// i (nibble c at bits 4 (c % 8) of w[c / 8]); on exit lane i holds column i
+// in the same layout. Step d (16, 8, 4, 2, 1) swaps, between lanes l and
+// l ^ d, the entries whose column bit d differs from the lane's bit d.
+__device__ __forceinline__ void transpose_nibbles(uint32_t (&w)[4], int lane) {
+  constexpr uint32_t kFull = 0xffffffffu;
+  {
+    const bool b = lane & 16;
+    const uint32_t y0 = __shfl_xor_sync(kFull, b ? w[0] : w[2], 16);
+    const uint32_t y1 = __shfl_xor_sync(kFull, b ? w[1] : w[3], 16);
+    if (b) {
+      w[0] = y0;
+      w[1] = y1;
+    } else {
+      w[2] = y0;
+      w[3] = y1;
+    }
+  }
+  {
+    const bool b = lane & 8;
+    const uint32_t y0 = __shfl_xor_sync(kFull, b ? w[0] : w[1], 8);
+    const uint32_t y1 = __shfl_xor_sync(kFull, b ? w[2] : w[3], 8);
+    if (b) {
+      w[0] = y0;
+      w[2] = y1;
+    } else {
+      w[1] = y0;
+      w[3] = y1;
+    }
+  }
+  {  // half words
+    const bool b = lane & 4;
+    const uint32_t ps = b ? 0x5410u : 0x7632u;
+    const uint32_t y0 = __shfl_xor_sync(kFull, __byte_perm(w[0], w[1], ps), 4);
+    const uint32_t y1 = __shfl_xor_sync(kFull, __byte_perm(w[2], w[3], ps), 4);
+    const uint32_t u0 = b ? 0x3254u : 0x5410u, u1 = b ? 0x3276u : 0x7610u;
+    w[0] = __byte_perm(w[0], y0, u0);
+    w[1] = __byte_perm(w[1], y0, u1);
+    w[2] = __byte_perm(w[2], y1, u0);
+    w[3] = __byte_perm(w[3], y1, u1);
+  }
+  {  // bytes
+    const bool b = lane & 2;
+    const uint32_t ps = b ? 0x6420u : 0x7531u;
+    const uint32_t y0 = __shfl_xor_sync(kFull, __byte_perm(w[0], w[1], ps), 2);
+    const uint32_t y1 = __shfl_xor_sync(kFull, __byte_perm(w[2], w[3], ps), 2);
+    const uint32_t u0 = b ? 0x3514u : 0x5240u, u1 = b ? 0x3716u : 0x7260u;
+    w[0] = __byte_perm(w[0], y0, u0);
+    w[1] = __byte_perm(w[1], y0, u1);
+    w[2] = __byte_perm(w[2], y1, u0);
+    w[3] = __byte_perm(w[3], y1, u1);
+  }
+  {  // nibbles
+    constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
+    const bool b = lane & 1;
+    const uint32_t x0 = b ? ((w[0] & kLo) | ((w[1] << 4) & kHi)) : (((w[0] >> 4) & kLo) | (w[1] & kHi));
+    const uint32_t x1 = b ? ((w[2] & kLo) | ((w[3] << 4) & kHi)) : (((w[2] >> 4) & kLo) | (w[3] & kHi));
+    const uint32_t y0 = __shfl_xor_sync(kFull, x0, 1);
+    const uint32_t y1 = __shfl_xor_sync(kFull, x1, 1);
+    if (b) {
+      w[0] = (y0 & kLo) | (w[0] & kHi);
+      w[1] = ((y0 >> 4) & kLo) | (w[1] & kHi);
+      w[2] = (y1 & kLo) | (w[2] & kHi);
+      w[3] = ((y1 >> 4) & kLo) | (w[3] & kHi);
+    } else {
+      w[0] = (w[0] & kLo) | ((y0 << 4) & kHi);
+      w[1] = (w[1] & kLo) | (y0 & kHi);
+      w[2] = (w[2] & kLo) | ((y1 << 4) & kHi);
+      w[3] = (w[3] & kLo) | (y1 & kHi);
+    }
+  }
+}
+
+// 32 codes (byte j of w: values 2j low nibble, 2j + 1 high nibble) with one
+// scale per pair of values (sc[j] = fp16 pair of the scales of values 2j and
+// 2j + 1) into 16 fp16x2 words, as decode_group32 does with one scale.
+__device__ __forceinline__ void decode_pairs32(const uint32_t (&w)[4], const uint32_t (&sc)[16], uint32_t (&out)[16]) {
+  const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
+  const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t rep = __byte_perm(w[i], 0u, 0x1111u * j);
+      const uint32_t v = lop3_and_or(rep, 0x00F0000Fu, 0x64006400u);
+      __half2 h = __hfma2(*reinterpret_cast<const __half2*>(&v), mul, add);
+      h = __hmul2(h, *reinterpret_cast<const __half2*>(&sc[i * 4 + j]));
+      out[i * 4 + j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Row m, reduction group g of the LoRA stage (columns [32 g, 32 g + 32)) as
+// 16 fp16 pairs: the LoRA B row of the weight row (rank contiguous), placed at
+// the rank block of its projection.
+template <int MODE>
+__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, int m, int g, uint32_t (&w)[16]) {
+  const int r = p.rank;
+  const uint16_t* src = nullptr;
+  int jlo = 0;
+  if constexpr (MODE == kModeGateUp) {
+    const bool up = m >= 64;
+    const int f = fc + (m & 63);
+    if (f < p.feat) src = (up ? p.lx1 : p.lx0) + (int64_t)e * p.lx_expert + (int64_t)f * p.lx_ld;
+    jlo = up ? p.rpad : 0;
+  } else {
+    if (fc + m < p.feat) src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)(fc + m) * p.lx_ld;
+  }
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    float v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int jj = 32 * g + 2 * t + u - jlo;
+      v[u] = (src != nullptr && jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
+    }
+    w[t] = pack_h2(v[0], v[1]);
+  }
+}
+
+// MN-major: weight row m (feature fc + m), reduction group g of the LoRA
+// stage: the LoRA A column of the feature (rank rows [32 g, 32 g + 32) of the
+// 64-wide stage: gate/up^T stacks gate ranks at [0, r) and up ranks at
+// [rpad, rpad + r)), as 16 fp16 pairs.
+template <int MODE>
+__device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int fc, int m, int g, uint32_t (&w)[16]) {
+  const int r = p.rank;
+  const int f = fc + m;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    float v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int kr = 32 * g + 2 * t + u;
+      const uint16_t* src = nullptr;
+      if (f < p.feat) {
+        if (kr < r)
+          src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)kr * p.lx_ld + f;
+        else if (MODE == kModeGateUpT && kr >= p.rpad && kr < p.rpad + r)
+          src = p.lx1 + (int64_t)e * p.lx_expert + (int64_t)(kr - p.rpad) * p.lx_ld + f;
+      }
+      v[u] = src ? bf16_bits_to_float(__ldg(src)) : 0.0f;
+    }
+    w[t] = pack_h2(v[0], v[1]);
+  }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_tm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  const CUtensorMap& tq0 = maps.q0;
+  const CUtensorMap& tq1 = maps.q1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem + kOffB;
+  uint8_t* sP = smem + kOffP;
+  uint8_t* sS = smem + kOffS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
+  uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read it
+  uint64_t* a_full = p_empty + kStagesP;     // leader: both CTAs' decoders stored A
+  uint64_t* a_empty = a_full + kAStages;     // both: the pair MMA finished reading A
+  uint64_t* b_full = a_empty + kAStages;     // leader: both CTAs' B halves landed
+  uint64_t* b_empty = b_full + kStagesB;     // both: the pair MMA finished reading B
+  uint64_t* s_full = b_empty + kStagesB;     // local: a stage's scales landed
+  uint64_t* s_empty = s_full + kStagesS;     // local: this CTA's decoders read them
+  uint64_t* acc_full = s_empty + kStagesS;   // both [2]: accumulator complete
+  uint64_t* acc_empty = acc_full + 2;        // leader [2]: both epilogues drained it
+  uint64_t* mma_drain = acc_empty + 2;       // leader: all issued MMAs finished (abort path)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  float* epi = reinterpret_cast<float*>(smem + kOffEpi);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = (int)cluster_ctarank();
+  const uint64_t lim = p.wait_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesP; ++i) {
+      mbar_init(&p_full[i], 1);
+      mbar_init(&p_empty[i], kDecWarps);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&a_full[i], 2 * kDecWarps);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kStagesB; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < kStagesS; ++i) {
+      mbar_init(&s_full[i], 32);
+      mbar_init(&s_empty[i], kDecWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 2 * 4);
+    }
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tq0);
+    tma_prefetch_desc(&tq1);
+    for (int i = 0; i < 4; ++i) {
+      tma_prefetch_desc(&maps.b[i]);
+      tma_prefetch_desc(&maps.bx[i]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // every barrier of both CTAs initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int n_rowblk = p.n_rowblk;
+  const int n_tiles = (p.need_saved && p.hdr->saved != 1u) ? 0 : p.hdr->n_tok_tiles * n_rowblk;
+  const int n_main = p.n_main;
+  const int tile0 = (int)cluster_id_x();
+  const int tile_step = (int)cluster_count_x();
+  uint32_t* status = p.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------ packed weight producer
+    Ring ring;
+    int issued = 0;
+    for (int tile = tile0; tile < n_tiles; tile += tile_step) {
+      const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
+      const int e = tt.x;
+      for (int s = 0; s < n_main; ++s) {
+        if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_p;
+        if (lane == 0) {
+          uint64_t* bar = &p_full[ring.stage];
+          uint8_t* dst = sP + ring.stage * kPBytes;
+          // 2 boxes of 64 rows x 32 bytes; rows past the tensor are zero-filled
+          // and still counted
+          mbar_expect_tx(bar, kPBytes);
+          if constexpr (MODE == kModeGateUp) {
+            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), fc, e);
+            tma_load_3d(dst + kPBytes / 2, &tq1, bar, s * (kBlockK / 2), fc, e);
+          } else if constexpr (MODE == kModeDown) {
+            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), fc, e);
+            tma_load_3d(dst + kPBytes / 2, &tq0, bar, s * (kBlockK / 2), fc + 64, e);
+          } else {
+            // one box of 64 stored rows x 64 bytes (this CTA's 128 weight rows)
+            const int k0 = s * kBlockK;
+            if (MODE == kModeDownT || k0 < p.stored_rows)
+              tma_load_3d(dst, &tq0, bar, fc / 2, k0, e);
+            else
+              tma_load_3d(dst, &tq1, bar, fc / 2, k0 - p.stored_rows, e);
+          }
+        }
+        __syncwarp();
+        ring.advance(kStagesP);
+        ++issued;
+      }
+    }
+    goto done;
+  drain_p:
+    if (lane == 0) drain_ring(p_full, ring, issued, kStagesP);
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------- scale loader
+    Ring ring;
+    for (int tile = tile0; tile < n_tiles; tile += tile_step) {
+      const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
+      for (int s = 0; s < n_main; ++s) {
+        if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
+        if constexpr (kAMnMajor<MODE>)
+          load_stage_scales_mn<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
+        else
+          load_stage_scales<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
+        cp_async_arrive_noinc(&s_full[ring.stage]);
+        ring.advance(kStagesS);
+      }
+    }
+  drain_s:
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 2) {
+    // ------------------------------------------------------ B tile producer
+    Ring ring;
+    int issued = 0;
+    for (int tile = tile0; tile < n_tiles; tile += tile_step) {
+      const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const int nb = pair_n(tt.z) / 2;  // this CTA's token rows (multiple of 16)
+      const int row0 = tt.y + cta * nb;
+      for (int s = 0; s <= n_main; ++s) {
+        if (!wait_warp(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_b;
+        if (lane == 0) {
+          uint8_t* dst = sB + ring.stage * kBBytes;
+          const uint32_t bar = cluster_addr(&b_full[ring.stage], 0);
+          if (cta == 0) mbar_expect_tx(&b_full[ring.stage], 2 * nb * 128);
+          int row = 0;
+          for (int lvl = 2; lvl >= 0; --lvl) {
+            const int h = 16 << lvl;
+            while (nb - row >= h) {
+              if (s < n_main)
+                tma_load_2d_pair(dst + row * 128, &maps.b[lvl], bar, s * kBlockK, row0 + row);
+              else
+                tma_load_2d_pair(dst + row * 128, &maps.bx[lvl], bar, 0, row0 + row);
+              row += h;
+            }
+          }
+        }
+        __syncwarp();
+        ring.advance(kStagesB);
+        ++issued;
+      }
+    }
+    goto done;
+  drain_b:
+    if (lane == 0) {
+      if (cta == 0) drain_ring(b_full, ring, issued, kStagesB);
+      grace_wait();
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------- pair UMMA issuer (leader)
+    if (cta == 0) {
+      Ring ra, rbr;
+      int it = 0;
+      const int ksteps_x = kext_steps<MODE>(p.rpad);
+      for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
+        const int4 tt = p.tok_tiles[tile / n_rowblk];
+        const int n_mma = pair_n(tt.z);
+        const uint32_t idesc = make_idesc_f16((uint32_t)n_mma, false, false, 256);
+        const int ab = it & 1;
+        if (!wait_warp(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status, lim)) goto drain_mma;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * kTmAccCols);
+        for (int s = 0; s <= n_main; ++s) {
+          if (!wait_warp(&a_full[ra.stage], ra.phase, abort_flag, status, lim)) goto drain_mma;
+          if (!wait_warp(&b_full[rbr.stage], rbr.phase, abort_flag, status, lim)) goto drain_mma;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_tm = tmem + kACol0 + (uint32_t)(32 * ra.stage);
+            const uint32_t b_base = smem_u32(sB + rbr.stage * kBBytes);
+            const int ksteps = (s < n_main) ? (kBlockK / 16) : ksteps_x;
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint64_t bdesc = make_sdesc_sw128(b_base + kk * 32, 16, 1024);
+              umma_f16_pair_ts(d_tmem, a_tm + (uint32_t)(8 * kk), bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit_pair(&a_empty[ra.stage], kPairMask);
+            umma_commit_pair(&b_empty[rbr.stage], kPairMask);
+          }
+          __syncwarp();
+          ra.advance(kAStages);
+          rbr.advance(kStagesB);
+        }
+        if (lane == 0) umma_commit_pair(&acc_full[ab], kPairMask);
+        __syncwarp();
+      }
+      goto done;
+    drain_mma:
+      // every MMA this thread issued has finished before the pair leaves
+      if (lane == 0) {
+        umma_commit_pair(mma_drain, 1);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(mma_drain, 0u)) {
+          if (globaltimer() - t0 > kDrainNs) break;
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp >= kEpiWarp0 && warp < kDecWarp0) {
+    // --------------------------------------------------------------- epilogue
+    const int q = warp & 3;       // TMEM lane quarter this warp may access
+    const int m = 32 * q + lane;  // accumulator row of this thread
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    int it = 0;
+    for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
+      const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const int rb = tile % n_rowblk;
+      const int fc = cta_f0<MODE>(rb, cta);
+      const int n_rows = tt.z;
+      const int p0 = tt.y;
+      const int ab = it & 1;
+      // the four epilogue warps leave together or not at all: a warp that
+      // went on alone would wait forever at the gate/up exchange barrier
+      const bool ok = wait_warp(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status, lim);
+      if (!named_bar_and(3, 128, ok)) goto done;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + lane_base + (uint32_t)(ab * kTmAccCols);
+      for (int c0 = 0; c0 < n_rows; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(d_tmem + (uint32_t)c0, v);
+        if constexpr (MODE == kModeGateUp) {
+          // lanes 0-63: gate features fc + m; lanes 64-127: up features fc + m - 64
+          float* xch = epi + (q & 1) * 32 * 33;
+          if (q >= 2) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) xch[lane * 33 + c] = __uint_as_float(v[c]);
+          }
+          named_bar_sync(1 + (q & 1), 64);
+          const int i = fc + m;
+          if (q < 2 && i < p.feat) {
+            const float L = p.limit;
+            bool overflow = false;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int n = c0 + c;
+              if (n < n_rows) {
+                const int64_t o = (int64_t)(p0 + n) * p.ld_out + i;
+                const float g = __uint_as_float(v[c]);
+                const float u = xch[lane * 33 + c];
+                const float gc = L > 0.f ? fminf(g, L) : g;
+                const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
+                const float h = gc * sigmoid_clamped(gc) * uc;
+                const __half hh = __float2half_rn(h);
+                overflow |= __hisinf(hh) != 0;
+                p.out_a[o] = g;
+                p.out_b[o] = u;
+                p.out_h[o] = *reinterpret_cast<const uint16_t*>(&hh);
+              }
+            }
+            if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
+          }
+          named_bar_sync(1 + (q & 1), 64);
+        } else if constexpr (MODE == kModeDown || MODE == kModeGateUpT) {
+          // down: Yw = w y; gate/up^T: dx rows as they are
+          const int f = fc + m;
+          float wl = 1.0f;
+          if constexpr (MODE == kModeDown) wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int n = c0 + c;
+            const float w = __shfl_sync(0xffffffffu, wl, c);
+            if (n < n_rows && f < p.feat) p.out_a[(int64_t)(p0 + n) * p.ld_out + f] = w * __uint_as_float(v[c]);
+          }
+        } else {  // kModeDownT
+          // dh = w acc; SwiGLU' with the clamp masks decided on the saved fp32
+          // G and U; dRoute partial = sum over this CTA's features of acc h
+          // (h from the saved G, U), reduced over the 128 rows through shared
+          // memory. The saved G/U of 4 tokens are loaded together ahead of use.
+          const float L = p.limit;
+          float* red = epi + q * 32 * 33;
+          float* red2 = epi + 4 * 32 * 33;
+          bool overflow = false;
+          const int i = fc + m;
+          const bool live = i < p.feat;
+          const float wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
+#pragma unroll
+          for (int cb = 0; cb < 32; cb += 4) {
+            float gq[4], uq[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int64_t row = p0 + min(c0 + cb + c, n_rows - 1);
+              gq[c] = live ? __ldg(p.in_g + row * p.ld_out + i) : 0.f;
+              uq[c] = live ? __ldg(p.in_u + row * p.ld_out + i) : 0.f;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int n = c0 + cb + c;
+              const float w = __shfl_sync(0xffffffffu, wl, cb + c);
+              float pr = 0.f;
+              if (live && n < n_rows) {
+                const int64_t row = p0 + n;
+                const float acc_v = __uint_as_float(v[cb + c]);
+                const float g = gq[c];
+                const float u = uq[c];
+                const float gc = L > 0.f ? fminf(g, L) : g;
+                const float uc = L > 0.f ? fminf(fmaxf(u, -L), L) : u;
+                const bool pass_g = !(L > 0.f) || g <= L;
+                const bool pass_u = !(L > 0.f) || (u >= -L && u <= L);
+                const float sg = sigmoid_clamped(gc);
+                const float silu = gc * sg;
+                const float dsilu = sg * (1.0f + gc * (1.0f - sg));
+                const float dh = w * acc_v;
+                const float dg = pass_g ? dh * uc * dsilu : 0.f;
+                const float du = pass_u ? dh * silu : 0.f;
+                const __half hg = __float2half_rn(dg);
+                const __half hu = __float2half_rn(du);
+                overflow |= (__hisinf(hg) | __hisinf(hu)) != 0;
+                p.out_h[row * (2 * p.inter) + i] = *reinterpret_cast<const uint16_t*>(&hg);
+                p.out_h[row * (2 * p.inter) + p.inter + i] = *reinterpret_cast<const uint16_t*>(&hu);
+                pr = acc_v * silu * uc;
+              }
+              red[lane * 33 + cb + c] = pr;
+            }
+          }
+          if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
+          __syncwarp();
+          float colsum = 0.f;
+#pragma unroll 8
+          for (int r2 = 0; r2 < 32; ++r2) colsum += red[r2 * 33 + lane];
+          red2[q * 32 + lane] = colsum;
+          named_bar_sync(3, 128);
+          if (q == 0) {
+            const int n = c0 + lane;
+            if (n < n_rows) {
+              const float sum = red2[lane] + red2[32 + lane] + red2[64 + lane] + red2[96 + lane];
+              p.droute_part[(int64_t)(p0 + n) * p.n_parts + 2 * rb + cta] = sum;
+            }
+          }
+          named_bar_sync(3, 128);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[ab], 0));
+    }
+  } else if (warp >= kDecWarp0) {
+    // --------------------------------------------------------------- decoders
+    const int q = warp & 3;
+    const int g = (warp - kDecWarp0) >> 2;  // reduction group of each stage
+    const int m = 32 * q + lane;            // weight row (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // the packed tile is loaded with 32-byte swizzling: the 16-byte half g of
+    // row m sits at half g ^ ((m >> 2) & 1), which spreads every 8 lanes over
+    // all bank groups
+    // MN-major: lane i loads stored row 32 g + i, the 16-byte chunk of the
+    // warp's 32 weight rows (64-byte swizzling: chunk q of row r at
+    // q ^ ((r >> 1) & 3), conflict-free over every 8 lanes)
+    const int kr = 32 * g + lane;
+    const uint32_t p_off = kAMnMajor<MODE> ? (uint32_t)(kr * 64 + 16 * (q ^ ((kr >> 1) & 3)))
+                                           : (uint32_t)(m * 32 + 16 * (g ^ ((m >> 2) & 1)));
+    const uint32_t s_off = kAMnMajor<MODE> ? (uint32_t)(kr * 8 + 2 * q) : (uint32_t)(m * 4 + g * 2);
+    uint32_t* tab = reinterpret_cast<uint32_t*>(smem + kOffScaleTab) + 16 * (warp - kDecWarp0);
+    Ring ra, rp, rs;
+    for (int tile = tile0; tile < n_tiles; tile += tile_step) {
+      const int4 tt = p.tok_tiles[tile / n_rowblk];
+      const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
+      const int e = tt.x;
+      uint32_t lora_w[16];
+      if constexpr (kAMnMajor<MODE>)
+        lora_values_mn<MODE>(p, e, fc, m, g, lora_w);
+      else
+        lora_values<MODE>(p, e, fc, m, g, lora_w);
+      for (int s = 0; s <= n_main; ++s) {
+        if (!wait_warp(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status, lim)) goto done;
+        const uint32_t a_tm = tmem + lane_base + kACol0 + (uint32_t)(32 * ra.stage + 16 * g);
+        if (s < n_main) {
+          if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
+          const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
+          if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
+          const uint4 q4 = *reinterpret_cast<const uint4*>(sP + rp.stage * kPBytes + p_off);
+          uint32_t w[16];
+          if constexpr (kAMnMajor<MODE>) {
+            // every stored row has its own scale: pair them up (lane 2t holds
+            // the scales of values 2t and 2t + 1) through a per-warp table
+            const __half hs = __float2half_rn(bf16_bits_to_float(sc));
+            const uint32_t hb = (uint32_t)(*reinterpret_cast<const uint16_t*>(&hs));
+            const uint32_t nb = __shfl_down_sync(0xffffffffu, hb, 1);
+            if ((lane & 1) == 0) tab[lane >> 1] = hb | (nb << 16);
+            __syncwarp();
+            uint32_t sp2[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 t4 = *reinterpret_cast<const uint4*>(tab + 4 * j);
+              sp2[4 * j] = t4.x;
+              sp2[4 * j + 1] = t4.y;
+              sp2[4 * j + 2] = t4.z;
+              sp2[4 * j + 3] = t4.w;
+            }
+            uint32_t nib[4] = {q4.x, q4.y, q4.z, q4.w};
+            transpose_nibbles(nib, lane);
+            decode_pairs32(nib, sp2, w);
+          } else {
+            decode_group32(q4, bf16_scale_to_h2(sc), w);
+          }
+          tmem_st16(a_tm, w);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            // the packed and scale stages are released after the values that
+            // consume their bytes were stored
+            mbar_arrive(&p_empty[rp.stage]);
+            mbar_arrive(&s_empty[rs.stage]);
+            mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
+          }
+          rs.advance(kStagesS);
+          rp.advance(kStagesP);
+        } else {
+          tmem_st16(a_tm, lora_w);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
+        }
+        ra.advance(kAStages);
+      }
+    }
+  }
+
+done:
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no MMA, commit or remote arrival of either CTA is still pending
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
+template <int MODE>
+bool set_smem_attr() {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  if (!device_flag_test(done, &dev)) {
+    if (cudaFuncSetAttribute(gemm_tm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return false;
+    device_flag_set(done, dev);
+  }
+  return true;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GemmParams& p, const GemmMaps& m, int clusters, cudaStream_t stream) {
+  if (!set_smem_attr<MODE>()) return cudaErrorInvalidValue;
+  gemm_tm_kernel<MODE><<<2 * clusters, kThreads, kSmemBytes, stream>>>(p, m);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+int max_clusters_mode() {
+  if (!set_smem_attr<MODE>()) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tm_kernel<MODE>, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace tmk
+
+cudaError_t launch_gemm_tm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
+  switch (mode) {
+    case kModeGateUp: return tmk::launch_mode<kModeGateUp>(p, maps, clusters, stream);
+    case kModeDown: return tmk::launch_mode<kModeDown>(p, maps, clusters, stream);
+    case kModeDownT: return tmk::launch_mode<kModeDownT>(p, maps, clusters, stream);
+    case kModeGateUpT: return tmk::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int gemm_tm_max_clusters(int mode) {
+  switch (mode) {
+    case kModeGateUp: return tmk::max_clusters_mode<kModeGateUp>();
+    case kModeDown: return tmk::max_clusters_mode<kModeDown>();
+    case kModeDownT: return tmk::max_clusters_mode<kModeDownT>();
+    case kModeGateUpT: return tmk::max_clusters_mode<kModeGateUpT>();
+    default: return 0;
+  }
+}
+
+}  // namespace r4

@@ -4,7 +4,7 @@
 namespace r4 {
 
 constexpr int kRouteChunk = 1024;  // flat slots per block of the counting sort
-constexpr int kTileRows = 256;     // max permuted rows (tokens) per GEMM tile = max UMMA N
+constexpr int kTileRows = 192;     // max permuted rows (tokens) per GEMM tile (a TMEM accumulator's columns)
 
 size_t route_scratch_bytes(int32_t routed_slots, int32_t experts);
 
@@ -18,7 +18,7 @@ cudaError_t launch_route(const int64_t* ids, const float* rw, int32_t qlen, int3
 __global__ void tail_fill_kernel(int32_t* perm, const int32_t* offsets, int32_t experts, int32_t total);
 
 inline int32_t max_tok_tiles(int32_t routed_slots, int32_t experts) {
-  // every expert's rows split into ceil(n/256) tiles: at most E + slots/256 tiles
+  // every expert's rows split into ceil(n/kTileRows) tiles: at most E + slots/kTileRows tiles
   return experts + (routed_slots + kTileRows - 1) / kTileRows;
 }
 

@@ -215,6 +215,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       } else {
         const GradItem g = grad_item(p, item);
         const SkJob& jb = p.job[g.job];
+        // every gradient is linear in grad_out, whose fp16 copy carries the scale 2^dy_exp
+        const float gsc = ldexpf(p.grad_scale, -p.hdr->dy_exp);
         const int row0 = p.offsets[g.e], row1 = p.offsets[g.e + 1];
         const int nk = (row1 - row0 + 63) / 64;
         for (int k = 0; k < nk; ++k) {
@@ -356,6 +358,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       } else {
         const GradItem g = grad_item(p, item);
         const SkJob& jb = p.job[g.job];
+        // every gradient is linear in grad_out, whose fp16 copy carries the scale 2^dy_exp
+        const float gsc = ldexpf(p.grad_scale, -p.hdr->dy_exp);
         const int rows = p.offsets[g.e + 1] - p.offsets[g.e];
         const int pf = 128 * g.fb + 32 * q + lane;  // feature of this lane
         // outputs of this item: the low rank block -> out_lo, except the
@@ -397,11 +401,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
         ++it;
         if (jb.transposed) {
-          grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, p.grad_scale, p.accumulate,
+          grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, gsc, p.accumulate,
                                 false, gstage, 32 * q + lane, threadIdx.x - 64);
         } else if (live) {
-          grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, p.grad_scale, p.accumulate, false);
-          if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v1, p.grad_scale, p.accumulate, false);
+          grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, gsc, p.accumulate, false);
+          if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v1, gsc, p.accumulate, false);
         }
       }
     }

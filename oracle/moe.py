@@ -43,7 +43,7 @@ from typing import Dict, Iterable, List, Optional
 
 import numpy as np
 
-from . import rawint4
+from . import mxfp4, rawint4
 
 LORA_NAMES = ("gate_lora_a", "gate_lora_b", "up_lora_a", "up_lora_b", "down_lora_a", "down_lora_b")
 
@@ -67,6 +67,9 @@ class Layer:
     lora: Dict[str, np.ndarray]
     alpha: float
     swiglu_limit: float = 0.0
+    # "rawint4" (scales: float64 or bf16 bit patterns) or "mxfp4" (E2M1
+    # codes, scales: UE8M0 bytes, uint8); only the dequantisation differs
+    weight_format: str = "rawint4"
 
     @property
     def experts(self) -> int:
@@ -96,6 +99,12 @@ class Layer:
 
     def dense(self, e: int):
         """Dense float64 W_g, W_u [I, H] and W_d [H, I] of expert e."""
+        if self.weight_format == "mxfp4":
+            return (mxfp4.dequantize_mxfp4(self.gate_q[e], self.gate_s[e]),
+                    mxfp4.dequantize_mxfp4(self.up_q[e], self.up_s[e]),
+                    mxfp4.dequantize_mxfp4(self.down_q[e], self.down_s[e]))
+        if self.weight_format != "rawint4":
+            raise ValueError(f"unknown weight format {self.weight_format!r}")
         return (rawint4.dequantize_rawint4(self.gate_q[e], self._scale(self.gate_s, e)),
                 rawint4.dequantize_rawint4(self.up_q[e], self._scale(self.up_s, e)),
                 rawint4.dequantize_rawint4(self.down_q[e], self._scale(self.down_s, e)))
@@ -294,6 +303,8 @@ def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
         grad_route[ec.slots] = np.sum(g * ec.y, axis=1)
         dy = ec.w[:, None] * g
         gd = dy @ lo["down_lora_b"]
+        if transpose_free and layer.weight_format != "rawint4":
+            raise ValueError("the transpose-free loop is written for RAWINT4 storage")
         if transpose_free:
             dh_base = rawint4.transpose_free_dx(dy, layer.down_q[e], Layer._scale(layer.down_s, e))
         else:

@@ -338,3 +338,75 @@ def test_smaller_qlen_than_workspace():
     close("grad_route", groute, groute_r, TOL_ROUTE)
     for n in LORA_NAMES:
         close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("cfg_id", [0, 1])
+@pytest.mark.parametrize("dy_exp", [-30, -20, 20])
+def test_grad_out_magnitudes(cfg_id, dy_exp):
+    """grad_out scaled by 2^dy_exp (exact in bf16). Per-element output gradients
+    of a loss averaged over many tokens sit far below fp16's normal range; the
+    backward scales grad_out by a power of two before its fp16 operands are
+    formed and undoes it in fp32, so every output keeps the same relative
+    accuracy at any magnitude (and large gradients do not overflow)."""
+    wl = make_workload(CONFIGS[cfg_id])
+    dy = (wl.grad_out.float() * 2.0 ** dy_exp).to(torch.bfloat16)
+    assert torch.equal(dy.float(), wl.grad_out.float() * 2.0 ** dy_exp)  # the scaling is exact
+    wl = Workload(wl.cfg, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora, wl.x,
+                  wl.expert_ids, wl.route_weights, dy)
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+def test_fp16_overflow_is_reported():
+    """An activation beyond the fp16 operand range (one x element of 1e5) sets
+    the fp16-overflow status bit instead of passing silently; reading the
+    status clears it, and the next in-range call reports nothing."""
+    from int4_quantised_moe_b200 import binding as B
+    wl = make_workload(CONFIGS[0])
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    x = g.x.clone()
+    x[1, 3] = 1e5
+    assert float(x[1, 3]) > 65504.0
+    layer.forward(g.expert_ids, g.route_weights, x, save_for_backward=False)
+    assert layer.status() & B.DEV_FP16_OVERFLOW
+    assert layer.status() == 0
+    layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False)
+    assert layer.status() == 0
+
+
+def test_wait_timeout_aborts_cleanly():
+    """A pipeline-wait bound far below a normal wait (1 ns) sends the GEMM
+    kernels down their abort path on purpose: the call reports
+    RAWINT4_DEV_TIMEOUT, and with the default bound restored the next call is
+    correct, so every warp left, every copy and MMA in flight landed, and the
+    tensor memory was released (the contract test's fail-fast intent: an
+    error surfaces, nothing hangs)."""
+    from int4_quantised_moe_b200 import binding as B
+    wl = make_workload(CONFIGS[0])
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    try:
+        B.set_wait_limit_ns(1)
+        layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False)
+        assert layer.status() & B.DEV_TIMEOUT
+    finally:
+        B.set_wait_limit_ns(0)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
