@@ -372,7 +372,7 @@ def main():
         layer.forward(wl.expert_ids, wl.route_weights, wl.x, out=out, save_for_backward=True)
         layer.backward(wl.grad_out, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
         if pg is not None:
-            dp.allreduce_lora_grads(grads)
+            dp.reduce_window_grads(grads)  # one-step window: reduce at its end
 
     # ---- device-timed region (inputs resident in HBM) with per-launch events
     ms_step, launches, clocks = device_timed(step, args.steps, args.warmup, layer, B, dev, stream, barrier,
@@ -407,7 +407,7 @@ def main():
             layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
             layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
             if pg is not None:
-                dp.allreduce_lora_grads(grads)
+                dp.reduce_window_grads(grads)  # one-step window: reduce at its end
             h_out.copy_(out, non_blocking=True)
             h_gin.copy_(gin, non_blocking=True)
             h_gr.copy_(groute, non_blocking=True)

@@ -2,11 +2,19 @@
 
 Every rank holds the whole frozen int4 base and the LoRA tensors and runs the
 forward/backward on its own tokens; the only exchange is the sum of the six
-LoRA-gradient buffers after each backward (the gradient of the layer over the
-union of the ranks' tokens is the sum of the per-rank gradients, since every
-token contributes independently). Process-group plumbing only: no arithmetic of
-the method lives here, and nothing here touches another GPU's memory from a
-kernel.
+LoRA-gradient buffers (the gradient of the layer over the union of the ranks'
+tokens is the sum of the per-rank gradients, since every token contributes
+independently). Process-group plumbing only: no arithmetic of the method lives
+here, and nothing here touches another GPU's memory from a kernel.
+
+Gradient window with data parallelism. The library keeps the contract test's
+authoritative window per rank: the first backward of a window overwrites the
+six buffers (accumulate = 0), later micro-steps add to them (accumulate = 1),
+all on the rank's own tokens and without any collective. At the end of the
+window, once, ``reduce_window_grads`` sums the ranks' buffers in fp32 and
+rounds the sum once into bf16 (on every rank, or on one owner rank); the next
+window then starts again with accumulate = 0. Reducing after every micro-step
+instead would re-add the already reduced part of the window on each rank.
 """
 
 from __future__ import annotations
@@ -36,12 +44,30 @@ def shard_tokens(qlen: int, rank: int, world: int) -> slice:
     return slice(start, start + base + (1 if rank < extra else 0))
 
 
-def allreduce_lora_grads(grads: Dict[str, torch.Tensor], group=None, names: Iterable[str] = GRAD_ORDER) -> None:
-    """Sum each LoRA-gradient buffer over the ranks, in place, in a fixed order."""
+def reduce_window_grads(local: Dict[str, torch.Tensor], out: Optional[Dict[str, torch.Tensor]] = None, group=None,
+                        dst: Optional[int] = None, names: Iterable[str] = GRAD_ORDER) -> Dict[str, torch.Tensor]:
+    """End of a gradient window: sum the ranks' local window buffers.
+
+    Each bf16 buffer is widened to fp32, summed over the ranks (all-reduce, or
+    reduce to rank ``dst``, in a fixed order), and rounded once into ``out``
+    (default: the local buffers themselves). With ``dst`` set, only that rank's
+    output holds the sum (the owner of the authoritative gradients); the
+    others are left untouched. Returns the output buffers.
+    """
     import torch.distributed as dist
 
+    target = local if out is None else out
+    me = dist.get_rank(group) if dst is not None else None
     for n in names:
-        dist.all_reduce(grads[n], op=dist.ReduceOp.SUM, group=group)
+        t = local[n].to(torch.float32)
+        if dst is None:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+            target[n].copy_(t)
+        else:
+            dist.reduce(t, dst=dst, op=dist.ReduceOp.SUM, group=group)
+            if me == dst:
+                target[n].copy_(t)
+    return target
 
 
 def max_over_ranks(value: float, device: Optional[torch.device] = None, group=None) -> float:
