@@ -241,6 +241,20 @@ RAWINT4_API size_t rawint4_moe_permute_static_max_bytes(void);
 RAWINT4_API int rawint4_moe_profile_begin(int max_launches);
 RAWINT4_API int rawint4_moe_profile_end(int max_out, int* n_out, const char** names, float* ms);
 
+/* Test export (no counterpart in the method): the saved forward context of
+ * `workspace` (left by the most recent saving rawint4_moe_lora_fwd and not yet
+ * consumed by a backward), copied into caller-owned device buffers:
+ *   perm    int32 [max_tokens * top_k]  permuted row -> flat slot f = t*k + s
+ *           (-1 past the routed rows)
+ *   g, u    fp32 [max_tokens * top_k, I]  the gate and up pre-activations G, U
+ *           of each permuted row, the fp32 values the backward decides the
+ *           clamp masks on (rows past the routed ones are unspecified)
+ *   routed  host int32: number of routed (permuted) rows
+ * Synchronises `stream`; changes nothing in the workspace. Returns
+ * RAWINT4_NO_SAVED_FORWARD when no saved context is pending. */
+RAWINT4_API int rawint4_moe_lora_saved_preacts(const rawint4_moe_cfg* cfg, const void* workspace, size_t ws_bytes,
+                                               int32_t* perm, float* g, float* u, int32_t* routed, void* stream);
+
 /* Test export (no counterpart in the method): the bound, in nanoseconds, on
  * every pipeline wait of the dequant GEMM kernels launched after this call
  * (default 4e9 ns; ns = 0 restores it). When a wait runs past the bound, the

@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_permute_static",
     "rawint4_moe_permute_static_max_bytes",
     "rawint4_moe_set_wait_limit_ns",
+    "rawint4_moe_lora_saved_preacts",
 )
 
 
@@ -99,6 +100,7 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_permute_static.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     lib.rawint4_moe_permute_static_max_bytes.argtypes = []
     lib.rawint4_moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.rawint4_moe_lora_saved_preacts.argtypes = [P(Cfg), vp, sz, vp, vp, vp, P(i32), vp]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
@@ -318,6 +320,22 @@ class Layer:
 
     def status(self, stream=None) -> int:
         return rawint4_moe_lora_status(self.workspace, stream)
+
+    def saved_preacts(self, stream=None):
+        """(perm int32 [R], G fp32 [R, I], U fp32 [R, I]) of the pending saved
+        forward, R = routed rows (test export; see include/rawint4_moe.h)."""
+        c = self.cfg
+        rows = int(c.max_tokens) * int(c.top_k)
+        dev = self.workspace.device
+        perm = torch.empty(rows, dtype=torch.int32, device=dev)
+        g = torch.empty((rows, int(c.inter)), dtype=torch.float32, device=dev)
+        u = torch.empty_like(g)
+        routed = ctypes.c_int32(0)
+        rc = _lib.rawint4_moe_lora_saved_preacts(ctypes.byref(self.cfg), _ptr(self.workspace), self.workspace.numel(),
+                                                 _ptr(perm), _ptr(g), _ptr(u), ctypes.byref(routed), _stream(stream))
+        _check(rc, "rawint4_moe_lora_saved_preacts")
+        n = int(routed.value)
+        return perm[:n], g[:n], u[:n]
 
 
 # ---------------------------------------------------------------------------

@@ -692,6 +692,28 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   return RAWINT4_OK;
 }
 
+int rawint4_moe_lora_saved_preacts(const rawint4_moe_cfg* cfg, const void* workspace, size_t ws_bytes, int32_t* perm,
+                                   float* g, float* u, int32_t* routed, void* stream_) {
+  if (!cfg_ok(cfg) || !workspace || !perm || !g || !u || !routed) return RAWINT4_INVALID_ARGUMENT;
+  const Layout L = make_layout(*cfg);
+  if (ws_bytes < L.total) return RAWINT4_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_);
+  void* ws = const_cast<void*>(workspace);
+  WsHeader h{};
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  if (cudaMemcpy(&h, at<WsHeader>(ws, L.hdr), sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return RAWINT4_CUDA_ERROR;
+  if (h.magic != kWsMagic || h.saved != 1u) return RAWINT4_NO_SAVED_FORWARD;
+  const size_t rows = (size_t)cfg->max_tokens * cfg->top_k;
+  const size_t row_bytes = (size_t)cfg->inter * sizeof(float);
+  if (cudaMemcpyAsync(perm, at<int32_t>(ws, L.perm), rows * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(g, at<float>(ws, L.g), rows * row_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(u, at<float>(ws, L.u), rows * row_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RAWINT4_CUDA_ERROR;
+  *routed = h.routed;
+  return RAWINT4_OK;
+}
+
 int rawint4_moe_set_wait_limit_ns(uint64_t ns) {
   g_wait_ns.store(ns == 0 ? 4000000000ull : (unsigned long long)ns);
   return RAWINT4_OK;

@@ -110,13 +110,17 @@ __device__ __forceinline__ void abort_pair(volatile int* abort_flag) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
 }
 
+// A bound below kPollBelowNs is polled with the non-blocking test (a
+// try_wait may suspend until the phase completes, outlasting a short bound).
+constexpr uint64_t kPollBelowNs = 1000000ull;
+
 __device__ __forceinline__ bool wait_lim(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
                                          uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool poll = limit_ns < kPollBelowNs;
+  if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > limit_ns) {
       raise_status(status, RAWINT4_DEV_TIMEOUT);

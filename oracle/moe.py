@@ -169,9 +169,15 @@ def swiglu(G: np.ndarray, U: np.ndarray, limit: float) -> np.ndarray:
     return Gc * sigmoid(Gc) * Uc
 
 
-def swiglu_backward(G: np.ndarray, U: np.ndarray, dh: np.ndarray, limit: float):
-    """d/dG and d/dU of h = silu(G') U' given dh (subgradient 1 on the bounds)."""
+def swiglu_backward(G: np.ndarray, U: np.ndarray, dh: np.ndarray, limit: float, masks=None):
+    """d/dG and d/dU of h = silu(G') U' given dh (subgradient 1 on the bounds).
+
+    ``masks`` = (pass_g, pass_u) replaces the clamp's own gradient-pass
+    decisions (used to check a GPU result whose pre-activation landed on the
+    other side of a bound within its fp32 accumulation error)."""
     Gc, Uc, mask_g, mask_u = clamp_preacts(G, U, limit)
+    if masks is not None:
+        mask_g, mask_u = masks
     sg = sigmoid(Gc)
     silu = Gc * sg
     dsilu = sg * (1.0 + Gc * (1.0 - sg))
@@ -272,7 +278,7 @@ def forward_token_loop(layer: Layer, x, expert_ids, route_weights):
 # Backward (hand-derived chain rule of the forward above)
 # ---------------------------------------------------------------------------
 
-def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
+def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False, masks=None):
     """Gradients of sum(grad_out * out) w.r.t. x, route weights and the LoRA tensors.
 
     Per expert, with g = grad_out rows, dy = w g, c = alpha / rank:
@@ -285,6 +291,8 @@ def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
     LoRA gradients are raw sums over this call (unscaled by grad_scale).
     ``transpose_free`` computes the base part of dh and dx with the
     group-at-a-time loop of oracle.rawint4 instead of the dense matrix.
+    ``masks`` maps an expert to (pass_g, pass_u) boolean [M, I] arrays (rows in
+    the order of its ExpertCtx) that replace the clamp's own decisions.
     """
     g_all = np.asarray(grad_out, dtype=np.float64)
     Q, k = ctx.qlen, ctx.top_k
@@ -312,7 +320,7 @@ def backward(layer: Layer, ctx: Ctx, grad_out, transpose_free: bool = False):
         dh = dh_base + c * gd @ lo["down_lora_a"]
         grads["down_lora_b"][e] = c * dy.T @ (ec.h @ lo["down_lora_a"].T)
         grads["down_lora_a"][e] = c * gd.T @ ec.h
-        dG, dU = swiglu_backward(ec.G, ec.U, dh, L)
+        dG, dU = swiglu_backward(ec.G, ec.U, dh, L, None if masks is None else masks.get(e))
         gb_g = dG @ lo["gate_lora_b"]
         gb_u = dU @ lo["up_lora_b"]
         if transpose_free:

@@ -320,3 +320,31 @@ def test_duplicate_expert_slots_are_independent():
     np.testing.assert_allclose(gr_d[:, 0], gr_m[:, 0], rtol=1e-12, atol=1e-12)
     for n in LORA_NAMES:
         np.testing.assert_allclose(gd[n], gm[n], rtol=1e-11, atol=1e-11)
+
+
+def test_mask_override_reproduces_and_flips_one_decision():
+    """backward(masks=...) with the clamp's own decisions is bit-identical to
+    backward(); flipping one gate decision of one row changes that row's
+    token alone, by the closed-form term dh U' silu'(G') times the gate row of
+    W_g (plus its LoRA term)."""
+    wl = _tiny(limit=1.0, x_std=2.0)
+    layer = oracle_layer(wl)
+    out, ctx = omoe.forward(layer, f64(wl.x), wl.expert_ids.numpy(), f64(wl.route_weights))
+    gin, groute, grads = omoe.backward(layer, ctx, f64(wl.grad_out))
+    own = {}
+    for e, ec in ctx.experts.items():
+        _, _, mg, mu = omoe.clamp_preacts(ec.G, ec.U, layer.swiglu_limit)
+        own[e] = (mg, mu)
+    gin2, groute2, grads2 = omoe.backward(layer, ctx, f64(wl.grad_out), masks=own)
+    assert np.array_equal(gin, gin2) and np.array_equal(groute, groute2)
+    for n in LORA_NAMES:
+        assert np.array_equal(grads[n], grads2[n])
+    # flip the decision of one clamped gate element
+    e = next(e for e, (mg, _) in own.items() if not mg.all())
+    row, col = map(int, np.argwhere(~own[e][0])[0])
+    flipped = {k: (mg.copy(), mu.copy()) for k, (mg, mu) in own.items()}
+    flipped[e][0][row, col] = True
+    gin3, _, _ = omoe.backward(layer, ctx, f64(wl.grad_out), masks=flipped)
+    tok = int(ctx.experts[e].tokens[row])
+    diff = gin3 - gin
+    assert np.count_nonzero(np.abs(diff).sum(axis=1)) == 1 and np.abs(diff[tok]).sum() > 0
