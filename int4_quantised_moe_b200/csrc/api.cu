@@ -400,8 +400,9 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
   const bool tm = use_tm_forward();
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 32, tm ? 64 : 128, tm) ||
-      !map_packed(&mp.q1, base->up_q, E, I, H / 2, 32, tm ? 64 : 128, tm) ||
+  // tensor-memory kernel: boxes of 64 rows x 128 bytes (4 reduction stages)
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
+      !map_packed(&mp.q1, base->up_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.wait_ns = g_wait_ns.load();
@@ -446,8 +447,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 32, tm ? 64 : 256, tm) ||
-      !map_packed(&mp.q1, base->down_q, E, H, I / 2, 32, tm ? 64 : 256, tm) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, tm ? 128 : 32, tm ? 64 : 256) ||
+      !map_packed(&mp.q1, base->down_q, E, H, I / 2, tm ? 128 : 32, tm ? 64 : 256) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -667,10 +668,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     gq.accumulate = accumulate;
     gq.grad_scale = grad_scale;
     // L (features), S (rank side), split, transposed, output features, outputs
-    gq.job[0] = SkJob{H, 0, H / 128, kSplitNone, 0, H, grads->down_b, nullptr};
-    gq.job[1] = SkJob{I, 0, I / 128, kSplitNone, 1, I, grads->down_a, nullptr};
-    gq.job[2] = SkJob{2 * I, 0, 2 * I / 128, kSplitFeature, 0, I, grads->gate_b, grads->up_b};
-    gq.job[3] = SkJob{H, 0, H / 128, kSplitRank, 1, H, grads->gate_a, grads->up_a};
+    auto nfb = [](int P) { return (P + 127) / 128; };  // a partial last block is masked
+    gq.job[0] = SkJob{H, 0, nfb(H), kSplitNone, 0, H, grads->down_b, nullptr};
+    gq.job[1] = SkJob{I, 0, nfb(I), kSplitNone, 1, I, grads->down_a, nullptr};
+    gq.job[2] = SkJob{2 * I, 0, nfb(2 * I), kSplitFeature, 0, I, grads->gate_b, grads->up_b};
+    gq.job[3] = SkJob{H, 0, nfb(H), kSplitRank, 1, H, grads->gate_a, grads->up_a};
     SkMaps gm;
     if (!map_act(&gm.a[0], at<uint16_t>(ws, L.gp), L.rows, H, 64) ||
         !map_act(&gm.b[0], at<uint16_t>(ws, L.hw), L.rows, kLoraPad, 64) ||
@@ -681,7 +683,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
         !map_act(&gm.a[3], at<uint16_t>(ws, L.xp), L.rows, H, 64) ||
         !map_act(&gm.b[3], at<uint16_t>(ws, L.gb), L.rows, kLoraPad, 64))
       return RAWINT4_CUDA_ERROR;
-    const int items = E * (H / 128 + I / 128 + 2 * I / 128 + H / 128);
+    const int items = E * (nfb(H) + nfb(I) + nfb(2 * I) + nfb(H));
     R4_PROF("lora_grads", st);
     R4_TRY(launch_skinny(kSkGrads, gq, gm, grid_for_tiles(sms, items, 1), st));
   }

@@ -321,6 +321,10 @@ __device__ __forceinline__ void cp_async_8(void* smem_dst, const void* gsrc, uin
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
                : "memory");
 }
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
 // Arrive on `bar` once all cp.async of this thread issued so far have landed
 // (the barrier's expected count includes these arrivals).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {

@@ -55,28 +55,47 @@ constexpr int kAStages = 4;                       // A stages in tensor memory (
 constexpr uint32_t kACol0 = 2 * kTmAccCols;       // first A column
 static_assert(kACol0 + 32 * kAStages <= 512, "tensor memory columns");
 constexpr int kStagesB = 10;                      // TMA-loaded B half tiles
-constexpr int kStagesP = 16;                      // TMA-loaded packed int4 tiles (4 KB each)
-constexpr int kStagesS = 16;                      // group scales of one stage (512 B each)
+// Packed weights and their scales arrive in slots of several reduction
+// stages: a TMA box row is one memory request, and a K-major row of one stage
+// is only 32 bytes, so a slot holds kPSub stages of each row (a 128-byte box
+// row). K-major: 4 stages per slot (16 KB, 4 slots); MN-major: 2 stages (two
+// 64-row boxes of 64-byte rows, 8 KB, 8 slots).
+template <int MODE>
+constexpr int kPSub = (MODE == kModeDownT || MODE == kModeGateUpT) ? 2 : 4;
+constexpr int kPSlotBytes = 16384;                // largest packed slot
+constexpr int kPRing = 65536;                     // bytes of the packed ring
+template <int MODE>
+constexpr int kStagesP = kPRing / (kPSub<MODE> * 4096);  // packed slots
+constexpr int kMaxStagesP = 16;
+constexpr int kSSlotBytes = 2048;                 // largest scale slot
+constexpr int kStagesS = 8;                       // scale slots
 constexpr int kThreads = 512;                     // 16 warps
 constexpr int kEpiWarp0 = 4;                      // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                      // warps 8..15: decoders
 constexpr int kDecWarps = 8;
+#ifndef R4_DEC_BATCH
+#define R4_DEC_BATCH 2
+#endif
+constexpr int kDecBatch = R4_DEC_BATCH;           // main stages a decoder warp handles per hand-off
+static_assert(kAStages >= 2 * kDecBatch, "the MMA consumes one batch while the next is decoded");
 
 constexpr int kBBytes = (kTmAccCols / 2) * kBlockK * 2;  // this CTA's half of <= kTmAccCols tokens
-constexpr int kPBytes = kRowsM * kBlockK / 2;            // 4 KB
-constexpr int kSBytes = 512;                             // 256 bf16 group scales
+template <int MODE>
+constexpr int kPBytes = kPSub<MODE> * 4096;              // one packed slot (4 KB per stage)
+template <int MODE>
+constexpr int kSBytes = kPSub<MODE> * 512;               // one scale slot (256 bf16 per stage)
 constexpr int kOffB = 0;
 constexpr int kOffP = kOffB + kStagesB * kBBytes;
-constexpr int kOffS = kOffP + kStagesP * kPBytes;
-constexpr int kOffBar = kOffS + kStagesS * kSBytes;
-constexpr int kNumBars = 2 * kStagesP + 2 * kAStages + 2 * kStagesB + 2 * kStagesS + 4 + 1;
+constexpr int kOffS = kOffP + kPRing;
+constexpr int kOffBar = kOffS + kStagesS * kSSlotBytes;
+constexpr int kNumBars = 2 * kMaxStagesP + 2 * kAStages + 2 * kStagesB + 2 * kStagesS + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
 constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // down^T dRoute partials; gate/up exchange uses 2 * 32 * 33
-constexpr int kTabBytes = 8 * 64;                 // MN-major: one 16-pair scale table per decoder warp
+constexpr int kTabBytes = 8 * 64 * 2;             // MN-major: 16-pair scale tables, two per decoder warp
 constexpr int kOffScaleTab = kOffEpi + kEpiFloats * 4;
 constexpr int kSmemBytes = kOffScaleTab + kTabBytes + 1024;  // + alignment slack
-static_assert(kBBytes % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte aligned stages");
+static_assert(kBBytes % 1024 == 0 && kPRing % kPSlotBytes == 0, "1024-byte aligned stages");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint16_t kPairMask = 3;
 constexpr uint64_t kDrainNs = 20000000ull;       // bound on the drains of an aborted call (20 ms)
@@ -95,6 +114,22 @@ __device__ __forceinline__ int kext_steps(int rpad) {
 template <int MODE>
 __device__ __forceinline__ int cta_f0(int rb, int cta) {
   return MODE == kModeGateUp ? rb * 128 + 64 * cta : rb * 256 + 128 * cta;
+}
+
+// First packed slot of work item (tile, feature block rb): the items of
+// one token tile start their reduction at evenly spread stages (and wrap
+// around), so the CTA pairs that work on the same token tile at the same time
+// read different activation rows from L2 instead of the same ones in step.
+__device__ __forceinline__ int k_rotation(int rb, int n_rowblk, int n_slots) {
+#ifdef R4_NO_KROT
+  return 0;
+#else
+  return (int)(((int64_t)rb * n_slots) / n_rowblk);
+#endif
+}
+__device__ __forceinline__ int rotated(int s, int rot, int n_main) {
+  const int k = s + rot;
+  return k >= n_main ? k - n_main : k;
 }
 
 // UMMA N of a token tile: rounded up to 32 so each CTA's half is a whole
@@ -162,10 +197,13 @@ __device__ __forceinline__ void grace_wait() {
 }
 
 // ----------------------------------------------------------- K-major decode
-// Scale slot of one stage: [128 rows][2] bf16 (the two groups of the stage's
-// 64 reduction elements of each weight row).
+// K-major scale slot j: [128 rows][8] bf16, the groups 8j..8j+7 of each
+// weight row (its two groups of each of the slot's 4 stages); entries past the
+// features or the reduction are zero.
 template <int MODE>
-__device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, int fc, int s, int ln, uint8_t* S) {
+__device__ __forceinline__ void load_slot_scales(const GemmParams& p, int e, int fc, int j, int n_main, int ln,
+                                                 uint8_t* S) {
+  const bool full = 4 * j + 4 <= n_main && (p.s_row & 7) == 0;  // 16-byte aligned whole slot
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     const int row = ln + 32 * t;
@@ -178,19 +216,30 @@ __device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, in
       f = fc + row;
     }
     const bool ok = f < p.feat;
-    const uint16_t* src = ok ? sp + (int64_t)e * p.s_expert + (int64_t)f * p.s_row + 2 * s : p.s0;
-    cp_async_4(S + row * 4, src, ok ? 4u : 0u);
+    const uint16_t* src = sp + (int64_t)e * p.s_expert + (int64_t)f * p.s_row + 8 * j;
+    if (full) {
+      cp_async_16(S + row * 16, ok ? src : p.s0, ok ? 16u : 0u);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool v = ok && 4 * j + u < n_main;
+        cp_async_4(S + row * 16 + 4 * u, v ? src + 2 * u : p.s0, v ? 4u : 0u);
+      }
+    }
   }
 }
 
-// MN-major scale slot: [64 stored rows][4] bf16, the group scales of this
-// CTA's 128 weight rows (4 groups of 32) at each stored row of the stage.
+// MN-major scale slot j: [128 stored rows][4] bf16, the group scales of this
+// CTA's 128 weight rows (4 groups of 32) at each stored row of the slot's two
+// stages (stored rows past the reduction are not read).
 template <int MODE>
-__device__ __forceinline__ void load_stage_scales_mn(const GemmParams& p, int e, int fc, int s, int ln, uint8_t* S) {
+__device__ __forceinline__ void load_slot_scales_mn(const GemmParams& p, int e, int fc, int j, int n_main, int ln,
+                                                    uint8_t* S) {
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  for (int t = 0; t < 4; ++t) {
     const int kr = ln + 32 * t;
-    int row = s * kBlockK + kr;
+    if (2 * j + (kr >> 6) >= n_main) continue;
+    int row = 2 * j * kBlockK + kr;
     const uint16_t* sp = p.s0;
     if (MODE == kModeGateUpT && row >= p.stored_rows) {
       row -= p.stored_rows;
@@ -369,8 +418,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* sS = smem + kOffS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
-  uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read it
-  uint64_t* a_full = p_empty + kStagesP;     // leader: both CTAs' decoders stored A
+  uint64_t* p_empty = p_full + kMaxStagesP;  // local: this CTA's decoders read it
+  uint64_t* a_full = p_empty + kMaxStagesP;  // leader: both CTAs' decoders stored A
   uint64_t* a_empty = a_full + kAStages;     // both: the pair MMA finished reading A
   uint64_t* b_full = a_empty + kAStages;     // leader: both CTAs' B halves landed
   uint64_t* b_empty = b_full + kStagesB;     // both: the pair MMA finished reading B
@@ -389,7 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint64_t lim = p.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStagesP; ++i) {
+    for (int i = 0; i < kStagesP<MODE>; ++i) {
       mbar_init(&p_full[i], 1);
       mbar_init(&p_empty[i], kDecWarps);
     }
@@ -434,6 +483,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_rowblk = p.n_rowblk;
   const int n_tiles = (p.need_saved && p.hdr->saved != 1u) ? 0 : p.hdr->n_tok_tiles * n_rowblk;
   const int n_main = p.n_main;
+  constexpr int PS = kPSub<MODE>;                   // reduction stages per packed slot
+  const int n_slots = (n_main + PS - 1) / PS;
   const int tile0 = (int)cluster_id_x();
   const int tile_step = (int)cluster_count_x();
   uint32_t* status = p.status;
@@ -446,37 +497,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       const int e = tt.x;
-      for (int s = 0; s < n_main; ++s) {
+      const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
+      for (int j0 = 0; j0 < n_slots; ++j0) {
+        const int j = rotated(j0, rot, n_slots);
         if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_p;
         if (lane == 0) {
           uint64_t* bar = &p_full[ring.stage];
-          uint8_t* dst = sP + ring.stage * kPBytes;
-          // 2 boxes of 64 rows x 32 bytes; rows past the tensor are zero-filled
-          // and still counted
-          mbar_expect_tx(bar, kPBytes);
+          uint8_t* dst = sP + ring.stage * kPBytes<MODE>;
+          // every box is counted in full, also where it reaches past the
+          // tensor (zero-filled rows or reduction columns of a partial slot)
+          mbar_expect_tx(bar, kPBytes<MODE>);
           if constexpr (MODE == kModeGateUp) {
-            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), fc, e);
-            tma_load_3d(dst + kPBytes / 2, &tq1, bar, s * (kBlockK / 2), fc, e);
+            // 64 rows x 128 bytes (4 stages) of gate, then of up
+            tma_load_3d(dst, &tq0, bar, j * 128, fc, e);
+            tma_load_3d(dst + kPBytes<MODE> / 2, &tq1, bar, j * 128, fc, e);
           } else if constexpr (MODE == kModeDown) {
-            tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), fc, e);
-            tma_load_3d(dst + kPBytes / 2, &tq0, bar, s * (kBlockK / 2), fc + 64, e);
+            tma_load_3d(dst, &tq0, bar, j * 128, fc, e);
+            tma_load_3d(dst + kPBytes<MODE> / 2, &tq0, bar, j * 128, fc + 64, e);
           } else {
-            // one box of 64 stored rows x 64 bytes (this CTA's 128 weight rows)
-            const int k0 = s * kBlockK;
-            if (MODE == kModeDownT || k0 < p.stored_rows)
-              tma_load_3d(dst, &tq0, bar, fc / 2, k0, e);
-            else
-              tma_load_3d(dst, &tq1, bar, fc / 2, k0 - p.stored_rows, e);
+            // two boxes of 64 stored rows x 64 bytes (this CTA's 128 weight
+            // rows), one per stage: a stage never straddles gate and up
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int k0 = (2 * j + u) * kBlockK;
+              if (MODE == kModeDownT || k0 < p.stored_rows)
+                tma_load_3d(dst + 4096 * u, &tq0, bar, fc / 2, k0, e);
+              else
+                tma_load_3d(dst + 4096 * u, &tq1, bar, fc / 2, k0 - p.stored_rows, e);
+            }
           }
         }
         __syncwarp();
-        ring.advance(kStagesP);
+        ring.advance(kStagesP<MODE>);
         ++issued;
       }
     }
     goto done;
   drain_p:
-    if (lane == 0) drain_ring(p_full, ring, issued, kStagesP);
+    if (lane == 0) drain_ring(p_full, ring, issued, kStagesP<MODE>);
     __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------- scale loader
@@ -484,12 +542,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
-      for (int s = 0; s < n_main; ++s) {
+      const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
+      for (int j0 = 0; j0 < n_slots; ++j0) {
+        const int j = rotated(j0, rot, n_slots);
         if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         if constexpr (kAMnMajor<MODE>)
-          load_stage_scales_mn<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
+          load_slot_scales_mn<MODE>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
         else
-          load_stage_scales<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
+          load_slot_scales<MODE>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
         cp_async_arrive_noinc(&s_full[ring.stage]);
         ring.advance(kStagesS);
       }
@@ -504,7 +564,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int nb = pair_n(tt.z) / 2;  // this CTA's token rows (multiple of 16)
       const int row0 = tt.y + cta * nb;
-      for (int s = 0; s <= n_main; ++s) {
+      const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
+      // the item's stage order: slot-rotated main stages, then the LoRA stage
+      for (int j0 = 0; j0 <= n_slots; ++j0) {
+        const int j = j0 < n_slots ? rotated(j0, rot, n_slots) : 0;
+        const int nsub = j0 < n_slots ? min(PS, n_main - PS * j) : 1;
+        for (int u = 0; u < nsub; ++u) {
+        const int s = j0 < n_slots ? PS * j + u : n_main;
         if (!wait_warp(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_b;
         if (lane == 0) {
           uint8_t* dst = sB + ring.stage * kBBytes;
@@ -525,6 +591,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
         ring.advance(kStagesB);
         ++issued;
+        }
       }
     }
     goto done;
@@ -725,81 +792,123 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int g = (warp - kDecWarp0) >> 2;  // reduction group of each stage
     const int m = 32 * q + lane;            // weight row (TMEM lane)
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    // the packed tile is loaded with 32-byte swizzling: the 16-byte half g of
-    // row m sits at half g ^ ((m >> 2) & 1), which spreads every 8 lanes over
-    // all bank groups
-    // MN-major: lane i loads stored row 32 g + i, the 16-byte chunk of the
-    // warp's 32 weight rows (64-byte swizzling: chunk q of row r at
-    // q ^ ((r >> 1) & 3), conflict-free over every 8 lanes)
-    const int kr = 32 * g + lane;
-    const uint32_t p_off = kAMnMajor<MODE> ? (uint32_t)(kr * 64 + 16 * (q ^ ((kr >> 1) & 3)))
-                                           : (uint32_t)(m * 32 + 16 * (g ^ ((m >> 2) & 1)));
-    const uint32_t s_off = kAMnMajor<MODE> ? (uint32_t)(kr * 8 + 2 * q) : (uint32_t)(m * 4 + g * 2);
-    uint32_t* tab = reinterpret_cast<uint32_t*>(smem + kOffScaleTab) + 16 * (warp - kDecWarp0);
+    // Packed slot layout. K-major: row m holds the 4 stages' 128 bytes with
+    // 128-byte swizzling (16-byte chunk c of row m at chunk c ^ (m & 7)); the
+    // thread reads chunk 2u + g of sub-stage u, and every 8 lanes hit all bank
+    // groups. MN-major: stage u's 64 stored rows of 64 bytes with 64-byte
+    // swizzling (chunk q of stored row r at q ^ ((r >> 1) & 3)); lane i reads
+    // stored row 32 g + i, the chunk of the warp's 32 weight rows.
+    auto p_off = [&](int u) -> uint32_t {
+      if constexpr (kAMnMajor<MODE>) {
+        const int kr = 32 * g + lane;
+        return (uint32_t)(4096 * u + kr * 64 + 16 * (q ^ ((kr >> 1) & 3)));
+      } else {
+        return (uint32_t)(m * 128 + 16 * ((2 * u + g) ^ (m & 7)));
+      }
+    };
+    // scale of this thread's group: K-major [128 rows][8] (2 per stage),
+    // MN-major [128 stored rows][4 groups]
+    auto s_off = [&](int u) -> uint32_t {
+      if constexpr (kAMnMajor<MODE>)
+        return (uint32_t)((64 * u + 32 * g + lane) * 8 + 2 * q);
+      else
+        return (uint32_t)(m * 16 + (2 * u + g) * 2);
+    };
+    uint32_t* tab = reinterpret_cast<uint32_t*>(smem + kOffScaleTab) + 32 * (warp - kDecWarp0);
     Ring ra, rp, rs;
+    // Decodes sub-stage u of packed slot rp / scale slot rs into w; table `tb`
+    // holds the MN-major scale pairs.
+    auto decode_stage = [&](const Ring& rs_, const Ring& rp_, int u, uint32_t* tb, uint32_t (&w)[16]) {
+      const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs_.stage * kSSlotBytes + s_off(u));
+      const uint4 q4 = *reinterpret_cast<const uint4*>(sP + rp_.stage * kPBytes<MODE> + p_off(u));
+      if constexpr (kAMnMajor<MODE>) {
+        // every stored row has its own scale: pair them up (lane 2t holds
+        // the scales of values 2t and 2t + 1) through a per-warp table
+        const __half hs = __float2half_rn(bf16_bits_to_float(sc));
+        const uint32_t hb = (uint32_t)(*reinterpret_cast<const uint16_t*>(&hs));
+        const uint32_t nb = __shfl_down_sync(0xffffffffu, hb, 1);
+        if ((lane & 1) == 0) tb[lane >> 1] = hb | (nb << 16);
+        __syncwarp();
+        uint32_t sp2[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 t4 = *reinterpret_cast<const uint4*>(tb + 4 * j);
+          sp2[4 * j] = t4.x;
+          sp2[4 * j + 1] = t4.y;
+          sp2[4 * j + 2] = t4.z;
+          sp2[4 * j + 3] = t4.w;
+        }
+        uint32_t nib[4] = {q4.x, q4.y, q4.z, q4.w};
+        transpose_nibbles(nib, lane);
+        decode_pairs32(nib, sp2, w);
+      } else {
+        decode_group32(q4, bf16_scale_to_h2(sc), w);
+      }
+    };
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       const int e = tt.x;
+      const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
       uint32_t lora_w[16];
       if constexpr (kAMnMajor<MODE>)
         lora_values_mn<MODE>(p, e, fc, m, g, lora_w);
       else
         lora_values<MODE>(p, e, fc, m, g, lora_w);
-      for (int s = 0; s <= n_main; ++s) {
-        if (!wait_warp(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status, lim)) goto done;
-        const uint32_t a_tm = tmem + lane_base + kACol0 + (uint32_t)(32 * ra.stage + 16 * g);
-        if (s < n_main) {
-          if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
-          const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
-          if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
-          const uint4 q4 = *reinterpret_cast<const uint4*>(sP + rp.stage * kPBytes + p_off);
-          uint32_t w[16];
-          if constexpr (kAMnMajor<MODE>) {
-            // every stored row has its own scale: pair them up (lane 2t holds
-            // the scales of values 2t and 2t + 1) through a per-warp table
-            const __half hs = __float2half_rn(bf16_bits_to_float(sc));
-            const uint32_t hb = (uint32_t)(*reinterpret_cast<const uint16_t*>(&hs));
-            const uint32_t nb = __shfl_down_sync(0xffffffffu, hb, 1);
-            if ((lane & 1) == 0) tab[lane >> 1] = hb | (nb << 16);
-            __syncwarp();
-            uint32_t sp2[16];
+      for (int j0 = 0; j0 < n_slots; ++j0) {
+        const int j = rotated(j0, rot, n_slots);
+        const int nsub = min(PS, n_main - PS * j);
+        if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
+        if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
+        // The slot's stages kDecBatch at a time: the decodes of a batch are
+        // independent, so the chain of waits, tensor-memory store completion,
+        // fence and arrivals is paid once per batch; the A ring
+        // (kAStages >= 2 kDecBatch) lets the MMA consume one batch while the
+        // next one is decoded.
+        for (int u = 0; u < nsub; u += kDecBatch) {
+          const int nb = min(kDecBatch, nsub - u);
+          Ring r_a[kDecBatch];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 t4 = *reinterpret_cast<const uint4*>(tab + 4 * j);
-              sp2[4 * j] = t4.x;
-              sp2[4 * j + 1] = t4.y;
-              sp2[4 * j + 2] = t4.z;
-              sp2[4 * j + 3] = t4.w;
-            }
-            uint32_t nib[4] = {q4.x, q4.y, q4.z, q4.w};
-            transpose_nibbles(nib, lane);
-            decode_pairs32(nib, sp2, w);
-          } else {
-            decode_group32(q4, bf16_scale_to_h2(sc), w);
+          for (int b = 0; b < kDecBatch; ++b) {
+            r_a[b] = ra;
+            if (b < nb) ra.advance(kAStages);
           }
-          tmem_st16(a_tm, w);
+#pragma unroll
+          for (int b = 0; b < kDecBatch; ++b)
+            if (b < nb && !wait_warp(&a_empty[r_a[b].stage], r_a[b].phase ^ 1u, abort_flag, status, lim)) goto done;
+          uint32_t w[kDecBatch][16];
+#pragma unroll
+          for (int b = 0; b < kDecBatch; ++b)
+            if (b < nb) decode_stage(rs, rp, u + b, tab + 16 * b, w[b]);
+#pragma unroll
+          for (int b = 0; b < kDecBatch; ++b)
+            if (b < nb) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * r_a[b].stage + 16 * g), w[b]);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
-            // the packed and scale stages are released after the values that
-            // consume their bytes were stored
-            mbar_arrive(&p_empty[rp.stage]);
-            mbar_arrive(&s_empty[rs.stage]);
-            mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
+#pragma unroll
+            for (int b = 0; b < kDecBatch; ++b)
+              if (b < nb) mbar_arrive_cluster(cluster_addr(&a_full[r_a[b].stage], 0));
           }
-          rs.advance(kStagesS);
-          rp.advance(kStagesP);
-        } else {
-          tmem_st16(a_tm, lora_w);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
         }
-        ra.advance(kAStages);
+        // the packed and scale slots are released after the values that
+        // consume their bytes were stored
+        if (lane == 0) {
+          mbar_arrive(&p_empty[rp.stage]);
+          mbar_arrive(&s_empty[rs.stage]);
+        }
+        rp.advance(kStagesP<MODE>);
+        rs.advance(kStagesS);
       }
+      // the LoRA stage
+      if (!wait_warp(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status, lim)) goto done;
+      tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * ra.stage + 16 * g), lora_w);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
+      ra.advance(kAStages);
     }
   }
 

@@ -137,6 +137,7 @@ __device__ __forceinline__ void grad_block_transposed(const SkJob& jb, int rank,
     const int rem = idx - o * rank * 16;
     const int j = rem >> 4, v8 = rem & 15;
     const float* src = st + o * 4096 + j * 128 + 8 * v8;
+    if (p0 + 8 * v8 >= jb.pout) continue;  // past the last feature (a partial last block)
     uint16_t* buf = o ? jb.out_hi : out0;
     uint4* dst = reinterpret_cast<uint4*>(buf + ((int64_t)e * rank + j) * jb.pout + p0 + 8 * v8);
     const uint4 old = accumulate ? *dst : make_uint4(0u, 0u, 0u, 0u);
@@ -368,7 +369,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         uint16_t* out0 = jb.out_lo;
         uint32_t col0 = 0;
         int pbase = 0;
-        if (jb.split == kSplitFeature && 128 * g.fb >= jb.P / 2) {
+        // the split point P/2 (= I) is a multiple of 32, so each warp's 32
+        // features lie on one side of it (a block may straddle it)
+        if (jb.split == kSplitFeature && 128 * g.fb + 32 * q >= jb.P / 2) {
           out0 = jb.out_hi;
           col0 = (uint32_t)p.rpad;
           pbase = jb.P / 2;

@@ -27,6 +27,7 @@ constexpr int kSkStages = 6;
 enum SkSplit : int {
   kSplitNone = 0,     // j < rank -> out_lo
   kSplitFeature = 1,  // feature p < P/2: out_lo[p] with D[j]; p >= P/2: out_hi[p - P/2] with D[rpad + j]
+                      // (P/2 a multiple of 32: decided per warp of 32 features)
   kSplitRank = 2,     // D[j] -> out_lo[.., j], D[rpad + j] -> out_hi[.., j]
 };
 
