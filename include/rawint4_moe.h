@@ -241,6 +241,29 @@ RAWINT4_API size_t rawint4_moe_permute_static_max_bytes(void);
 RAWINT4_API int rawint4_moe_profile_begin(int max_launches);
 RAWINT4_API int rawint4_moe_profile_end(int max_out, int* n_out, const char** names, float* ms);
 
+/* Router hand-off (test_gemma4_moe.py, Gemma4TextRouter.forward: softmax
+ * over all experts, top-k, renormalise over the k, times a per-expert scale).
+ * rawint4_moe_router_topk turns expert scores into the layer's inputs:
+ *   scores   fp32 [Q, E] (device), the router's expert scores
+ *   escale   fp32 [E] per-expert scale (device, may be NULL: all 1)
+ *   ids      int64 [Q, k] (device, out): the k experts of largest probability,
+ *            largest first, equal probabilities to the lower index
+ *   weights  fp32 [Q, k] (device, out): renormalised probabilities * escale
+ * rawint4_moe_router_bwd hands the layer's grad_route (= dL/dweights, from
+ * rawint4_moe_lora_bwd) back to the router:
+ *   grad_scores  fp32 [Q, E] (device, out): dL/dscores; 0 outside each
+ *                token's k experts (the renormalisation cancels the softmax's
+ *                normalisation over all E)
+ *   grad_escale  fp32 [E] (device, out, may be NULL): dL/descale, summed over
+ *                the slots routed to each expert in token order
+ * Limits: 1 <= k <= min(E, 32), E <= 4096, Q >= 0; RAWINT4_INVALID_ARGUMENT
+ * otherwise. Both only enqueue work on `stream`. */
+RAWINT4_API int rawint4_moe_router_topk(const float* scores, int32_t qlen, int32_t experts, int32_t top_k,
+                                        const float* escale, int64_t* ids, float* weights, void* stream);
+RAWINT4_API int rawint4_moe_router_bwd(const float* scores, int32_t qlen, int32_t experts, int32_t top_k,
+                                       const int64_t* ids, const float* grad_route, const float* escale,
+                                       float* grad_scores, float* grad_escale, void* stream);
+
 /* Test export (no counterpart in the method): the saved forward context of
  * `workspace` (left by the most recent saving rawint4_moe_lora_fwd and not yet
  * consumed by a backward), copied into caller-owned device buffers:

@@ -48,6 +48,8 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_permute_static_max_bytes",
     "rawint4_moe_set_wait_limit_ns",
     "rawint4_moe_lora_saved_preacts",
+    "rawint4_moe_router_topk",
+    "rawint4_moe_router_bwd",
 )
 
 
@@ -101,6 +103,8 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_permute_static_max_bytes.argtypes = []
     lib.rawint4_moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.rawint4_moe_lora_saved_preacts.argtypes = [P(Cfg), vp, sz, vp, vp, vp, P(i32), vp]
+    lib.rawint4_moe_router_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+    lib.rawint4_moe_router_bwd.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
@@ -341,6 +345,37 @@ class Layer:
 # ---------------------------------------------------------------------------
 # Timing hook (measurement only)
 # ---------------------------------------------------------------------------
+
+def router_topk(scores: torch.Tensor, top_k: int, escale: Optional[torch.Tensor] = None, stream=None):
+    """Expert ids int64 [Q, k] and route weights fp32 [Q, k] from router scores fp32 [Q, E]
+    (softmax, top-k, renormalised, times the per-expert scale)."""
+    q, E = scores.shape
+    _expect(scores, "scores", torch.float32, (q, E))
+    if escale is not None:
+        _expect(escale, "escale", torch.float32, (E,), scores.device)
+    ids = torch.empty((q, int(top_k)), dtype=torch.int64, device=scores.device)
+    w = torch.empty((q, int(top_k)), dtype=torch.float32, device=scores.device)
+    _check(_lib.rawint4_moe_router_topk(_ptr(scores), q, E, int(top_k), _ptr(escale), _ptr(ids), _ptr(w),
+                                        _stream(stream)), "rawint4_moe_router_topk")
+    return ids, w
+
+
+def router_bwd(scores: torch.Tensor, ids: torch.Tensor, grad_route: torch.Tensor, escale: Optional[torch.Tensor] = None,
+               want_escale_grad: bool = False, stream=None):
+    """dL/dscores fp32 [Q, E] (and dL/descale fp32 [E]) from the layer's grad_route."""
+    q, E = scores.shape
+    k = ids.shape[1] if ids.dim() == 2 else -1
+    _expect(scores, "scores", torch.float32, (q, E))
+    _expect(ids, "ids", torch.int64, (q, k), scores.device)
+    _expect(grad_route, "grad_route", torch.float32, (q, k), scores.device)
+    if escale is not None:
+        _expect(escale, "escale", torch.float32, (E,), scores.device)
+    dz = torch.empty_like(scores)
+    dc = torch.empty(E, dtype=torch.float32, device=scores.device) if want_escale_grad else None
+    _check(_lib.rawint4_moe_router_bwd(_ptr(scores), q, E, k, _ptr(ids), _ptr(grad_route), _ptr(escale), _ptr(dz),
+                                       _ptr(dc), _stream(stream)), "rawint4_moe_router_bwd")
+    return (dz, dc) if want_escale_grad else dz
+
 
 def set_wait_limit_ns(ns: int) -> None:
     """Bound on every pipeline wait of the GEMM kernels launched from now on

@@ -11,6 +11,7 @@
 #include "gemm.cuh"
 #include "prof.cuh"
 #include "route.cuh"
+#include "router.cuh"
 #include "skinny.cuh"
 
 namespace r4 {
@@ -691,6 +692,36 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("header_end", st);
     R4_TRY(launch_header_end_bwd(hdr, st));
   }
+  return RAWINT4_OK;
+}
+
+static bool router_args_ok(const float* scores, int32_t qlen, int32_t experts, int32_t top_k) {
+  return qlen >= 0 && experts >= 1 && experts <= 4096 && top_k >= 1 && top_k <= 32 && top_k <= experts &&
+         (qlen == 0 || scores != nullptr);
+}
+
+int rawint4_moe_router_topk(const float* scores, int32_t qlen, int32_t experts, int32_t top_k, const float* escale,
+                            int64_t* ids, float* weights, void* stream_) {
+  if (!router_args_ok(scores, qlen, experts, top_k) || (qlen > 0 && (!ids || !weights))) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  R4_PROF("router_topk", static_cast<cudaStream_t>(stream_));
+  R4_TRY(launch_router_topk(scores, qlen, experts, top_k, escale, ids, weights, static_cast<cudaStream_t>(stream_)));
+  return RAWINT4_OK;
+}
+
+int rawint4_moe_router_bwd(const float* scores, int32_t qlen, int32_t experts, int32_t top_k, const int64_t* ids,
+                           const float* grad_route, const float* escale, float* grad_scores, float* grad_escale,
+                           void* stream_) {
+  if (!router_args_ok(scores, qlen, experts, top_k) || (qlen > 0 && (!ids || !grad_route || !grad_scores)))
+    return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  R4_PROF("router_bwd", static_cast<cudaStream_t>(stream_));
+  R4_TRY(launch_router_bwd(scores, qlen, experts, top_k, ids, grad_route, escale, grad_scores, grad_escale,
+                           static_cast<cudaStream_t>(stream_)));
   return RAWINT4_OK;
 }
 

@@ -50,7 +50,6 @@ namespace r4 {
 
 namespace tmk {
 
-constexpr int kRowsM = 128;                       // weight rows per CTA (256 per pair)
 constexpr int kAStages = 4;                       // A stages in tensor memory (32 columns each)
 constexpr uint32_t kACol0 = 2 * kTmAccCols;       // first A column
 static_assert(kACol0 + 32 * kAStages <= 512, "tensor memory columns");
