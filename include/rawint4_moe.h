@@ -79,7 +79,9 @@ enum {
  * LoRA rank r and alpha (scaling c = alpha / r), swiglu_limit L (0 disables
  * the clamp; must be finite and >= 0) and max_tokens (the largest qlen a
  * workspace is sized for; the reference's max_len).
- * Limits: H % 128 == 0, I % 128 == 0, 1 <= rank <= 32, 1 <= top_k <= experts. */
+ * Limits: H % 64 == 0, I % 64 == 0 (the kernels reduce in stages of 64 and
+ * mask a partial last block of output features), 1 <= rank <= 32,
+ * 1 <= top_k <= experts. */
 typedef struct rawint4_moe_cfg {
   int32_t experts;
   int32_t top_k;
@@ -194,6 +196,17 @@ RAWINT4_API const char* rawint4_moe_lora_strerror(int code);
  *   the fp16 rounding of the same product (exact for scales in range). */
 RAWINT4_API int rawint4_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, float* out_f32,
                    uint16_t* out_f16, void* stream);
+
+/* Bit-exact check export for the MXFP4 base format (the pages' sibling
+ * format, weight layout mxfp4-e2m1-ue8m0-g32): one E2M1 code per nibble, low
+ * nibble first, one UE8M0 scale byte e per 32 input features whose value is
+ * 2^(e - 127) (the bf16 bit-cast e << 7: e == 0 is 0, e == 255 is +inf).
+ *   q [N, K/2] uint8, s [N, K/32] uint8 (device); K % 32 == 0.
+ *   out_f32 [N, K] fp32 (device, may be NULL): E2M1 value * 2^(e - 127).
+ *   out_f16 [N, K] fp16 bits (device, may be NULL): the tensor-core operand
+ *   the MXFP4 GEMM producers decode, exact for e in [104, 140]. */
+RAWINT4_API int rawint4_mxfp4_decode(const uint8_t* q, const uint8_t* s, int64_t n, int64_t k, float* out_f32,
+                                     uint16_t* out_f16, void* stream);
 
 /* Bit-exact check export: the token->expert permutation of the forward.
  * ids int64 [Q, k] (device). Outputs (device, int32):

@@ -50,6 +50,7 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_lora_saved_preacts",
     "rawint4_moe_router_topk",
     "rawint4_moe_router_bwd",
+    "rawint4_mxfp4_decode",
 )
 
 
@@ -105,6 +106,7 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_lora_saved_preacts.argtypes = [P(Cfg), vp, sz, vp, vp, vp, P(i32), vp]
     lib.rawint4_moe_router_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     lib.rawint4_moe_router_bwd.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.rawint4_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
@@ -203,6 +205,14 @@ def rawint4_decode(q: torch.Tensor, s: torch.Tensor, out_f32=None, out_f16=None,
     rows = q.numel() // k2
     _check(_lib.rawint4_decode(_ptr(q), _ptr(s), rows, 2 * k2, _ptr(out_f32), _ptr(out_f16), _stream(stream)),
            "rawint4_decode")
+
+
+def rawint4_mxfp4_decode(q: torch.Tensor, s: torch.Tensor, out_f32=None, out_f16=None, stream=None) -> None:
+    """MXFP4 check decode: q uint8 [N, K/2], s uint8 [N, K/32] -> fp32 and/or fp16 [N, K]."""
+    k2 = q.shape[-1]
+    rows = q.numel() // k2
+    _check(_lib.rawint4_mxfp4_decode(_ptr(q), _ptr(s), rows, 2 * k2, _ptr(out_f32), _ptr(out_f16), _stream(stream)),
+           "rawint4_mxfp4_decode")
 
 
 def rawint4_moe_permute(expert_ids: torch.Tensor, experts: int, offsets, perm, inv, stream=None) -> None:

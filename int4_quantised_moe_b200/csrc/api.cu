@@ -81,8 +81,8 @@ bool cfg_ok(const rawint4_moe_cfg* c) {
   if (!c) return false;
   if (c->experts < 1 || c->experts > 4096) return false;
   if (c->top_k < 1 || c->top_k > c->experts) return false;
-  if (c->hidden < 128 || c->hidden % 128 != 0) return false;
-  if (c->inter < 128 || c->inter % 128 != 0) return false;
+  if (c->hidden < 64 || c->hidden % 64 != 0) return false;
+  if (c->inter < 64 || c->inter % 64 != 0) return false;
   if (c->rank < 1 || c->rank > 32) return false;
   if (!std::isfinite(c->alpha)) return false;
   if (!std::isfinite(c->swiglu_limit) || c->swiglu_limit < 0.f) return false;
@@ -771,6 +771,17 @@ int rawint4_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, fl
   int rc = check_device(&sms);
   if (rc != RAWINT4_OK) return rc;
   if (launch_decode(q, s, n, k, out_f32, out_f16, static_cast<cudaStream_t>(stream_)) != cudaSuccess)
+    return RAWINT4_CUDA_ERROR;
+  return RAWINT4_OK;
+}
+
+int rawint4_mxfp4_decode(const uint8_t* q, const uint8_t* s, int64_t n, int64_t k, float* out_f32, uint16_t* out_f16,
+                         void* stream_) {
+  if (!q || !s || n < 0 || k < 0 || k % 32 != 0 || (!out_f32 && !out_f16)) return RAWINT4_INVALID_ARGUMENT;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  if (launch_decode_mxfp4(q, s, n, k, out_f32, out_f16, static_cast<cudaStream_t>(stream_)) != cudaSuccess)
     return RAWINT4_CUDA_ERROR;
   return RAWINT4_OK;
 }

@@ -166,6 +166,42 @@ __global__ void decode_kernel(const uint8_t* __restrict__ q, const uint16_t* __r
   }
 }
 
+// MXFP4 check: out_f16 from the GEMM producers' routine; out_f32 from the
+// format's definition, value table times 2^(e - 127), written separately.
+__constant__ float kE2M1[16] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f,
+                                -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f};
+
+__global__ void decode_mxfp4_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s, int64_t n, int64_t k,
+                                    float* __restrict__ out_f32, uint16_t* __restrict__ out_f16) {
+  const int64_t groups = n * (k / 32);
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = g / (k / 32);
+    const int64_t grp = g - row * (k / 32);
+    const uint8_t* src = q + row * (k / 2) + grp * 16;
+    const uint32_t e = s[row * (k / 32) + grp];
+    uint4 qv;
+    uint8_t* qb = reinterpret_cast<uint8_t*>(&qv);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) qb[i] = src[i];
+    const int64_t o = row * k + grp * 32;
+    if (out_f16) {
+      const uint32_t hb = ue8m0_to_h(e);
+      uint32_t w[16];
+      decode_group32_mxfp4(qv, __halves2half2(*reinterpret_cast<const __half*>(&hb), *reinterpret_cast<const __half*>(&hb)), w);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        out_f16[o + 2 * i] = (uint16_t)(w[i] & 0xFFFFu);
+        out_f16[o + 2 * i + 1] = (uint16_t)(w[i] >> 16);
+      }
+    }
+    if (out_f32) {
+      const float sc = e == 0 ? 0.0f : (e == 255 ? INFINITY : ldexpf(1.0f, (int)e - 127));
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out_f32[o + i] = kE2M1[(qb[i >> 1] >> (4 * (i & 1))) & 15] * sc;
+    }
+  }
+}
+
 int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
   if (g > 148 * 16) g = 148 * 16;
@@ -224,6 +260,13 @@ cudaError_t launch_header_end_bwd(WsHeader* hdr, cudaStream_t stream) {
 cudaError_t launch_fill_u16(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream) {
   if (count <= 0) return cudaSuccess;
   fill_u16_kernel<<<grid_for(count, 256), 256, 0, stream>>>(p, count, value);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_mxfp4(const uint8_t* q, const uint8_t* s, int64_t n, int64_t k, float* out_f32,
+                                uint16_t* out_f16, cudaStream_t stream) {
+  if (n <= 0 || k <= 0) return cudaSuccess;
+  decode_mxfp4_kernel<<<grid_for(n * (k / 32), 128), 128, 0, stream>>>(q, s, n, k, out_f32, out_f16);
   return cudaGetLastError();
 }
 

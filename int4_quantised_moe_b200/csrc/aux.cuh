@@ -33,7 +33,9 @@ cudaError_t launch_header_end_bwd(WsHeader* hdr, cudaStream_t stream);
 // Zero `count` fp16/bf16 elements (generic 16-bit fill) and fp32 fill.
 cudaError_t launch_fill_u16(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream);
 
-// Bit-exact decode check export.
+// Bit-exact decode check exports (RAWINT4 with bf16 scales; MXFP4 with UE8M0 scale bytes).
+cudaError_t launch_decode_mxfp4(const uint8_t* q, const uint8_t* s, int64_t n, int64_t k, float* out_f32,
+                                uint16_t* out_f16, cudaStream_t stream);
 cudaError_t launch_decode(const uint8_t* q, const uint16_t* s, int64_t n, int64_t k, float* out_f32, uint16_t* out_f16,
                           cudaStream_t stream);
 

@@ -489,6 +489,41 @@ __device__ __forceinline__ void decode_group32(const uint4 q, const __half2 s2, 
   }
 }
 
+// ------------------------------------------------------------------ MXFP4
+// UE8M0 scale byte e -> fp16 bits of its value 2^(e - 127) (the pages' bit-cast
+// of e into a bf16 exponent). fp16 holds it exactly for e in [103, 142]
+// (normal for e >= 113, subnormal below); e == 0 -> 0, a larger e -> inf, a
+// smaller nonzero e -> 0 (outside the supported range).
+__device__ __forceinline__ uint32_t ue8m0_to_h(uint32_t e) {
+  if (e >= 113u && e <= 142u) return (e - 112u) << 10;
+  if (e >= 103u && e < 113u) return 1u << (e - 103u);
+  return e > 142u ? 0x7C00u : 0u;
+}
+
+// Two E2M1 codes (bits 0-3: first value, 4-7: second) -> fp16 pair, by the
+// hardware conversion (exact: every E2M1 value is an fp16 number).
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte_lo8) {
+  uint32_t d;
+  asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(d) : "r"(byte_lo8));
+  return d;
+}
+
+// Decode 16 packed bytes (32 E2M1 codes, low nibble first) that share one
+// group scale (fp16 pair `s2`) into 16 fp16x2 words, element order preserved.
+// Exact whenever the product is an fp16 number (scale bytes in [104, 140]).
+__device__ __forceinline__ void decode_group32_mxfp4(const uint4 q, const __half2 s2, uint32_t (&out)[16]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t v = e2m1x2_to_h2(w[i] >> (8 * j));
+      __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&v), s2);
+      out[i * 4 + j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+
 // Plain fp32 decode of one code (for the check export's fp32 output).
 __device__ __forceinline__ float decode_one_f32(uint8_t byte, int hi, uint16_t scale_bits) {
   const int code = hi ? (byte >> 4) : (byte & 15);

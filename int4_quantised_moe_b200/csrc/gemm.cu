@@ -216,7 +216,9 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int rb, 
     const uint16_t* src = nullptr;
     int jlo = 0;  // first reduction column holding this row's values
     if constexpr (MODE == kModeGateUp) {
-      src = (dt < 128 ? p.lx0 : p.lx1) + (int64_t)e * p.lx_expert + (int64_t)(f0 + (dt & 127)) * p.lx_ld;
+      // rows past the features (a partial last block) read nothing
+      if (f0 + (dt & 127) < p.feat)
+        src = (dt < 128 ? p.lx0 : p.lx1) + (int64_t)e * p.lx_expert + (int64_t)(f0 + (dt & 127)) * p.lx_ld;
       jlo = dt < 128 ? 0 : p.rpad;
     } else {
       if (f0 + dt < p.feat) src = p.lx0 + (int64_t)e * p.lx_expert + (int64_t)(f0 + dt) * p.lx_ld;
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int n = c0 + c;
-            if (n < n_rows) {
+            if (n < n_rows && i < p.feat) {
               const int64_t o = (int64_t)(p0 + n) * p.ld_out + i;
               const float g = __uint_as_float(v0[c]);
               const float u = __uint_as_float(v1[c]);
@@ -558,8 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a *= w;
                 b *= w;
               }
-              p.out_a[row * p.ld_out + f0 + m] = a;
-              if (two) p.out_a[row * p.ld_out + f0 + 128 + m] = b;
+              if (f0 + m < p.feat) p.out_a[row * p.ld_out + f0 + m] = a;  // a partial last block
+              if (two && f0 + 128 + m < p.feat) p.out_a[row * p.ld_out + f0 + 128 + m] = b;
             }
           }
         }

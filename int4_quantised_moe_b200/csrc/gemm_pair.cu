@@ -164,9 +164,11 @@ __device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, in
         row -= p.stored_rows;
         sp = p.s1;
       }
-      const bool ok = fc < p.feat;
-      const uint16_t* src = ok ? sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + fc / 32 : p.s0;
-      cp_async_8(S + kr * 8, src, ok ? 8u : 0u);
+      // groups past the features are zero (features come in multiples of 64)
+      const uint16_t* src = sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + fc / 32;
+      const bool ok0 = fc < p.feat, ok1 = fc + 64 < p.feat;
+      cp_async_4(S + kr * 8, ok0 ? src : p.s0, ok0 ? 4u : 0u);
+      cp_async_4(S + kr * 8 + 4, ok1 ? src + 2 : p.s0, ok1 ? 4u : 0u);
     }
   }
 }
@@ -512,21 +514,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_ld32(d_tmem + (uint32_t)c0, v);
             const float wl = __ldg(p.w_perm + p0 + min(c0 + lane, n_rows - 1));
             const int i = fc + m;
+            const bool row_live = i < p.feat;  // a partial last block
 #pragma unroll
             for (int cb = 0; cb < 32; cb += 4) {
               float gq[4], uq[4];
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 const int64_t row = p0 + min(c0 + cb + c, n_rows - 1);
-                gq[c] = __ldg(p.in_g + row * p.ld_out + i);
-                uq[c] = __ldg(p.in_u + row * p.ld_out + i);
+                gq[c] = row_live ? __ldg(p.in_g + row * p.ld_out + i) : 0.f;
+                uq[c] = row_live ? __ldg(p.in_u + row * p.ld_out + i) : 0.f;
               }
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 const int n = c0 + cb + c;
                 const float w = __shfl_sync(0xffffffffu, wl, cb + c);
                 float pr = 0.f;
-                if (n < n_rows) {
+                if (n < n_rows && row_live) {
                   const int64_t row = p0 + n;
                   const float acc_v = __uint_as_float(v[cb + c]);
                   const float g = gq[c];

@@ -47,9 +47,11 @@ def test_workspace_size_and_cfg_validation(lib):
     assert n > 0 and n % 256 == 0
     big = lib.make_cfg(4, 2, 256, 256, 8, 16.0, 0.0, 1000)
     assert lib.rawint4_moe_lora_workspace_size(big) > n
+    gemma = lib.make_cfg(128, 8, 2816, 704, 8, 16.0, 0.0, 32)  # H, I multiples of 64 (not of 128)
+    assert lib.rawint4_moe_lora_workspace_size(gemma) > 0
     bad = [
-        lib.make_cfg(4, 2, 200, 256, 8, 16.0, 0.0, 32),   # H not a multiple of 128
-        lib.make_cfg(4, 2, 256, 96, 8, 16.0, 0.0, 32),    # I not a multiple of 128
+        lib.make_cfg(4, 2, 200, 256, 8, 16.0, 0.0, 32),   # H not a multiple of 64
+        lib.make_cfg(4, 2, 256, 96, 8, 16.0, 0.0, 32),    # I not a multiple of 64
         lib.make_cfg(4, 5, 256, 256, 8, 16.0, 0.0, 32),   # top_k > experts
         lib.make_cfg(4, 2, 256, 256, 0, 16.0, 0.0, 32),   # rank 0
         lib.make_cfg(4, 2, 256, 256, 33, 16.0, 0.0, 32),  # rank > 32
@@ -137,4 +139,4 @@ def test_binding_rejects_wrong_tensors(lib):
     with pytest.raises(ValueError, match="shape"):
         create(gate_q=torch.zeros((E, I, H // 4), dtype=torch.uint8))
     with pytest.raises(lib.RawInt4Error):
-        lib.Layer.create(E, k, 200, I, r, 16.0, 0.0, 8, *q.values(), lora)  # H not a multiple of 128
+        lib.Layer.create(E, k, 200, I, r, 16.0, 0.0, 8, *q.values(), lora)  # H not a multiple of 64

@@ -74,3 +74,26 @@ def test_permutation_bit_exact(B, case):
     assert p[:n_valid].tolist() == ref_perm.tolist()
     assert np.all(p[n_valid:] == -1)
     assert inv.cpu().numpy().tolist() == ref_inv.tolist()
+
+
+@pytest.mark.parametrize("n,k", [(3, 64), (128, 7168), (33, 2048)])
+def test_mxfp4_decode_bit_exact(B, n, k):
+    """MXFP4 decode: fp32 output equals the oracle's E2M1 value times the
+    UE8M0 scale bit for bit; the fp16 tensor-core operand equals its fp16
+    rounding, which is exact for scale bytes in [104, 140] (all of them here,
+    plus the zero scale byte)."""
+    from oracle import mxfp4 as ofp4
+    gen = torch.Generator().manual_seed(n * 7 + k)
+    q = torch.randint(0, 256, (n, k // 2), generator=gen, dtype=torch.uint8)
+    s = torch.randint(104, 141, (n, k // 32), generator=gen, dtype=torch.uint8)
+    q[0, :16] = torch.arange(16, dtype=torch.uint8) * 17  # every code, in both nibbles
+    s[0, 0] = 0
+    out32 = torch.empty((n, k), dtype=torch.float32, device="cuda")
+    out16 = torch.empty((n, k), dtype=torch.float16, device="cuda")
+    B.rawint4_mxfp4_decode(q.cuda(), s.cuda(), out32, out16)
+    torch.cuda.synchronize()
+    ref = ofp4.dequantize_mxfp4(q.numpy(), s.numpy())
+    assert np.array_equal(out32.cpu().double().numpy(), ref)
+    ref16 = ref.astype(np.float16)
+    assert np.array_equal(ref16.astype(np.float64), ref)
+    assert np.array_equal(out16.cpu().numpy().view(np.uint16), ref16.view(np.uint16))

@@ -410,3 +410,25 @@ def test_wait_timeout_aborts_cleanly():
     close("grad_route", groute, groute_r, TOL_ROUTE)
     for n in LORA_NAMES:
         close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("limit", [0.0, 5.0])
+def test_gemma4_shape_parity(limit):
+    """The adjacent MoE system's layer shape (test_gemma4_moe.py,
+    TestGemma4FullLayerIntegration.real_config: hidden 2816, 128 experts,
+    top-8, intermediate 704). H and I are multiples of 64 but I is not one of
+    128 or 256, so the last output-feature block of gate/up and of down^T is
+    partial and its missing rows must neither be read nor written."""
+    cfg = small_config("gemma4", 128, 8, 2816, 704, 8, 48, swiglu_limit=limit, routing="normal_topk", x_std=1.0)
+    wl = make_workload(cfg, seed=2026)
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
