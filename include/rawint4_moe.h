@@ -79,9 +79,19 @@ enum {
  * LoRA rank r and alpha (scaling c = alpha / r), swiglu_limit L (0 disables
  * the clamp; must be finite and >= 0) and max_tokens (the largest qlen a
  * workspace is sized for; the reference's max_len).
+ * weight_format selects the frozen base format: RAWINT4 (the method) or the
+ * pages' sibling MXFP4 format (the ext_bindings.cpp commit log's MXFP4
+ * routed-expert LoRA path: E2M1 codes with UE8M0 group scales; only the
+ * dequantisation differs, the LoRA, clamp, transpose-free dX and gradient
+ * window are the same).
  * Limits: H % 64 == 0, I % 64 == 0 (the kernels reduce in stages of 64 and
- * mask a partial last block of output features), 1 <= rank <= 32,
- * 1 <= top_k <= experts. */
+ * mask a partial last block of output features; MXFP4: H % 128 == 0 and
+ * I % 128 == 0, its scale bytes are fetched four at a time),
+ * 1 <= rank <= 32, 1 <= top_k <= experts. */
+enum {
+  RAWINT4_FORMAT_RAWINT4 = 0, /* codes 0..15 -> (code - 8) * bf16 scale */
+  RAWINT4_FORMAT_MXFP4 = 1    /* E2M1 codes * 2^(e - 127), e a UE8M0 scale byte */
+};
 typedef struct rawint4_moe_cfg {
   int32_t experts;
   int32_t top_k;
@@ -91,18 +101,21 @@ typedef struct rawint4_moe_cfg {
   float alpha;
   float swiglu_limit;
   int32_t max_tokens;
+  int32_t weight_format; /* RAWINT4_FORMAT_*; 0 = RAWINT4 */
 } rawint4_moe_cfg;
 
 /* Frozen base weights (device, read-only; never written).
- * gate_q, up_q: uint8 [E, I, H/2]; gate_s, up_s: bf16 [E, I, H/32]
- * down_q:       uint8 [E, H, I/2]; down_s:       bf16 [E, H, I/32]
+ * gate_q, up_q: uint8 [E, I, H/2]; gate_s, up_s: [E, I, H/32]
+ * down_q:       uint8 [E, H, I/2]; down_s:       [E, H, I/32]
  * Layout of one projection: rawint4_sft_reference.py, _validate_rawint4_layout
- * (packed uint8 [N_out, K_in/2], scales bf16 [N_out, K_in/32]). */
+ * (packed uint8 [N_out, K_in/2], one scale per 32 inputs). Scales are bf16
+ * for RAWINT4 and UE8M0 bytes (uint8) for MXFP4; both formats pack two codes
+ * per byte, low nibble first. */
 /* Every base and LoRA pointer must be 16-byte aligned (RAWINT4_INVALID_ARGUMENT
  * otherwise): the kernels read them with TMA and 16-byte vector loads. */
 typedef struct rawint4_moe_base {
   const uint8_t *gate_q, *up_q, *down_q;
-  const uint16_t *gate_s, *up_s, *down_s;
+  const void *gate_s, *up_s, *down_s;
 } rawint4_moe_base;
 
 /* LoRA adapters (device, bf16), the six tensors of the contract test

@@ -57,7 +57,7 @@ EXPORTED_SYMBOLS = (
 class Cfg(ctypes.Structure):
     _fields_ = [("experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("hidden", ctypes.c_int32),
                 ("inter", ctypes.c_int32), ("rank", ctypes.c_int32), ("alpha", ctypes.c_float),
-                ("swiglu_limit", ctypes.c_float), ("max_tokens", ctypes.c_int32)]
+                ("swiglu_limit", ctypes.c_float), ("max_tokens", ctypes.c_int32), ("weight_format", ctypes.c_int32)]
 
 
 class Base(ctypes.Structure):
@@ -148,9 +148,14 @@ def _stream(stream) -> Optional[int]:
     return int(stream)
 
 
-def make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens) -> Cfg:
+FORMAT_RAWINT4 = 0
+FORMAT_MXFP4 = 1
+FORMATS = {"rawint4": FORMAT_RAWINT4, "mxfp4": FORMAT_MXFP4}
+
+
+def make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens, weight_format="rawint4") -> Cfg:
     return Cfg(int(experts), int(top_k), int(hidden), int(inter), int(rank), float(alpha), float(swiglu_limit),
-               int(max_tokens))
+               int(max_tokens), FORMATS[weight_format])
 
 
 def rawint4_moe_lora_workspace_size(cfg: Cfg) -> int:
@@ -277,17 +282,19 @@ class Layer:
 
     @classmethod
     def create(cls, experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens, gate_q, gate_s, up_q, up_s,
-               down_q, down_s, lora: Dict[str, torch.Tensor], device=None):
-        cfg = make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens)
+               down_q, down_s, lora: Dict[str, torch.Tensor], device=None, weight_format="rawint4"):
+        """weight_format "rawint4" (bf16 scales) or "mxfp4" (E2M1 codes, UE8M0 scale bytes, uint8)."""
+        cfg = make_cfg(experts, top_k, hidden, inter, rank, alpha, swiglu_limit, max_tokens, weight_format)
         nbytes = rawint4_moe_lora_workspace_size(cfg)  # validates the configuration
         dev = device if device is not None else gate_q.device
         E, H, I = int(experts), int(hidden), int(inter)
+        sdt = torch.uint8 if weight_format == "mxfp4" else torch.bfloat16
         for name, t, dt, shape in (("gate_q", gate_q, torch.uint8, (E, I, H // 2)),
                                    ("up_q", up_q, torch.uint8, (E, I, H // 2)),
                                    ("down_q", down_q, torch.uint8, (E, H, I // 2)),
-                                   ("gate_s", gate_s, torch.bfloat16, (E, I, H // 32)),
-                                   ("up_s", up_s, torch.bfloat16, (E, I, H // 32)),
-                                   ("down_s", down_s, torch.bfloat16, (E, H, I // 32))):
+                                   ("gate_s", gate_s, sdt, (E, I, H // 32)),
+                                   ("up_s", up_s, sdt, (E, I, H // 32)),
+                                   ("down_s", down_s, sdt, (E, H, I // 32))):
             _expect(t, name, dt, shape, gate_q.device)
         for name, shape in lora_tensor_shapes(E, H, I, int(rank)).items():
             if name not in lora:

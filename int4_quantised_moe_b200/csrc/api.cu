@@ -87,6 +87,8 @@ bool cfg_ok(const rawint4_moe_cfg* c) {
   if (!std::isfinite(c->alpha)) return false;
   if (!std::isfinite(c->swiglu_limit) || c->swiglu_limit < 0.f) return false;
   if (c->max_tokens < 1) return false;
+  if (c->weight_format != RAWINT4_FORMAT_RAWINT4 && c->weight_format != RAWINT4_FORMAT_MXFP4) return false;
+  if (c->weight_format == RAWINT4_FORMAT_MXFP4 && (c->hidden % 128 != 0 || c->inter % 128 != 0)) return false;
   if ((int64_t)c->max_tokens * c->top_k > (1 << 24)) return false;
   return true;
 }
@@ -242,30 +244,30 @@ int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
 }
 
 // CTA pairs for a launch of the tensor-memory GEMM (gemm_tm.cu).
-int tm_clusters(int mode, int sms, int max_tiles, int rowblk) {
-  static std::atomic<int> cached[64][4];  // per device and mode; 0 = not queried yet
+int tm_clusters(int mode, int fmt, int sms, int max_tiles, int rowblk) {
+  static std::atomic<int> cached[64][2][4];  // per device, format and mode; 0 = not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  int fit = cached[dev][mode].load();
+  int fit = cached[dev][fmt][mode].load();
   if (fit <= 0) {
-    const int n = gemm_tm_max_clusters(mode);
+    const int n = gemm_tm_max_clusters(mode, fmt);
     fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);
-    cached[dev][mode].store(fit);
+    cached[dev][fmt][mode].store(fit);
   }
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }
 
-// Which GEMM kernels run: the tensor-memory pair kernels (gemm_tm.cu) when
-// the environment selects them (RAWINT4_GEMM=tm), the shared-memory operand
-// kernels (gemm.cu, gemm_pair.cu) otherwise.
-bool use_tm_forward() {
+// Which GEMM kernels run: the tensor-memory pair kernels (gemm_tm.cu) for an
+// MXFP4 base or when the environment selects them (RAWINT4_GEMM=tm), the
+// shared-memory operand kernels (gemm.cu, gemm_pair.cu) otherwise.
+bool use_tm_gemm(int fmt) {
   static int v = -1;
   if (v < 0) {
     const char* e = getenv("RAWINT4_GEMM");
     v = (e && strcmp(e, "tm") == 0) ? 1 : 0;
   }
-  return v == 1;
+  return v == 1 || fmt == RAWINT4_FORMAT_MXFP4;
 }
 
 // Bound on any pipeline wait of the GEMM kernels (test export can shorten it).
@@ -400,7 +402,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.limit = c.swiglu_limit;
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
-  const bool tm = use_tm_forward();
+  const int fmt = c.weight_format;
+  const bool tm = use_tm_gemm(fmt);
   // tensor-memory kernel: boxes of 64 rows x 128 bytes (4 reduction stages)
   if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
       !map_packed(&mp.q1, base->up_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
@@ -410,8 +413,10 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.n_rowblk = (I + 127) / 128;
   gp.feat = I;
   gp.n_main = H / kBlockK;
-  gp.s0 = base->gate_s;
-  gp.s1 = base->up_s;
+  gp.s0 = static_cast<const uint16_t*>(base->gate_s);
+  gp.s1 = static_cast<const uint16_t*>(base->up_s);
+  gp.e0 = static_cast<const uint8_t*>(base->gate_s);
+  gp.e1 = static_cast<const uint8_t*>(base->up_s);
   gp.s_expert = (int64_t)I * (H / 32);
   gp.s_row = H / 32;
   gp.stored_rows = I;
@@ -426,7 +431,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_gate_up", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeGateUp, gp, mp, tm_clusters(kModeGateUp, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeGateUp, fmt, gp, mp, tm_clusters(kModeGateUp, fmt, sms, max_tiles, gp.n_rowblk), st));
     else
       R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
@@ -455,7 +460,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.n_rowblk = (H + 255) / 256;
   gp.feat = H;
   gp.n_main = I / kBlockK;
-  gp.s0 = gp.s1 = base->down_s;
+  gp.s0 = gp.s1 = static_cast<const uint16_t*>(base->down_s);
+  gp.e0 = gp.e1 = static_cast<const uint8_t*>(base->down_s);
   gp.s_expert = (int64_t)H * (I / 32);
   gp.s_row = I / 32;
   gp.stored_rows = H;
@@ -469,7 +475,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_down", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeDown, gp, mp, tm_clusters(kModeDown, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeDown, fmt, gp, mp, tm_clusters(kModeDown, fmt, sms, max_tiles, gp.n_rowblk), st));
     else
       R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }
@@ -569,14 +575,16 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.wait_ns = g_wait_ns.load();
 
   // down, transpose-free: dh = w (g W_d + gd A_d); SwiGLU' -> dG | dU; dRoute partials
-  const bool tm = use_tm_forward();
+  const int fmt = c.weight_format;
+  const bool tm = use_tm_gemm(fmt);
   if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 64, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 64, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.gp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gd), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (I + 255) / 256;
   gp.feat = I;
   gp.n_main = H / kBlockK;
-  gp.s0 = gp.s1 = base->down_s;
+  gp.s0 = gp.s1 = static_cast<const uint16_t*>(base->down_s);
+  gp.e0 = gp.e1 = static_cast<const uint8_t*>(base->down_s);
   gp.s_expert = (int64_t)H * (I / 32);
   gp.s_row = I / 32;
   gp.stored_rows = H;
@@ -594,7 +602,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_down_t", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeDownT, gp, mp, tm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeDownT, fmt, gp, mp, tm_clusters(kModeDownT, fmt, sms, max_tiles, gp.n_rowblk), st));
     else
       R4_TRY(launch_gemm_pair(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
   }
@@ -624,8 +632,10 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.n_rowblk = (H + 255) / 256;
   gp.feat = H;
   gp.n_main = 2 * I / kBlockK;
-  gp.s0 = base->gate_s;
-  gp.s1 = base->up_s;
+  gp.s0 = static_cast<const uint16_t*>(base->gate_s);
+  gp.s1 = static_cast<const uint16_t*>(base->up_s);
+  gp.e0 = static_cast<const uint8_t*>(base->gate_s);
+  gp.e1 = static_cast<const uint8_t*>(base->up_s);
   gp.s_expert = (int64_t)I * (H / 32);
   gp.s_row = H / 32;
   gp.stored_rows = I;
@@ -641,7 +651,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_gate_up_t", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeGateUpT, gp, mp, tm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeGateUpT, fmt, gp, mp, tm_clusters(kModeGateUpT, fmt, sms, max_tiles, gp.n_rowblk), st));
     else
       R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
   }

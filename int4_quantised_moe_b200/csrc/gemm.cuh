@@ -35,6 +35,8 @@ struct GemmParams {
   // frozen base scales of projection 0 and 1 (bf16)
   const uint16_t* s0;
   const uint16_t* s1;
+  const uint8_t* e0;         // MXFP4 base (gemm_tm.cu): UE8M0 scale bytes of projection 0 and 1
+  const uint8_t* e1;
   int64_t s_expert;          // scale elements per expert
   int s_row;                 // scales per stored row
   int stored_rows;           // stored rows per expert of one projection
@@ -73,8 +75,11 @@ cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
 // CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
 int gemm_pair_max_clusters(int mode);
-// CTA pairs with the decoded weights in tensor memory (gemm_tm.cu): gate/up and down.
-cudaError_t launch_gemm_tm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
-int gemm_tm_max_clusters(int mode);
+// CTA pairs with the decoded weights in tensor memory (gemm_tm.cu), every
+// mode; fmt: RAWINT4_FORMAT_RAWINT4 (bf16 scales s0/s1) or
+// RAWINT4_FORMAT_MXFP4 (E2M1 codes, UE8M0 scale bytes e0/e1).
+cudaError_t launch_gemm_tm(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+                           cudaStream_t stream);
+int gemm_tm_max_clusters(int mode, int fmt);
 
 }  // namespace r4

@@ -199,9 +199,32 @@ __device__ __forceinline__ void grace_wait() {
 // K-major scale slot j: [128 rows][8] bf16, the groups 8j..8j+7 of each
 // weight row (its two groups of each of the slot's 4 stages); entries past the
 // features or the reduction are zero.
-template <int MODE>
+template <int MODE, int FMT>
 __device__ __forceinline__ void load_slot_scales(const GemmParams& p, int e, int fc, int j, int n_main, int ln,
                                                  uint8_t* S) {
+  if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {
+    // UE8M0 bytes: [128 rows][8], 4 bytes (two stages) per copy; rows are
+    // 4-byte aligned (K % 128 == 0)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int row = ln + 32 * t;
+      const uint8_t* ep = p.e0;
+      int f;
+      if constexpr (MODE == kModeGateUp) {
+        ep = row < 64 ? p.e0 : p.e1;
+        f = fc + (row & 63);
+      } else {
+        f = fc + row;
+      }
+      const bool ok = f < p.feat;
+      const uint8_t* src = ep + (int64_t)e * p.s_expert + (int64_t)f * p.s_row + 8 * j;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const bool v = ok && 4 * j + 2 * h < n_main;
+        cp_async_4(S + row * 8 + 4 * h, v ? src + 4 * h : p.e0, v ? 4u : 0u);
+      }
+    }
+  } else {
   const bool full = 4 * j + 4 <= n_main && (p.s_row & 7) == 0;  // 16-byte aligned whole slot
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
@@ -226,14 +249,29 @@ __device__ __forceinline__ void load_slot_scales(const GemmParams& p, int e, int
       }
     }
   }
+  }
 }
 
-// MN-major scale slot j: [128 stored rows][4] bf16, the group scales of this
-// CTA's 128 weight rows (4 groups of 32) at each stored row of the slot's two
-// stages (stored rows past the reduction are not read).
-template <int MODE>
+template <int MODE, int FMT>
 __device__ __forceinline__ void load_slot_scales_mn(const GemmParams& p, int e, int fc, int j, int n_main, int ln,
                                                     uint8_t* S) {
+  if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {
+    // UE8M0 bytes: [128 stored rows][4] (this CTA's 4 groups; features and
+    // stored rows are multiples of 128 for MXFP4, so a group is all in or out)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int kr = ln + 32 * t;
+      if (2 * j + (kr >> 6) >= n_main) continue;
+      int row = 2 * j * kBlockK + kr;
+      const uint8_t* ep = p.e0;
+      if (MODE == kModeGateUpT && row >= p.stored_rows) {
+        row -= p.stored_rows;
+        ep = p.e1;
+      }
+      const bool ok = fc < p.feat;
+      cp_async_4(S + kr * 4, ok ? ep + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + fc / 32 : p.e0, ok ? 4u : 0u);
+    }
+  } else {
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     const int kr = ln + 32 * t;
@@ -250,6 +288,7 @@ __device__ __forceinline__ void load_slot_scales_mn(const GemmParams& p, int e, 
     const bool ok0 = fc < p.feat, ok1 = fc + 64 < p.feat;
     cp_async_4(S + kr * 8, ok0 ? src : p.s0, ok0 ? 4u : 0u);
     cp_async_4(S + kr * 8 + 4, ok1 ? src + 2 : p.s0, ok1 ? 4u : 0u);
+  }
   }
 }
 
@@ -345,6 +384,20 @@ __device__ __forceinline__ void decode_pairs32(const uint32_t (&w)[4], const uin
   }
 }
 
+// As decode_pairs32 for E2M1 codes (hardware conversion of each byte).
+__device__ __forceinline__ void decode_pairs32_mxfp4(const uint32_t (&w)[4], const uint32_t (&sc)[16],
+                                                     uint32_t (&out)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t v = e2m1x2_to_h2(w[i] >> (8 * j));
+      __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&v), *reinterpret_cast<const __half2*>(&sc[i * 4 + j]));
+      out[i * 4 + j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -405,7 +458,7 @@ __device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int f
   }
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
   const CUtensorMap& tq0 = maps.q0;
@@ -546,9 +599,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int j = rotated(j0, rot, n_slots);
         if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         if constexpr (kAMnMajor<MODE>)
-          load_slot_scales_mn<MODE>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
+          load_slot_scales_mn<MODE, FMT>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
         else
-          load_slot_scales<MODE>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
+          load_slot_scales<MODE, FMT>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
         cp_async_arrive_noinc(&s_full[ring.stage]);
         ring.advance(kStagesS);
       }
@@ -808,23 +861,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // scale of this thread's group: K-major [128 rows][8] (2 per stage),
     // MN-major [128 stored rows][4 groups]
     auto s_off = [&](int u) -> uint32_t {
-      if constexpr (kAMnMajor<MODE>)
+      if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {  // scale bytes
+        if constexpr (kAMnMajor<MODE>)
+          return (uint32_t)((64 * u + 32 * g + lane) * 4 + q);
+        else
+          return (uint32_t)(m * 8 + 2 * u + g);
+      } else if constexpr (kAMnMajor<MODE>) {
         return (uint32_t)((64 * u + 32 * g + lane) * 8 + 2 * q);
-      else
+      } else {
         return (uint32_t)(m * 16 + (2 * u + g) * 2);
+      }
     };
     uint32_t* tab = reinterpret_cast<uint32_t*>(smem + kOffScaleTab) + 32 * (warp - kDecWarp0);
     Ring ra, rp, rs;
     // Decodes sub-stage u of packed slot rp / scale slot rs into w; table `tb`
     // holds the MN-major scale pairs.
     auto decode_stage = [&](const Ring& rs_, const Ring& rp_, int u, uint32_t* tb, uint32_t (&w)[16]) {
-      const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs_.stage * kSSlotBytes + s_off(u));
+      const uint8_t* sptr = sS + rs_.stage * kSSlotBytes + s_off(u);
+      // fp16 bits of this thread's group scale
+      uint32_t hb;
+      if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {
+        hb = ue8m0_to_h(*sptr);
+      } else {
+        const __half hs = __float2half_rn(bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(sptr)));
+        hb = (uint32_t)(*reinterpret_cast<const uint16_t*>(&hs));
+      }
       const uint4 q4 = *reinterpret_cast<const uint4*>(sP + rp_.stage * kPBytes<MODE> + p_off(u));
       if constexpr (kAMnMajor<MODE>) {
         // every stored row has its own scale: pair them up (lane 2t holds
         // the scales of values 2t and 2t + 1) through a per-warp table
-        const __half hs = __float2half_rn(bf16_bits_to_float(sc));
-        const uint32_t hb = (uint32_t)(*reinterpret_cast<const uint16_t*>(&hs));
         const uint32_t nb = __shfl_down_sync(0xffffffffu, hb, 1);
         if ((lane & 1) == 0) tb[lane >> 1] = hb | (nb << 16);
         __syncwarp();
@@ -839,9 +904,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         uint32_t nib[4] = {q4.x, q4.y, q4.z, q4.w};
         transpose_nibbles(nib, lane);
-        decode_pairs32(nib, sp2, w);
+        if constexpr (FMT == RAWINT4_FORMAT_MXFP4)
+          decode_pairs32_mxfp4(nib, sp2, w);
+        else
+          decode_pairs32(nib, sp2, w);
       } else {
-        decode_group32(q4, bf16_scale_to_h2(sc), w);
+        const uint32_t h2 = hb | (hb << 16);
+        if constexpr (FMT == RAWINT4_FORMAT_MXFP4)
+          decode_group32_mxfp4(q4, *reinterpret_cast<const __half2*>(&h2), w);
+        else
+          decode_group32(q4, *reinterpret_cast<const __half2*>(&h2), w);
       }
     };
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
@@ -919,12 +991,12 @@ done:
   if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 bool set_smem_attr() {
   static std::atomic<unsigned long long> done{0};
   int dev = 0;
   if (!device_flag_test(done, &dev)) {
-    if (cudaFuncSetAttribute(gemm_tm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+    if (cudaFuncSetAttribute(gemm_tm_kernel<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
       return false;
     device_flag_set(done, dev);
@@ -932,16 +1004,16 @@ bool set_smem_attr() {
   return true;
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 cudaError_t launch_mode(const GemmParams& p, const GemmMaps& m, int clusters, cudaStream_t stream) {
-  if (!set_smem_attr<MODE>()) return cudaErrorInvalidValue;
-  gemm_tm_kernel<MODE><<<2 * clusters, kThreads, kSmemBytes, stream>>>(p, m);
+  if (!set_smem_attr<MODE, FMT>()) return cudaErrorInvalidValue;
+  gemm_tm_kernel<MODE, FMT><<<2 * clusters, kThreads, kSmemBytes, stream>>>(p, m);
   return cudaGetLastError();
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 int max_clusters_mode() {
-  if (!set_smem_attr<MODE>()) return 0;
+  if (!set_smem_attr<MODE, FMT>()) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -954,28 +1026,39 @@ int max_clusters_mode() {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tm_kernel<MODE>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tm_kernel<MODE, FMT>, &cfg) != cudaSuccess) return 0;
   return n;
 }
 
 }  // namespace tmk
 
-cudaError_t launch_gemm_tm(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
-  switch (mode) {
-    case kModeGateUp: return tmk::launch_mode<kModeGateUp>(p, maps, clusters, stream);
-    case kModeDown: return tmk::launch_mode<kModeDown>(p, maps, clusters, stream);
-    case kModeDownT: return tmk::launch_mode<kModeDownT>(p, maps, clusters, stream);
-    case kModeGateUpT: return tmk::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
+cudaError_t launch_gemm_tm(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+                           cudaStream_t stream) {
+  constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
+  switch (mode * 2 + (fmt == X ? 1 : 0)) {
+    case kModeGateUp * 2: return tmk::launch_mode<kModeGateUp, R>(p, maps, clusters, stream);
+    case kModeGateUp * 2 + 1: return tmk::launch_mode<kModeGateUp, X>(p, maps, clusters, stream);
+    case kModeDown * 2: return tmk::launch_mode<kModeDown, R>(p, maps, clusters, stream);
+    case kModeDown * 2 + 1: return tmk::launch_mode<kModeDown, X>(p, maps, clusters, stream);
+    case kModeDownT * 2: return tmk::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
+    case kModeDownT * 2 + 1: return tmk::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
+    case kModeGateUpT * 2: return tmk::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
+    case kModeGateUpT * 2 + 1: return tmk::launch_mode<kModeGateUpT, X>(p, maps, clusters, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-int gemm_tm_max_clusters(int mode) {
-  switch (mode) {
-    case kModeGateUp: return tmk::max_clusters_mode<kModeGateUp>();
-    case kModeDown: return tmk::max_clusters_mode<kModeDown>();
-    case kModeDownT: return tmk::max_clusters_mode<kModeDownT>();
-    case kModeGateUpT: return tmk::max_clusters_mode<kModeGateUpT>();
+int gemm_tm_max_clusters(int mode, int fmt) {
+  constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
+  switch (mode * 2 + (fmt == X ? 1 : 0)) {
+    case kModeGateUp * 2: return tmk::max_clusters_mode<kModeGateUp, R>();
+    case kModeGateUp * 2 + 1: return tmk::max_clusters_mode<kModeGateUp, X>();
+    case kModeDown * 2: return tmk::max_clusters_mode<kModeDown, R>();
+    case kModeDown * 2 + 1: return tmk::max_clusters_mode<kModeDown, X>();
+    case kModeDownT * 2: return tmk::max_clusters_mode<kModeDownT, R>();
+    case kModeDownT * 2 + 1: return tmk::max_clusters_mode<kModeDownT, X>();
+    case kModeGateUpT * 2: return tmk::max_clusters_mode<kModeGateUpT, R>();
+    case kModeGateUpT * 2 + 1: return tmk::max_clusters_mode<kModeGateUpT, X>();
     default: return 0;
   }
 }

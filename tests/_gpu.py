@@ -28,7 +28,7 @@ def make_layer(wl: Workload, max_tokens: Optional[int] = None) -> "B.Layer":
     c = wl.cfg
     return B.Layer.create(c.experts, c.top_k, c.hidden, c.inter, c.rank, c.alpha, c.swiglu_limit,
                           max_tokens or max(c.qlen, 1), wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s,
-                          wl.lora)
+                          wl.lora, weight_format=c.weight_format)
 
 
 def grad_buffers(wl: Workload, fill: float = 7.0) -> Dict[str, torch.Tensor]:

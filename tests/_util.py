@@ -33,13 +33,16 @@ def u8(t: torch.Tensor) -> np.ndarray:
 def oracle_layer(wl: Workload, lazy_scales: bool = False) -> omoe.Layer:
     """``lazy_scales`` keeps scales as bf16 bit patterns (widened per expert)."""
     c = wl.cfg
-    sc = bf16_bits if lazy_scales else f64
+    if c.weight_format == "mxfp4":
+        sc = u8  # UE8M0 scale bytes, as stored
+    else:
+        sc = bf16_bits if lazy_scales else f64
     return omoe.Layer(
         gate_q=u8(wl.gate_q), gate_s=sc(wl.gate_s),
         up_q=u8(wl.up_q), up_s=sc(wl.up_s),
         down_q=u8(wl.down_q), down_s=sc(wl.down_s),
         lora={n: f64(wl.lora[n]) for n in LORA_NAMES},
-        alpha=c.alpha, swiglu_limit=c.swiglu_limit,
+        alpha=c.alpha, swiglu_limit=c.swiglu_limit, weight_format=c.weight_format,
     )
 
 

@@ -432,3 +432,34 @@ def test_gemma4_shape_parity(limit):
     close("grad_route", groute, groute_r, TOL_ROUTE)
     for n in LORA_NAMES:
         close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("cfg_id,limit", [(0, 0.0), (1, 2.0), (1, 0.0)])
+def test_mxfp4_base_parity(cfg_id, limit):
+    """The sibling MXFP4 base (E2M1 codes, UE8M0 group scales; the
+    ext_bindings.cpp commit log's MXFP4 routed-expert LoRA kernels): the same
+    layer, LoRA, clamp, transpose-free backward and gradient window with
+    only the dequantisation changed, against the oracle's MXFP4 layer."""
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS[cfg_id], weight_format="mxfp4", swiglu_limit=limit)
+    wl = make_workload(cfg)
+    assert wl.gate_s.dtype == torch.uint8
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+    # frozen-base inference forward of the MXFP4 layer
+    zero_b = {n: (torch.zeros_like(t) if n.endswith("_b") else t) for n, t in wl.lora.items()}
+    zb = Workload(wl.cfg, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, zero_b, wl.x,
+                  wl.expert_ids, wl.route_weights, wl.grad_out)
+    base_r, _ = omoe.forward(oracle_layer(zb), f64(zb.x), zb.expert_ids.numpy(), f64(zb.route_weights))
+    base = layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False, use_lora=False)
+    assert layer.status() == 0
+    close("base_only.out", base, base_r, TOL_OUT)

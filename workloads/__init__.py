@@ -44,6 +44,7 @@ class LayerConfig:
     x_std: float = 1.0
     lora_std: float = 0.02
     zipf_s: float = 1.1
+    weight_format: str = "rawint4"  # or "mxfp4": E2M1 codes, UE8M0 scale bytes
 
     @property
     def routed(self) -> int:
@@ -112,6 +113,17 @@ def _scales(shape, gen, device):
     return (torch.rand(shape, generator=gen, dtype=torch.float32, device=device) * 0.06 + 0.01).to(torch.bfloat16)
 
 
+# MXFP4 scale bytes: 2^(e - 127) for e in [119, 123], i.e. group scales from
+# 2^-8 to 2^-4; with E2M1 magnitudes up to 6 the weights span the same range
+# as the RAWINT4 ones ((code - 8) times a scale in [0.01, 0.07)).
+MXFP4_SCALE_BYTES = (119, 124)
+
+
+def _scale_bytes(shape, gen, device):
+    return torch.randint(MXFP4_SCALE_BYTES[0], MXFP4_SCALE_BYTES[1], shape, generator=gen, dtype=torch.uint8,
+                         device=device)
+
+
 def _normal_bf16(shape, std, gen, device):
     return (torch.randn(shape, generator=gen, dtype=torch.float32, device=device) * std).to(torch.bfloat16)
 
@@ -119,19 +131,22 @@ def _normal_bf16(shape, std, gen, device):
 def make_base(cfg: LayerConfig, gen: torch.Generator, device="cpu"):
     """Draw gate/up/down packed bytes and scales, expert by expert."""
     E, H, I = cfg.experts, cfg.hidden, cfg.inter
+    mx = cfg.weight_format == "mxfp4"
+    sdt = torch.uint8 if mx else torch.bfloat16
+    draw_s = _scale_bytes if mx else _scales
     gate_q = torch.empty((E, I, H // 2), dtype=torch.uint8, device=device)
     up_q = torch.empty_like(gate_q)
     down_q = torch.empty((E, H, I // 2), dtype=torch.uint8, device=device)
-    gate_s = torch.empty((E, I, H // GROUP), dtype=torch.bfloat16, device=device)
+    gate_s = torch.empty((E, I, H // GROUP), dtype=sdt, device=device)
     up_s = torch.empty_like(gate_s)
-    down_s = torch.empty((E, H, I // GROUP), dtype=torch.bfloat16, device=device)
+    down_s = torch.empty((E, H, I // GROUP), dtype=sdt, device=device)
     for e in range(E):
         gate_q[e] = _uniform_bytes((I, H // 2), gen, device)
-        gate_s[e] = _scales((I, H // GROUP), gen, device)
+        gate_s[e] = draw_s((I, H // GROUP), gen, device)
         up_q[e] = _uniform_bytes((I, H // 2), gen, device)
-        up_s[e] = _scales((I, H // GROUP), gen, device)
+        up_s[e] = draw_s((I, H // GROUP), gen, device)
         down_q[e] = _uniform_bytes((H, I // 2), gen, device)
-        down_s[e] = _scales((H, I // GROUP), gen, device)
+        down_s[e] = draw_s((H, I // GROUP), gen, device)
     return gate_q, gate_s, up_q, up_s, down_q, down_s
 
 
@@ -207,6 +222,6 @@ def expert_counts(expert_ids: torch.Tensor, experts: int) -> torch.Tensor:
 
 
 def small_config(name, experts, top_k, hidden, inter, rank, qlen, swiglu_limit=0.0, routing="normal_topk",
-                 alpha=None, x_std=1.0) -> LayerConfig:
+                 alpha=None, x_std=1.0, weight_format="rawint4") -> LayerConfig:
     return LayerConfig(name, experts, top_k, hidden, inter, rank, float(alpha if alpha is not None else 2 * rank),
-                       qlen, swiglu_limit, routing, x_std=x_std)
+                       qlen, swiglu_limit, routing, x_std=x_std, weight_format=weight_format)
