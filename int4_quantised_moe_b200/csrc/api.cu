@@ -258,9 +258,11 @@ int tm_clusters(int mode, int fmt, int sms, int max_tiles, int rowblk) {
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }
 
-// Which GEMM kernels run: the tensor-memory pair kernels (gemm_tm.cu) for an
-// MXFP4 base or when the environment selects them (RAWINT4_GEMM=tm), the
-// shared-memory operand kernels (gemm.cu, gemm_pair.cu) otherwise.
+// Which kernel runs the transpose-free backward GEMMs (down^T, gate/up^T):
+// the shared-memory operand pair kernel (gemm_pair.cu: MN-major decoded
+// tiles, no transposition), or the tensor-memory pair kernel (gemm_tm.cu) for
+// an MXFP4 base or when the environment selects it (RAWINT4_GEMM=tm). The
+// forward GEMMs always run on the tensor-memory kernel.
 bool use_tm_gemm(int fmt) {
   static int v = -1;
   if (v < 0) {
@@ -403,10 +405,9 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
 
   // gate/up: G, U (fp32, saved) and h = silu(G') U' (fp16)
   const int fmt = c.weight_format;
-  const bool tm = use_tm_gemm(fmt);
   // tensor-memory kernel: boxes of 64 rows x 128 bytes (4 reduction stages)
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
-      !map_packed(&mp.q1, base->up_q, E, I, H / 2, tm ? 128 : 32, tm ? 64 : 128) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 128, 64) ||
+      !map_packed(&mp.q1, base->up_q, E, I, H / 2, 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.xp), L.rows, H) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.xa), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.wait_ns = g_wait_ns.load();
@@ -430,10 +431,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_gate_up", st);
-    if (tm)
-      R4_TRY(launch_gemm_tm(kModeGateUp, fmt, gp, mp, tm_clusters(kModeGateUp, fmt, sms, max_tiles, gp.n_rowblk), st));
-    else
-      R4_TRY(launch_gemm(kModeGateUp, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm_tm(kModeGateUp, fmt, gp, mp, tm_clusters(kModeGateUp, fmt, sms, max_tiles, gp.n_rowblk), st));
   }
 
   // ha = c * h A_d^T and hw = w * ha
@@ -453,8 +451,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // down: Yw = w * (h W_d^T + ha B_d^T)
-  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, tm ? 128 : 32, tm ? 64 : 256) ||
-      !map_packed(&mp.q1, base->down_q, E, H, I / 2, tm ? 128 : 32, tm ? 64 : 256) ||
+  if (!map_packed(&mp.q0, base->down_q, E, H, I / 2, 128, 64) || !map_packed(&mp.q1, base->down_q, E, H, I / 2, 128, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.h), L.rows, I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.ha), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -474,10 +471,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_down", st);
-    if (tm)
-      R4_TRY(launch_gemm_tm(kModeDown, fmt, gp, mp, tm_clusters(kModeDown, fmt, sms, max_tiles, gp.n_rowblk), st));
-    else
-      R4_TRY(launch_gemm(kModeDown, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+    R4_TRY(launch_gemm_tm(kModeDown, fmt, gp, mp, tm_clusters(kModeDown, fmt, sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_out", st);
@@ -625,8 +619,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
 
   // gate/up, transpose-free: dx = dG W_g + dU W_u + gb [A_g; A_u]
-  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, tm ? 64 : 128, 64) ||
-      !map_packed(&mp.q1, base->up_q, E, I, H / 2, tm ? 64 : 128, 64) ||
+  if (!map_packed(&mp.q0, base->gate_q, E, I, H / 2, 64, 64) || !map_packed(&mp.q1, base->up_q, E, I, H / 2, 64, 64) ||
       !map_act_boxes(mp.b, at<uint16_t>(ws, L.dgu), L.rows, 2 * I) || !map_act_boxes(mp.bx, at<uint16_t>(ws, L.gb), L.rows, kLoraPad))
     return RAWINT4_CUDA_ERROR;
   gp.n_rowblk = (H + 255) / 256;
@@ -653,7 +646,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     if (tm)
       R4_TRY(launch_gemm_tm(kModeGateUpT, fmt, gp, mp, tm_clusters(kModeGateUpT, fmt, sms, max_tiles, gp.n_rowblk), st));
     else
-      R4_TRY(launch_gemm(kModeGateUpT, gp, mp, grid_for_tiles(sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_pair(kModeGateUpT, gp, mp, gemm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
   }
   {
     R4_PROF("combine_dx", st);

@@ -4,15 +4,18 @@
 namespace r4 {
 
 // The four dequant-fused grouped GEMMs of the layer. Weight rows (output
-// features) sit on the UMMA M side and up to 256 permuted tokens of one expert
-// on the N side: D[m, n] = sum_k A[m, k] * B[n, k]. Two kernels implement
-// them (both take the same parameters):
-//   gemm.cu       one CTA per SM, 256 weight rows per work item as two
-//                 M = 128 MMAs sharing every B tile (gate/up, down, gate/up^T)
-//   gemm_pair.cu  CTA pairs on SM pairs (tcgen05 cta_group::2), 256 weight
-//                 rows per item as one M = 256 pair MMA; each SM's TMEM holds
-//                 only 128 rows, so 256-token accumulators double-buffer and
-//                 a heavy epilogue overlaps the next item (down^T)
+// features) sit on the UMMA M side and up to kTileRows permuted tokens of one
+// expert on the N side: D[m, n] = sum_k A[m, k] * B[n, k]. Both kernels run on
+// CTA pairs (tcgen05 cta_group::2, M = 256 per pair MMA, each SM's TMEM
+// holding its 128 rows x N, so two accumulators double-buffer and the
+// epilogue of an item overlaps the next item's mainloop); they take the same
+// parameters and differ in where the decoded weights go:
+//   gemm_tm.cu    into tensor memory (UMMA A operand read from TMEM): the
+//                 forward GEMMs (K-major decode), and every mode of an MXFP4
+//                 base
+//   gemm_pair.cu  into shared memory (UMMA A operand from a descriptor): the
+//                 transpose-free backward GEMMs of a RAWINT4 base, whose
+//                 MN-major tiles need no transposition there
 enum GemmMode : int {
   kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
   kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
@@ -23,6 +26,91 @@ enum GemmMode : int {
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
 constexpr int kTmAccCols = 192;    // gemm_tm.cu: columns of one TMEM accumulator = max token-tile rows
 constexpr int kLoraPad = 64;       // width of the LoRA side matrices (>= 2 * rank)
+
+// ------------------------------------------------ shared by the pair kernels
+constexpr uint64_t kDrainNs = 20000000ull;  // bound on the drains of an aborted call (20 ms)
+
+// UMMA N of a token tile: rounded up to 32 so each CTA's half is a whole
+// number of 16-row boxes.
+__device__ __forceinline__ int pair_n(int rows) { return max(32, (rows + 31) & ~31); }
+
+// ------------------------------------------------------------ bounded waits
+// Sets this CTA's abort flag and the peer's (distributed shared memory), so
+// that every role of the pair leaves at its next wait.
+__device__ __forceinline__ void abort_pair(volatile int* abort_flag) {
+  *abort_flag = 1;
+  const uint32_t peer = cluster_addr((const void*)abort_flag, cluster_ctarank() ^ 1u);
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
+}
+
+// A bound below kPollBelowNs is polled with the non-blocking test (a
+// try_wait may suspend until the phase completes, outlasting a short bound).
+constexpr uint64_t kPollBelowNs = 1000000ull;
+
+__device__ __forceinline__ bool wait_lim(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                         uint64_t limit_ns) {
+  const bool poll = limit_ns < kPollBelowNs;
+  if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      raise_status(status, RAWINT4_DEV_TIMEOUT);
+      abort_pair(abort_flag);
+      return false;
+    }
+  }
+}
+// The UMMA issuer's wait: never suspends (a suspended issuer resumes late and
+// the tensor pipe drains meanwhile); the bound is checked every 256 polls.
+__device__ __forceinline__ bool wait_issuer(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                            uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        raise_status(status, RAWINT4_DEV_TIMEOUT);
+        abort_pair(abort_flag);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                          uint64_t limit_ns) {
+  const bool ok = wait_lim(bar, parity, abort_flag, status, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Waits (bounded) for the fills of the last `n` (at most `stages`) stages a
+// producer issued into `full`: a call that aborts must not leave with copies
+// still landing in its shared memory.
+__device__ __forceinline__ void drain_ring(uint64_t* full, Ring r, int issued, int stages) {
+  const int n = issued < stages ? issued : stages;
+  const uint64_t t0 = globaltimer();
+  for (int j = 0; j < n; ++j) {
+    // step back to the previous issue
+    if (r.stage == 0) {
+      r.stage = stages - 1;
+      r.phase ^= 1u;
+    } else {
+      --r.stage;
+    }
+    while (!mbar_try_wait(&full[r.stage], r.phase)) {
+      if (globaltimer() - t0 > kDrainNs) return;
+    }
+  }
+}
+// Copies whose completion is counted on the leader's barrier cannot be
+// observed by the peer: it waits a grace period that any issued copy ends in.
+__device__ __forceinline__ void grace_wait() {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+}
 
 struct GemmParams {
   const int4* tok_tiles;     // {expert, first permuted row, rows, 0}
@@ -59,7 +147,7 @@ struct GemmParams {
   int ld_out;                // row length of out_a / out_b / out_h / in_*
   int inter;
   float limit;
-  unsigned long long wait_ns;  // bound on any pipeline wait (gemm_tm.cu)
+  unsigned long long wait_ns;  // bound on any pipeline wait
 };
 
 struct GemmMaps {
@@ -69,9 +157,9 @@ struct GemmMaps {
   CUtensorMap bx[4];  // B LoRA: 2D fp16 {64, rows}, 128B swizzle, boxes {64, 16 << i}
 };
 
-// One CTA per SM; `grid` CTAs (at most one per SM).
-cudaError_t launch_gemm(int mode, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t stream);
-// CTA pairs (down^T only); `clusters` pairs (at most the number resident at once).
+// CTA pairs with the decoded weights in shared memory (gemm_pair.cu), the
+// transpose-free modes down^T and gate/up^T of a RAWINT4 base; `clusters`
+// pairs (at most the number resident at once).
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
 // CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
 int gemm_pair_max_clusters(int mode);

@@ -21,6 +21,15 @@
 // peer's decoders and epilogue, the peer's TMA bytes counted on the leader's
 // barrier); the MMA's commits arrive on both CTAs' barriers.
 //
+// Hand-off granularity: every synchronisation point in the UMMA issuer's
+// stream costs the tensor pipe a few hundred idle cycles, so the issuer waits
+// once per group of kGroup stages, on one barrier that means "A and B of the
+// whole group are ready": both CTAs' decoders arrive on it after storing the
+// group's A tiles, the leader's first decoder warp only once the group's B
+// tiles have landed. The decoders decode a group into registers before they
+// wait for its A tiles to be free, so only the shared-memory stores sit on
+// the chain from the MMA's release of an A tile to its next fill.
+//
 // The LoRA side product of each projection runs as one extra 64-wide
 // reduction stage in the same accumulators: its A operand is the LoRA tensor
 // of the expert (loaded into registers at the start of the item and stored
@@ -31,15 +40,18 @@
 // the decoders write the same packed bytes into an MN-major A tile, so no
 // transposed or dense copy of any base weight ever exists.
 #include "gemm.cuh"
+#include "route.cuh"
 
 namespace r4 {
 
 namespace pairk {
 
 constexpr int kRowsM = 128;        // weight rows per CTA (256 per CTA pair)
-constexpr int kStagesA = 4;        // decoded FP16 A tiles (16 KB each)
-constexpr int kStagesB = 6;        // TMA-loaded B tiles (up to 128 tokens, 16 KB each)
-constexpr int kStagesP = 8;        // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kStagesA = 4;        // decoded FP16 A tiles (16 KB each): two groups
+constexpr int kGroup = 2;          // stages per hand-off (issuer wait, decoder arrival)
+constexpr int kAGroups = kStagesA / kGroup;
+constexpr int kStagesB = 6;        // TMA-loaded B tiles (this CTA's half of up to kTileRows tokens)
+constexpr int kStagesP = 16;       // TMA-loaded packed int4 tiles (4 KB each)
 constexpr int kStagesS = 16;       // group scales of one stage (512 B each)
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
@@ -47,7 +59,7 @@ constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
 constexpr int kDecThreads = 256;
 
 constexpr int kABytes = kRowsM * kBlockK * 2;  // 16 KB
-constexpr int kBBytes = 128 * kBlockK * 2;     // 16 KB: this CTA's half of <= 256 tokens
+constexpr int kBBytes = (kTileRows / 2) * kBlockK * 2;  // 12 KB: this CTA's half of <= kTileRows tokens
 constexpr int kPBytes = kRowsM * kBlockK / 2;  // 4 KB
 constexpr int kSBytes = 512;                   // 256 bf16 group scales of one stage
 constexpr int kOffA = 0;
@@ -55,7 +67,7 @@ constexpr int kOffB = kOffA + kStagesA * kABytes;
 constexpr int kOffP = kOffB + kStagesB * kBBytes;
 constexpr int kOffS = kOffP + kStagesP * kPBytes;
 constexpr int kOffBar = kOffS + kStagesS * kSBytes;
-constexpr int kNumBars = 2 * kStagesP + 2 * kStagesA + 2 * kStagesB + 2 * kStagesS + 4;
+constexpr int kNumBars = 2 * kStagesP + 2 * kStagesA + 2 * kStagesB + 2 * kStagesS + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
 constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // DOWN_T route partials; gate/up exchange uses the first 2 * 32 * 33
@@ -234,10 +246,6 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, 
   }
 }
 
-// UMMA N of a token tile: rounded up to 32 so each CTA's half is a whole
-// number of 16-row boxes.
-__device__ __forceinline__ int pair_n(int rows) { return max(32, (rows + 31) & ~31); }
-
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
@@ -252,14 +260,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
   uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read it
-  uint64_t* a_full = p_empty + kStagesP;     // leader: both CTAs' decoders stored A
-  uint64_t* a_empty = a_full + kStagesA;     // both: the pair MMA finished reading A
+  uint64_t* a_full = p_empty + kStagesP;     // leader [kAGroups]: the group's A (both CTAs) and B are ready
+  uint64_t* a_empty = a_full + kStagesA;     // both [kAGroups]: the pair MMA finished reading the group's A
   uint64_t* b_full = a_empty + kStagesA;     // leader: both CTAs' B halves landed
   uint64_t* b_empty = b_full + kStagesB;     // both: the pair MMA finished reading B
   uint64_t* s_full = b_empty + kStagesB;     // local: a stage's scales landed
   uint64_t* s_empty = s_full + kStagesS;     // local: this CTA's decoders read them
   uint64_t* acc_full = s_empty + kStagesS;   // both [2]: accumulator complete
   uint64_t* acc_empty = acc_full + 2;        // leader [2]: both epilogues drained it
+  uint64_t* mma_drain = acc_empty + 2;       // leader: all issued MMAs finished (abort path)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* epi = reinterpret_cast<float*>(smem + kOffEpi);
@@ -267,13 +276,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = (int)cluster_ctarank();
+  const uint64_t lim = p.wait_ns;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStagesP; ++i) {
       mbar_init(&p_full[i], 1);
       mbar_init(&p_empty[i], kDecThreads / 32);
     }
-    for (int i = 0; i < kStagesA; ++i) {
+    for (int i = 0; i < kAGroups; ++i) {
       mbar_init(&a_full[i], 2 * kDecThreads / 32);
       mbar_init(&a_empty[i], 1);
     }
@@ -289,6 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 2 * 4);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -320,12 +331,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ packed weight producer
     Ring ring;
+    int issued = 0;
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       const int e = tt.x;
       for (int s = 0; s < n_main; ++s) {
-        if (!wait_all(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
+        if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_p;
         if (lane == 0) {
           uint64_t* bar = &p_full[ring.stage];
           uint8_t* dst = sP + ring.stage * kPBytes;
@@ -349,8 +361,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ring.advance(kStagesP);
+        ++issued;
       }
     }
+    goto done;
+  drain_p:
+    if (lane == 0) drain_ring(p_full, ring, issued, kStagesP);
+    __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------- scale loader
     Ring ring;
@@ -358,21 +375,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       for (int s = 0; s < n_main; ++s) {
-        if (!wait_all(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
+        if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         load_stage_scales<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
         cp_async_arrive_noinc(&s_full[ring.stage]);
         ring.advance(kStagesS);
       }
     }
+  drain_s:
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 2) {
     // ------------------------------------------------------ B tile producer
     Ring ring;
+    int issued = 0;
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int nb = pair_n(tt.z) / 2;  // this CTA's token rows (multiple of 16)
       const int row0 = tt.y + cta * nb;
       for (int s = 0; s <= n_main; ++s) {
-        if (!wait_all_cl(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status)) goto done;
+        if (!wait_warp(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_b;
         if (lane == 0) {
           uint8_t* dst = sB + ring.stage * kBBytes;
           const uint32_t bar = cluster_addr(&b_full[ring.stage], 0);
@@ -391,49 +411,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ring.advance(kStagesB);
+        ++issued;
       }
     }
+    goto done;
+  drain_b:
+    if (lane == 0) {
+      if (cta == 0) drain_ring(b_full, ring, issued, kStagesB);
+      grace_wait();
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------- pair UMMA issuer (leader)
+    // One thread runs the whole issue loop: per group of stages it waits once
+    // (A and B of the group ready), issues the group's UMMAs, frees each B
+    // tile and then the group's A tiles by commits.
     if (cta == 0) {
-      Ring ra, rbr;
-      int it = 0;
-      const int ksteps_x = kext_steps<MODE>(p.rpad);
-      for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
-        const int4 tt = p.tok_tiles[tile / n_rowblk];
-        const int n_mma = pair_n(tt.z);
-        const uint32_t idesc = make_idesc_f16((uint32_t)n_mma, kAMnMajor<MODE>, false, 256);
-        const int ab = it & 1;
-        if (!wait_all_cl(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status)) goto done;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(ab * 256);
-        for (int s = 0; s <= n_main; ++s) {
-          if (!wait_all_cl(&a_full[ra.stage], ra.phase, abort_flag, status)) goto done;
-          if (!wait_all_cl(&b_full[rbr.stage], rbr.phase, abort_flag, status)) goto done;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_base = smem_u32(sA + ra.stage * kABytes);
-            const uint32_t b_base = smem_u32(sB + rbr.stage * kBBytes);
-            const int ksteps = (s < n_main) ? (kBlockK / 16) : ksteps_x;
-            for (int kk = 0; kk < ksteps; ++kk) {
-              uint64_t adesc;
-              if constexpr (kAMnMajor<MODE>)
-                adesc = make_sdesc_sw128(a_base + kk * 2048, 8192, 1024);
-              else
-                adesc = make_sdesc_sw128(a_base + kk * 32, 16, 1024);
-              const uint64_t bdesc = make_sdesc_sw128(b_base + kk * 32, 16, 1024);
-              umma_f16_pair(d_tmem, adesc, bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit_pair(&a_empty[ra.stage], kPairMask);
-            umma_commit_pair(&b_empty[rbr.stage], kPairMask);
+      if (lane == 0) {
+        Ring rg, rbr;
+        int it = 0;
+        bool aborted = false;
+        const int ksteps_x = kext_steps<MODE>(p.rpad);
+        // descriptors of A tile 0 and B tile 0; a tile adds its bytes, a
+        // 16-wide reduction step 32 bytes (K-major) or 2048 bytes (MN-major
+        // A: 16 rows of two 8 KB halves), all in 16-byte units
+        const uint64_t adesc0 = kAMnMajor<MODE> ? make_sdesc_sw128(smem_u32(sA), 8192, 1024)
+                                                : make_sdesc_sw128(smem_u32(sA), 16, 1024);
+        const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(sB), 16, 1024);
+        constexpr uint64_t kAStep = kAMnMajor<MODE> ? 2048 / 16 : 32 / 16;
+        for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
+          const int4 tt = p.tok_tiles[tile / n_rowblk];
+          const uint32_t idesc = make_idesc_f16((uint32_t)pair_n(tt.z), kAMnMajor<MODE>, false, 256);
+          const int ab = it & 1;
+          if (!wait_issuer(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status, lim)) {
+            aborted = true;
+            goto mma_out;
           }
-          __syncwarp();
-          ra.advance(kStagesA);
-          rbr.advance(kStagesB);
+          tc_fence_after();
+          {
+            const uint32_t d_tmem = tmem + (uint32_t)(ab * 256);
+            uint32_t acc = 0u;  // the item's first UMMA overwrites the accumulator
+            // main stages in groups of kGroup, then the LoRA stage alone
+            for (int s = 0; s <= n_main; s += kGroup) {
+              const bool lora = s == n_main;
+              const int nb = lora ? 1 : min(kGroup, n_main - s);
+              if (!wait_issuer(&a_full[rg.stage], rg.phase, abort_flag, status, lim)) {
+                aborted = true;
+                goto mma_out;
+              }
+              tc_fence_after();
+              for (int b = 0; b < nb; ++b) {
+                const uint64_t ad = adesc0 + (uint64_t)(((kGroup * rg.stage + b) * kABytes) >> 4);
+                const uint64_t bd = bdesc0 + (uint64_t)((rbr.stage * kBBytes) >> 4);
+                if (!lora) {
+#pragma unroll
+                  for (int kk = 0; kk < kBlockK / 16; ++kk) {
+                    umma_f16_pair(d_tmem, ad + kAStep * kk, bd + (uint64_t)(2 * kk), idesc, acc);
+                    acc = 1u;
+                  }
+                } else {
+                  for (int kk = 0; kk < ksteps_x; ++kk) {
+                    umma_f16_pair(d_tmem, ad + kAStep * kk, bd + (uint64_t)(2 * kk), idesc, acc);
+                    acc = 1u;
+                  }
+                }
+                umma_commit_pair(&b_empty[rbr.stage], kPairMask);
+                rbr.advance(kStagesB);
+              }
+              umma_commit_pair(&a_empty[rg.stage], kPairMask);
+              rg.advance(kAGroups);
+              if (lora) break;
+              if (s + kGroup > n_main) s = n_main - kGroup;  // an odd last main stage was its own group
+            }
+          }
+          umma_commit_pair(&acc_full[ab], kPairMask);
         }
-        if (lane == 0) umma_commit_pair(&acc_full[ab], kPairMask);
-        __syncwarp();
+      mma_out:
+        if (aborted) {
+          // every MMA this thread issued has finished before the pair leaves
+          umma_commit_pair(mma_drain, 1);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(mma_drain, 0u)) {
+            if (globaltimer() - t0 > kDrainNs) break;
+          }
+        }
       }
+      __syncwarp();
     }
   } else if (warp >= kEpiWarp0 && warp < kDecWarp0) {
     // --------------------------------------------------------------- epilogue
@@ -449,7 +512,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int n_rows = tt.z;
       const int p0 = tt.y;
       const int ab = it & 1;
-      if (!wait_all_cl(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status)) goto done;
+      // the four epilogue warps leave together or not at all: a warp that
+      // went on alone would wait forever at the exchange barriers
+      const bool ok = wait_warp(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status, lim);
+      if (!named_bar_and(3, 128, ok)) goto done;
       tc_fence_after();
       const uint32_t d_tmem = tmem + lane_base + (uint32_t)(ab * 256);
       for (int c0 = 0; c0 < n_rows; c0 += 32) {
@@ -496,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 32; ++c) {
               const int n = c0 + c;
               const float w = __shfl_sync(0xffffffffu, wl, c);
-              if (n < n_rows) {
+              if (n < n_rows && fc + m < p.feat) {
                 float a = __uint_as_float(v[c]);
                 if constexpr (MODE == kModeDown) a *= w;
                 p.out_a[(int64_t)(p0 + n) * p.ld_out + fc + m] = a;
@@ -582,7 +648,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= kDecWarp0) {
     // --------------------------------------------------------------- decoders
     const int dt = threadIdx.x - kDecWarp0 * 32;
-    Ring ra, rp, rs;
+    // the leader's first decoder warp also waits for each group's B tiles
+    const bool b_watch = cta == 0 && warp == kDecWarp0;
+    Ring rg, rp, rs, rbd;
     const uint32_t s_off = scale_off<MODE>(dt);
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
@@ -590,70 +658,80 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int e = tt.x;
       uint32_t lora_w[16];
       lora_values<MODE>(p, e, fc, dt, lora_w);
-      // Main stages two at a time (n_main is even): the two decodes are
-      // independent, so each warp's dependent chain of waits, shared loads,
-      // decode arithmetic, stores, proxy fence and arrivals is paid once per
-      // pair of stages.
-      for (int s = 0; s < n_main; s += 2) {
-        Ring ra1 = ra, rs1 = rs, rp1 = rp;
-        ra1.advance(kStagesA);
-        rs1.advance(kStagesS);
-        rp1.advance(kStagesP);
-        if (!wait_all_cl(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
-        if (!wait_all_cl(&a_empty[ra1.stage], ra1.phase ^ 1u, abort_flag, status)) goto done;
-        if (!wait_all(&s_full[rs.stage], rs.phase, abort_flag, status)) goto done;
-        if (!wait_all(&s_full[rs1.stage], rs1.phase, abort_flag, status)) goto done;
-        const uint16_t sc0 = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
-        const uint16_t sc1 = *reinterpret_cast<const uint16_t*>(sS + rs1.stage * kSBytes + s_off);
-        if (!wait_all(&p_full[rp.stage], rp.phase, abort_flag, status)) goto done;
-        if (!wait_all(&p_full[rp1.stage], rp1.phase, abort_flag, status)) goto done;
-        const uint4 q0 = packed_group<MODE>(sP + rp.stage * kPBytes, dt);
-        const uint4 q1 = packed_group<MODE>(sP + rp1.stage * kPBytes, dt);
-        uint32_t w0[16], w1[16];
-        decode_group32(q0, bf16_scale_to_h2(sc0), w0);
-        decode_group32(q1, bf16_scale_to_h2(sc1), w1);
-        uint8_t* A0 = sA + ra.stage * kABytes;
-        uint8_t* A1 = sA + ra1.stage * kABytes;
+      for (int s = 0; s < n_main; s += kGroup) {
+        const int nb = min(kGroup, n_main - s);
+        // decode the group into registers (needs only its packed and scale
+        // stages), then wait for its A tiles to be free and store
+        Ring rp_[kGroup], rs_[kGroup];
+        uint32_t w[kGroup][16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<uint4*>(A0 + a_chunk_off<MODE>(dt, j)) =
-              make_uint4(w0[4 * j], w0[4 * j + 1], w0[4 * j + 2], w0[4 * j + 3]);
-          *reinterpret_cast<uint4*>(A1 + a_chunk_off<MODE>(dt, j)) =
-              make_uint4(w1[4 * j], w1[4 * j + 1], w1[4 * j + 2], w1[4 * j + 3]);
+        for (int b = 0; b < kGroup; ++b) {
+          rp_[b] = rp;
+          rs_[b] = rs;
+          if (b < nb) {
+            if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
+            if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
+            const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
+            const uint4 q4 = packed_group<MODE>(sP + rp.stage * kPBytes, dt);
+            decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
+            rp.advance(kStagesP);
+            rs.advance(kStagesS);
+          }
         }
-        fence_proxy_async_smem();
+        // The packed and scale stages are released once every lane has used
+        // the values it loaded from them: the empty asm makes the decoded
+        // words (which depend on every loaded byte and on the scale) inputs,
+        // so the loads have returned before the release. A release right after
+        // the loads were issued could let the refill of the stage land under
+        // loads still in flight.
+#pragma unroll
+        for (int b = 0; b < kGroup; ++b)
+          if (b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
         __syncwarp();
         if (lane == 0) {
-          // The packed and scale stages are released only here, after the
-          // decoded values that consume their bytes were stored: an arrive
-          // issued right after the shared loads can overtake them, and the
-          // refill of the stage then lands under loads still in flight.
-          mbar_arrive(&p_empty[rp.stage]);
-          mbar_arrive(&p_empty[rp1.stage]);
-          mbar_arrive(&s_empty[rs.stage]);
-          mbar_arrive(&s_empty[rs1.stage]);
-          mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
-          mbar_arrive_cluster(cluster_addr(&a_full[ra1.stage], 0));
+          for (int b = 0; b < nb; ++b) {
+            mbar_arrive(&p_empty[rp_[b].stage]);
+            mbar_arrive(&s_empty[rs_[b].stage]);
+          }
         }
-        ra1.advance(kStagesA);
-        rs1.advance(kStagesS);
-        rp1.advance(kStagesP);
-        ra = ra1;
-        rs = rs1;
-        rp = rp1;
+        if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
+#pragma unroll
+        for (int b = 0; b < kGroup; ++b) {
+          if (b < nb) {
+            uint8_t* A = sA + (kGroup * rg.stage + b) * kABytes;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
+                  make_uint4(w[b][4 * j], w[b][4 * j + 1], w[b][4 * j + 2], w[b][4 * j + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        if (b_watch) {
+          for (int b = 0; b < nb; ++b) {
+            if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+            rbd.advance(kStagesB);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
+        rg.advance(kAGroups);
       }
-      // the LoRA reduction stage
+      // the LoRA reduction stage, a group of its own
       {
-        if (!wait_all_cl(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status)) goto done;
-        uint8_t* A = sA + ra.stage * kABytes;
+        if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
+        uint8_t* A = sA + (kGroup * rg.stage) * kABytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
               make_uint4(lora_w[4 * j], lora_w[4 * j + 1], lora_w[4 * j + 2], lora_w[4 * j + 3]);
         fence_proxy_async_smem();
+        if (b_watch) {
+          if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+          rbd.advance(kStagesB);
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
-        ra.advance(kStagesA);
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
+        rg.advance(kAGroups);
       }
     }
   }
@@ -706,20 +784,19 @@ int max_clusters_mode() {
 
 }  // namespace pairk
 
-// The library runs only the down^T GEMM on CTA pairs (its epilogue is the
-// one that needs double-buffered 256-token accumulators); the kernel itself
-// is written for every mode.
-// The library runs only the down^T GEMM on CTA pairs (its epilogue is the
-// one that needs double-buffered 256-token accumulators); the kernel itself
-// is written for every mode.
+// The library runs the two transpose-free backward GEMMs (MN-major decoded
+// A tiles in shared memory) on this kernel; the kernel itself is written for
+// every mode.
 cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
-  if (mode != kModeDownT) return cudaErrorInvalidValue;
-  return pairk::launch_mode<kModeDownT>(p, maps, clusters, stream);
+  if (mode == kModeDownT) return pairk::launch_mode<kModeDownT>(p, maps, clusters, stream);
+  if (mode == kModeGateUpT) return pairk::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
+  return cudaErrorInvalidValue;
 }
 
 int gemm_pair_max_clusters(int mode) {
-  if (mode != kModeDownT) return 0;
-  return pairk::max_clusters_mode<kModeDownT>();
+  if (mode == kModeDownT) return pairk::max_clusters_mode<kModeDownT>();
+  if (mode == kModeGateUpT) return pairk::max_clusters_mode<kModeGateUpT>();
+  return 0;
 }
 
 }  // namespace r4

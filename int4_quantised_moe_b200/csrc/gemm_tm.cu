@@ -17,6 +17,14 @@
 //   [2 kAccCols, + 32 kAStages)     A stages: 128 weight rows x 64 reduction fp16
 // so a token tile has at most kAccCols rows (the tile list is cut to that).
 //
+// Hand-off granularity: every synchronisation point in the UMMA issuer's
+// stream (a barrier wait, also one delegated to another warp) leaves the
+// tensor pipe idle for a few hundred cycles, so the issuer waits once per
+// group of kGroup stages (4 kGroup UMMAs) on one barrier that means "A and B
+// of the whole group are ready": the decoders arrive on it after storing the
+// group's A stages, and the leader's first decoder warp arrives only once the
+// group's B stages have landed. The A stages form kAStages / kGroup groups.
+//
 // Warp roles, in each CTA:
 //   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP)
 //   warp 1      leader CTA: pair-wide UMMA issuer; both CTAs: TMEM allocation
@@ -72,11 +80,9 @@ constexpr int kThreads = 512;                     // 16 warps
 constexpr int kEpiWarp0 = 4;                      // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                      // warps 8..15: decoders
 constexpr int kDecWarps = 8;
-#ifndef R4_DEC_BATCH
-#define R4_DEC_BATCH 2
-#endif
-constexpr int kDecBatch = R4_DEC_BATCH;           // main stages a decoder warp handles per hand-off
-static_assert(kAStages >= 2 * kDecBatch, "the MMA consumes one batch while the next is decoded");
+constexpr int kGroup = 2;                         // stages per hand-off (issuer wait, decoder arrival)
+constexpr int kAGroups = kAStages / kGroup;       // groups of A stages in tensor memory
+static_assert(kAGroups >= 2, "the MMA consumes one group while the next is decoded");
 
 constexpr int kBBytes = (kTmAccCols / 2) * kBlockK * 2;  // this CTA's half of <= kTmAccCols tokens
 template <int MODE>
@@ -97,7 +103,6 @@ constexpr int kSmemBytes = kOffScaleTab + kTabBytes + 1024;  // + alignment slac
 static_assert(kBBytes % 1024 == 0 && kPRing % kPSlotBytes == 0, "1024-byte aligned stages");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint16_t kPairMask = 3;
-constexpr uint64_t kDrainNs = 20000000ull;       // bound on the drains of an aborted call (20 ms)
 
 template <int MODE>
 constexpr bool kAMnMajor = (MODE == kModeDownT || MODE == kModeGateUpT);
@@ -129,70 +134,6 @@ __device__ __forceinline__ int k_rotation(int rb, int n_rowblk, int n_slots) {
 __device__ __forceinline__ int rotated(int s, int rot, int n_main) {
   const int k = s + rot;
   return k >= n_main ? k - n_main : k;
-}
-
-// UMMA N of a token tile: rounded up to 32 so each CTA's half is a whole
-// number of 16-row boxes.
-__device__ __forceinline__ int pair_n(int rows) { return max(32, (rows + 31) & ~31); }
-
-// ------------------------------------------------------------ bounded waits
-// Sets this CTA's abort flag and the peer's (distributed shared memory), so
-// that every role of the pair leaves at its next wait.
-__device__ __forceinline__ void abort_pair(volatile int* abort_flag) {
-  *abort_flag = 1;
-  const uint32_t peer = cluster_addr((const void*)abort_flag, cluster_ctarank() ^ 1u);
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
-}
-
-// A bound below kPollBelowNs is polled with the non-blocking test (a
-// try_wait may suspend until the phase completes, outlasting a short bound).
-constexpr uint64_t kPollBelowNs = 1000000ull;
-
-__device__ __forceinline__ bool wait_lim(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
-                                         uint64_t limit_ns) {
-  const bool poll = limit_ns < kPollBelowNs;
-  if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (;;) {
-    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > limit_ns) {
-      raise_status(status, RAWINT4_DEV_TIMEOUT);
-      abort_pair(abort_flag);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
-                                          uint64_t limit_ns) {
-  const bool ok = wait_lim(bar, parity, abort_flag, status, limit_ns);
-  return __all_sync(0xffffffffu, ok);
-}
-
-// Waits (bounded) for the fills of the last `n` (at most `stages`) stages a
-// producer issued into `full`: a call that aborts must not leave with copies
-// still landing in its shared memory.
-__device__ __forceinline__ void drain_ring(uint64_t* full, Ring r, int issued, int stages) {
-  const int n = issued < stages ? issued : stages;
-  const uint64_t t0 = globaltimer();
-  for (int j = 0; j < n; ++j) {
-    // step back to the previous issue
-    if (r.stage == 0) {
-      r.stage = stages - 1;
-      r.phase ^= 1u;
-    } else {
-      --r.stage;
-    }
-    while (!mbar_try_wait(&full[r.stage], r.phase)) {
-      if (globaltimer() - t0 > kDrainNs) return;
-    }
-  }
-}
-// Copies whose completion is counted on the leader's barrier cannot be
-// observed by the peer: it waits a grace period that any issued copy ends in.
-__device__ __forceinline__ void grace_wait() {
-  const uint64_t t0 = globaltimer();
-  while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
 }
 
 // ----------------------------------------------------------- K-major decode
@@ -471,8 +412,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
   uint64_t* p_empty = p_full + kMaxStagesP;  // local: this CTA's decoders read it
-  uint64_t* a_full = p_empty + kMaxStagesP;  // leader: both CTAs' decoders stored A
-  uint64_t* a_empty = a_full + kAStages;     // both: the pair MMA finished reading A
+  uint64_t* a_full = p_empty + kMaxStagesP;  // leader [kAGroups]: the group's A (both CTAs) and B are ready
+  uint64_t* a_empty = a_full + kAStages;     // both [kAGroups]: the pair MMA finished reading the group's A
   uint64_t* b_full = a_empty + kAStages;     // leader: both CTAs' B halves landed
   uint64_t* b_empty = b_full + kStagesB;     // both: the pair MMA finished reading B
   uint64_t* s_full = b_empty + kStagesB;     // local: a stage's scales landed
@@ -494,7 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 1);
       mbar_init(&p_empty[i], kDecWarps);
     }
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kAGroups; ++i) {
       mbar_init(&a_full[i], 2 * kDecWarps);
       mbar_init(&a_empty[i], 1);
     }
@@ -655,48 +596,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------- pair UMMA issuer (leader)
+    // One thread runs the whole issue loop: per group of stages it waits once
+    // (A and B of the group ready), issues the group's UMMAs, frees each B
+    // stage and then the group's A stages by commits.
     if (cta == 0) {
-      Ring ra, rbr;
-      int it = 0;
-      const int ksteps_x = kext_steps<MODE>(p.rpad);
-      for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
-        const int4 tt = p.tok_tiles[tile / n_rowblk];
-        const int n_mma = pair_n(tt.z);
-        const uint32_t idesc = make_idesc_f16((uint32_t)n_mma, false, false, 256);
-        const int ab = it & 1;
-        if (!wait_warp(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status, lim)) goto drain_mma;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(ab * kTmAccCols);
-        for (int s = 0; s <= n_main; ++s) {
-          if (!wait_warp(&a_full[ra.stage], ra.phase, abort_flag, status, lim)) goto drain_mma;
-          if (!wait_warp(&b_full[rbr.stage], rbr.phase, abort_flag, status, lim)) goto drain_mma;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_tm = tmem + kACol0 + (uint32_t)(32 * ra.stage);
-            const uint32_t b_base = smem_u32(sB + rbr.stage * kBBytes);
-            const int ksteps = (s < n_main) ? (kBlockK / 16) : ksteps_x;
-            for (int kk = 0; kk < ksteps; ++kk) {
-              const uint64_t bdesc = make_sdesc_sw128(b_base + kk * 32, 16, 1024);
-              umma_f16_pair_ts(d_tmem, a_tm + (uint32_t)(8 * kk), bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit_pair(&a_empty[ra.stage], kPairMask);
-            umma_commit_pair(&b_empty[rbr.stage], kPairMask);
-          }
-          __syncwarp();
-          ra.advance(kAStages);
-          rbr.advance(kStagesB);
-        }
-        if (lane == 0) umma_commit_pair(&acc_full[ab], kPairMask);
-        __syncwarp();
-      }
-      goto done;
-    drain_mma:
-      // every MMA this thread issued has finished before the pair leaves
       if (lane == 0) {
-        umma_commit_pair(mma_drain, 1);
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(mma_drain, 0u)) {
-          if (globaltimer() - t0 > kDrainNs) break;
+        Ring rg, rbr;
+        int it = 0;
+        bool aborted = false;
+        const int ksteps_x = kext_steps<MODE>(p.rpad);
+        // shared-memory descriptor of B stage 0; stage s adds s kBBytes, a
+        // 16-wide reduction step adds 32 bytes (both in 16-byte units)
+        const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(sB), 16, 1024);
+        const uint32_t a_col0 = tmem + kACol0;
+        for (int tile = tile0; tile < n_tiles; tile += tile_step, ++it) {
+          const int4 tt = p.tok_tiles[tile / n_rowblk];
+          const uint32_t idesc = make_idesc_f16((uint32_t)pair_n(tt.z), false, false, 256);
+          const int ab = it & 1;
+          const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
+          if (!wait_issuer(&acc_empty[ab], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, status, lim)) {
+            aborted = true;
+            goto mma_out;
+          }
+          tc_fence_after();
+          {
+            const uint32_t d_tmem = tmem + (uint32_t)(ab * kTmAccCols);
+            uint32_t acc = 0u;  // the item's first UMMA overwrites the accumulator
+            // the item's stages: slot-rotated main stages in groups within each
+            // slot, then the LoRA stage as a group of its own
+            for (int j0 = 0; j0 <= n_slots; ++j0) {
+              const bool lora = j0 == n_slots;
+              const int nsub = lora ? 1 : min(PS, n_main - PS * rotated(j0, rot, n_slots));
+              for (int u = 0; u < nsub; u += kGroup) {
+                const int nb = min(kGroup, nsub - u);
+                if (!wait_issuer(&a_full[rg.stage], rg.phase, abort_flag, status, lim)) {
+                  aborted = true;
+                  goto mma_out;
+                }
+                tc_fence_after();
+                for (int b = 0; b < nb; ++b) {
+                  const uint32_t a_tm = a_col0 + (uint32_t)(64 * rg.stage + 32 * b);
+                  const uint64_t bd = bdesc0 + (uint64_t)((rbr.stage * kBBytes) >> 4);
+                  if (!lora) {
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; ++kk) {
+                      umma_f16_pair_ts(d_tmem, a_tm + (uint32_t)(8 * kk), bd + (uint64_t)(2 * kk), idesc, acc);
+                      acc = 1u;
+                    }
+                  } else {
+                    for (int kk = 0; kk < ksteps_x; ++kk) {
+                      umma_f16_pair_ts(d_tmem, a_tm + (uint32_t)(8 * kk), bd + (uint64_t)(2 * kk), idesc, acc);
+                      acc = 1u;
+                    }
+                  }
+                  umma_commit_pair(&b_empty[rbr.stage], kPairMask);
+                  rbr.advance(kStagesB);
+                }
+                umma_commit_pair(&a_empty[rg.stage], kPairMask);
+                rg.advance(kAGroups);
+              }
+            }
+          }
+          umma_commit_pair(&acc_full[ab], kPairMask);
+        }
+      mma_out:
+        if (aborted) {
+          // every MMA this thread issued has finished before the pair leaves
+          umma_commit_pair(mma_drain, 1);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(mma_drain, 0u)) {
+            if (globaltimer() - t0 > kDrainNs) break;
+          }
         }
       }
       __syncwarp();
@@ -873,7 +843,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     };
     uint32_t* tab = reinterpret_cast<uint32_t*>(smem + kOffScaleTab) + 32 * (warp - kDecWarp0);
-    Ring ra, rp, rs;
+    Ring rg, rp, rs, rbd;
+    // the leader's first decoder warp also waits for each group's B stages
+    const bool b_watch = cta == 0 && warp == kDecWarp0;
     // Decodes sub-stage u of packed slot rp / scale slot rs into w; table `tb`
     // holds the MN-major scale pairs.
     auto decode_stage = [&](const Ring& rs_, const Ring& rp_, int u, uint32_t* tb, uint32_t (&w)[16]) {
@@ -931,37 +903,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nsub = min(PS, n_main - PS * j);
         if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
         if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
-        // The slot's stages kDecBatch at a time: the decodes of a batch are
-        // independent, so the chain of waits, tensor-memory store completion,
-        // fence and arrivals is paid once per batch; the A ring
-        // (kAStages >= 2 kDecBatch) lets the MMA consume one batch while the
-        // next one is decoded.
-        for (int u = 0; u < nsub; u += kDecBatch) {
-          const int nb = min(kDecBatch, nsub - u);
-          Ring r_a[kDecBatch];
+        // the slot's stages a group at a time: decoded into registers first
+        // (that needs only the packed and scale slots), then one wait for the
+        // group's A stages, the tensor-memory stores, one store completion,
+        // fence and arrival: only the stores sit on the chain from the MMA's
+        // release of the A stages to their next fill
+        for (int u = 0; u < nsub; u += kGroup) {
+          const int nb = min(kGroup, nsub - u);
+          uint32_t w[kGroup][16];
 #pragma unroll
-          for (int b = 0; b < kDecBatch; ++b) {
-            r_a[b] = ra;
-            if (b < nb) ra.advance(kAStages);
-          }
-#pragma unroll
-          for (int b = 0; b < kDecBatch; ++b)
-            if (b < nb && !wait_warp(&a_empty[r_a[b].stage], r_a[b].phase ^ 1u, abort_flag, status, lim)) goto done;
-          uint32_t w[kDecBatch][16];
-#pragma unroll
-          for (int b = 0; b < kDecBatch; ++b)
+          for (int b = 0; b < kGroup; ++b)
             if (b < nb) decode_stage(rs, rp, u + b, tab + 16 * b, w[b]);
+          if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
 #pragma unroll
-          for (int b = 0; b < kDecBatch; ++b)
-            if (b < nb) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * r_a[b].stage + 16 * g), w[b]);
+          for (int b = 0; b < kGroup; ++b)
+            if (b < nb) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 32 * b + 16 * g), w[b]);
           tmem_wait_st();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-#pragma unroll
-            for (int b = 0; b < kDecBatch; ++b)
-              if (b < nb) mbar_arrive_cluster(cluster_addr(&a_full[r_a[b].stage], 0));
+          if (b_watch) {
+            for (int b = 0; b < nb; ++b) {
+              if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+              rbd.advance(kStagesB);
+            }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
+          rg.advance(kAGroups);
         }
         // the packed and scale slots are released after the values that
         // consume their bytes were stored
@@ -972,14 +939,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         rp.advance(kStagesP<MODE>);
         rs.advance(kStagesS);
       }
-      // the LoRA stage
-      if (!wait_warp(&a_empty[ra.stage], ra.phase ^ 1u, abort_flag, status, lim)) goto done;
-      tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * ra.stage + 16 * g), lora_w);
+      // the LoRA stage, a group of its own
+      if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
+      tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 16 * g), lora_w);
       tmem_wait_st();
       tc_fence_before();
+      if (b_watch) {
+        if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+        rbd.advance(kStagesB);
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[ra.stage], 0));
-      ra.advance(kAStages);
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
+      rg.advance(kAGroups);
     }
   }
 
