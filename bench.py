@@ -382,52 +382,88 @@ def main():
     roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, args.config)
     step_roofline["experts_hit"] = hit
 
-    # ---- end to end through the public API from pinned host buffers
+    # ---- end to end through the public API from pinned host buffers. Steps
+    # are pipelined as a host loop would run them: the inputs of step i+1 go
+    # up and the outputs of step i-1 come down on two copy streams while step
+    # i's kernels run; device inputs and outputs are double-buffered, and
+    # events order each buffer's upload, use and download. Every step still
+    # copies its whole input from pinned host memory and its whole result
+    # back, all inside the timed region (from the first upload to the last
+    # download).
     e2e = None
     if not args.no_e2e:
         h_x = wl.x.cpu().pin_memory()
         h_ids = wl.expert_ids.cpu().pin_memory()
         h_w = wl.route_weights.cpu().pin_memory()
         h_g = wl.grad_out.cpu().pin_memory()
-        h_out = torch.empty_like(h_x).pin_memory()
-        h_gin = torch.empty_like(h_x).pin_memory()
-        h_gr = torch.empty(groute.shape, dtype=torch.float32).pin_memory()
-        d_x, d_ids, d_w, d_g = torch.empty_like(wl.x), torch.empty_like(wl.expert_ids), torch.empty_like(
-            wl.route_weights), torch.empty_like(wl.grad_out)
+        h_out = [torch.empty_like(h_x).pin_memory() for _ in range(2)]
+        h_gin = [torch.empty_like(h_x).pin_memory() for _ in range(2)]
+        h_gr = [torch.empty(groute.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+        d_in = [(torch.empty_like(wl.x), torch.empty_like(wl.expert_ids), torch.empty_like(wl.route_weights),
+                 torch.empty_like(wl.grad_out)) for _ in range(2)]
+        d_res = [(torch.empty_like(out), torch.empty_like(gin), torch.empty_like(groute)) for _ in range(2)]
+        up = torch.cuda.Stream(device=dev)
+        down = torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        uploaded = [ev(), ev()]    # inputs of buffer b on the device
+        computed = [ev(), ev()]    # kernels of buffer b done (inputs free, results ready)
+        downloaded = [ev(), ev()]  # results of buffer b on the host (result buffers free)
+        used = [False, False]
 
-        def e2e_step():
-            d_x.copy_(h_x, non_blocking=True)
-            d_ids.copy_(h_ids, non_blocking=True)
-            d_w.copy_(h_w, non_blocking=True)
+        def e2e_step(i):
+            b = i & 1
+            d_x, d_ids, d_w, d_g = d_in[b]
+            r_out, r_gin, r_gr = d_res[b]
+            with torch.cuda.stream(up):
+                if used[b]:
+                    up.wait_event(computed[b])
+                d_x.copy_(h_x, non_blocking=True)
+                d_ids.copy_(h_ids, non_blocking=True)
+                d_w.copy_(h_w, non_blocking=True)
+                if not infer:
+                    d_g.copy_(h_g, non_blocking=True)
+                uploaded[b].record(up)
+            stream.wait_event(uploaded[b])
+            if used[b]:
+                stream.wait_event(downloaded[b])
             if infer:
-                layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=False, use_lora=False)
-                h_out.copy_(out, non_blocking=True)
-                return
-            d_g.copy_(h_g, non_blocking=True)
-            layer.forward(d_ids, d_w, d_x, out=out, save_for_backward=True)
-            layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=gin, grad_route=groute)
-            if pg is not None:
-                dp.reduce_window_grads(grads)  # one-step window: reduce at its end
-            h_out.copy_(out, non_blocking=True)
-            h_gin.copy_(gin, non_blocking=True)
-            h_gr.copy_(groute, non_blocking=True)
+                layer.forward(d_ids, d_w, d_x, out=r_out, save_for_backward=False, use_lora=False)
+            else:
+                layer.forward(d_ids, d_w, d_x, out=r_out, save_for_backward=True)
+                layer.backward(d_g, grads, accumulate=False, grad_scale=1.0, grad_in=r_gin, grad_route=r_gr)
+                if pg is not None:
+                    dp.reduce_window_grads(grads)  # one-step window: reduce at its end
+            computed[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                h_out[b].copy_(r_out, non_blocking=True)
+                if not infer:
+                    h_gin[b].copy_(r_gin, non_blocking=True)
+                    h_gr[b].copy_(r_gr, non_blocking=True)
+                downloaded[b].record(down)
+            used[b] = True
 
-        e2e_step()
+        e2e_step(0)
+        e2e_step(1)
         torch.cuda.synchronize(dev)
         barrier()
         e_start = torch.cuda.Event(enable_timing=True)
         e_end = torch.cuda.Event(enable_timing=True)
         e_start.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        up.wait_event(e_start)
+        for i in range(args.steps):
+            e2e_step(i)
+        for b in range(2):
+            stream.wait_event(downloaded[b])
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps
         h2d = sum(t.numel() * t.element_size() for t in ((h_x, h_ids, h_w) if infer else (h_x, h_ids, h_w, h_g)))
-        d2h = sum(t.numel() * t.element_size() for t in ((h_out,) if infer else (h_out, h_gin, h_gr)))
+        d2h = sum(t.numel() * t.element_size() for t in ((h_out[0],) if infer else (h_out[0], h_gin[0], h_gr[0])))
         e2e = {"value": round(cfg.qlen * cfg.top_k * world / (e_ms / 1e3), 1), "unit": UNIT,
-               "ms_per_step": round(e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": round(e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelined": "uploads of step i+1 and downloads of step i-1 overlap step i on two copy streams"}
 
     st = layer.status()
     cpu = None
