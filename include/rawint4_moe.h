@@ -31,7 +31,16 @@
  * FP16 operands and FP32 accumulation. (code - 8) * scale has at most 12
  * significant bits, so every decoded weight is exact in FP16 as long as
  * |scale| lies in [2^-14, 8188]; activations are rounded once to FP16
- * (relative error 2^-11) where they become MMA operands.
+ * (relative error 2^-11) where they become MMA operands. An activation
+ * beyond the FP16 range raises RAWINT4_DEV_FP16_OVERFLOW. The backward
+ * scales grad_out by an exact power of two chosen from its largest
+ * magnitude before its FP16 operands are formed and undoes it in FP32, so
+ * small gradients (1e-9 and below) keep their precision.
+ * The LoRA tensors are copied to FP16 per call: exact for magnitudes in
+ * [2^-14, 65504] (a bf16 value has 8 significant bits, FP16 holds 11),
+ * rounded to FP16 subnormals below 2^-14 (absolute error at most 2^-25) and
+ * to infinity above 65504 (no status bit: LoRA factors of that size are
+ * outside any training regime).
  */
 #ifndef RAWINT4_MOE_H
 #define RAWINT4_MOE_H
