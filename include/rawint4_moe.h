@@ -96,7 +96,8 @@ enum {
  * Limits: H % 64 == 0, I % 64 == 0 (the kernels reduce in stages of 64 and
  * mask a partial last block of output features; MXFP4: H % 128 == 0 and
  * I % 128 == 0, its scale bytes are fetched four at a time),
- * 1 <= rank <= 32, 1 <= top_k <= experts. */
+ * 1 <= rank <= 64 (the gate and up rank blocks, each padded to a multiple
+ * of 16, take one or two 64-wide reduction stages), 1 <= top_k <= experts. */
 enum {
   RAWINT4_FORMAT_RAWINT4 = 0, /* codes 0..15 -> (code - 8) * bf16 scale */
   RAWINT4_FORMAT_MXFP4 = 1    /* E2M1 codes * 2^(e - 127), e a UE8M0 scale byte */

@@ -83,7 +83,7 @@ bool cfg_ok(const rawint4_moe_cfg* c) {
   if (c->top_k < 1 || c->top_k > c->experts) return false;
   if (c->hidden < 64 || c->hidden % 64 != 0) return false;
   if (c->inter < 64 || c->inter % 64 != 0) return false;
-  if (c->rank < 1 || c->rank > 32) return false;
+  if (c->rank < 1 || c->rank > 64) return false;
   if (!std::isfinite(c->alpha)) return false;
   if (!std::isfinite(c->swiglu_limit) || c->swiglu_limit < 0.f) return false;
   if (c->max_tokens < 1) return false;
@@ -195,11 +195,16 @@ bool map_act_boxes(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t c
 }
 
 // fp16 per-expert matrices [E, rows, cols]; box {64, rows, 1}, 128-byte swizzle
-bool map_expert_rows(CUtensorMap* m, const uint16_t* base, int64_t E, int64_t rows, int64_t cols) {
+// fp16 [E, expert_rows, cols]: `rows` rows of every expert (from `base`), box
+// {64, rows, 1}, 128-byte swizzle (expert_rows = rows unless a block of rows
+// of a taller per-expert matrix is mapped)
+bool map_expert_rows(CUtensorMap* m, const uint16_t* base, int64_t E, int64_t rows, int64_t cols,
+                     int64_t expert_rows = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  if (expert_rows <= 0) expert_rows = rows;
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)E};
-  cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(cols * rows * 2)};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(cols * expert_rows * 2)};
   cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
@@ -373,14 +378,24 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   SkMaps sm;
   const int rows_grid = grid_for_tiles(sms, 2 * max_tiles, 1);
 
-  // xa = c * X_perm [A_g; A_u]^T: gate in columns [0, r), up in [rp, rp + r)
-  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.xp), L.rows, H, 128) ||
-      !map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.gu16), E, 2 * rp, H))
-    return RAWINT4_CUDA_ERROR;
-  sp.nseg = 1;
+  // xa = c * X_perm [A_g; A_u]^T: gate in columns [0, r), up in [rp, rp + r);
+  // both rank blocks in one 64-wide segment up to rank 32, one segment each
+  // above (the same X_perm columns, the gate and up halves of gu16)
+  if (!map_act(&sm.a[0], at<uint16_t>(ws, L.xp), L.rows, H, 128)) return RAWINT4_CUDA_ERROR;
+  if (2 * rp <= 64) {
+    if (!map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.gu16), E, 2 * rp, H)) return RAWINT4_CUDA_ERROR;
+    sp.nseg = 1;
+    sp.sw = 2 * rp;
+  } else {
+    if (!map_expert_rows(&sm.b[0], at<uint16_t>(ws, L.gu16), E, rp, H, 2 * rp) ||
+        !map_expert_rows(&sm.b[1], at<uint16_t>(ws, L.gu16) + (int64_t)rp * H, E, rp, H, 2 * rp))
+      return RAWINT4_CUDA_ERROR;
+    sp.nseg = 2;
+    sp.seg_lcol[1] = 0;
+    sp.sw = rp;
+  }
   sp.seg_lcol[0] = 0;
   sp.nk = H / 64;
-  sp.sw = 2 * rp;
   sp.out0 = at<uint16_t>(ws, L.xa);
   sp.out1 = nullptr;
   if (has_lora) {
@@ -668,15 +683,28 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     gq.rpad = rp;
     gq.offsets = at<int32_t>(ws, L.offsets);
     gq.experts = E;
-    gq.njobs = 4;
     gq.accumulate = accumulate;
     gq.grad_scale = grad_scale;
-    // L (features), S (rank side), split, transposed, output features, outputs
+    // features, first L column, L map, S map, first S column, feature
+    // blocks, split, transposed, output features, outputs. Maps: L = gp, h,
+    // dgu, xp; S = hw, gdw, xa, gb (each S holds the rank blocks at [0, r)
+    // and, for the gate/up pairs, [rp, rp + r)).
     auto nfb = [](int P) { return (P + 127) / 128; };  // a partial last block is masked
-    gq.job[0] = SkJob{H, 0, nfb(H), kSplitNone, 0, H, grads->down_b, nullptr};
-    gq.job[1] = SkJob{I, 0, nfb(I), kSplitNone, 1, I, grads->down_a, nullptr};
-    gq.job[2] = SkJob{2 * I, 0, nfb(2 * I), kSplitFeature, 0, I, grads->gate_b, grads->up_b};
-    gq.job[3] = SkJob{H, 0, nfb(H), kSplitRank, 1, H, grads->gate_a, grads->up_a};
+    gq.job[0] = SkJob{H, 0, 0, 0, 0, nfb(H), kSplitNone, 0, H, grads->down_b, nullptr};
+    gq.job[1] = SkJob{I, 0, 1, 1, 0, nfb(I), kSplitNone, 1, I, grads->down_a, nullptr};
+    if (2 * rp <= 64) {
+      // both rank blocks inside the 64 D columns of one job
+      gq.njobs = 4;
+      gq.job[2] = SkJob{2 * I, 0, 2, 2, 0, nfb(2 * I), kSplitFeature, 0, I, grads->gate_b, grads->up_b};
+      gq.job[3] = SkJob{H, 0, 3, 3, 0, nfb(H), kSplitRank, 1, H, grads->gate_a, grads->up_a};
+    } else {
+      // a job per gate/up buffer, each reading its rank block of S
+      gq.njobs = 6;
+      gq.job[2] = SkJob{I, 0, 2, 2, 0, nfb(I), kSplitNone, 0, I, grads->gate_b, nullptr};
+      gq.job[3] = SkJob{I, I, 2, 2, rp, nfb(I), kSplitNone, 0, I, grads->up_b, nullptr};
+      gq.job[4] = SkJob{H, 0, 3, 3, 0, nfb(H), kSplitNone, 1, H, grads->gate_a, nullptr};
+      gq.job[5] = SkJob{H, 0, 3, 3, rp, nfb(H), kSplitNone, 1, H, grads->up_a, nullptr};
+    }
     SkMaps gm;
     if (!map_act(&gm.a[0], at<uint16_t>(ws, L.gp), L.rows, H, 64) ||
         !map_act(&gm.b[0], at<uint16_t>(ws, L.hw), L.rows, kLoraPad, 64) ||
@@ -687,7 +715,8 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
         !map_act(&gm.a[3], at<uint16_t>(ws, L.xp), L.rows, H, 64) ||
         !map_act(&gm.b[3], at<uint16_t>(ws, L.gb), L.rows, kLoraPad, 64))
       return RAWINT4_CUDA_ERROR;
-    const int items = E * (nfb(H) + nfb(I) + nfb(2 * I) + nfb(H));
+    int items = 0;
+    for (int j = 0; j < gq.njobs; ++j) items += E * gq.job[j].nfb;
     R4_PROF("lora_grads", st);
     R4_TRY(launch_skinny(kSkGrads, gq, gm, grid_for_tiles(sms, items, 1), st));
   }

@@ -65,6 +65,9 @@ __device__ __forceinline__ int dy_scale_exponent(uint32_t amax_bits16) {
   return min(120, max(-120, 1 - e));
 }
 constexpr uint32_t kWsMagic = 0x52344d45u;  // "R4ME"
+// Width (fp16 columns) of the rank-side matrices of the LoRA products: the gate
+// and up rank blocks, each padded to a multiple of 16 (rank <= 64).
+constexpr int kLoraPad = 128;
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s bound on any spin
 

@@ -25,7 +25,6 @@ enum GemmMode : int {
 
 constexpr int kBlockK = 64;        // reduction elements per pipeline stage
 constexpr int kTmAccCols = 192;    // gemm_tm.cu: columns of one TMEM accumulator = max token-tile rows
-constexpr int kLoraPad = 64;       // width of the LoRA side matrices (>= 2 * rank)
 
 // ------------------------------------------------ shared by the pair kernels
 constexpr uint64_t kDrainNs = 20000000ull;  // bound on the drains of an aborted call (20 ms)

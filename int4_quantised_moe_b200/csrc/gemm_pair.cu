@@ -190,12 +190,13 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// This thread's 32 values of the A tile of the LoRA reduction stage, as 16
-// fp16 pairs in decode order (see a_chunk_off). Loaded at the start of a work
-// item, long before the stage is stored, which takes the latency of these
-// loads off the critical path.
+// This thread's 32 values of the A tile of the LoRA reduction stage that
+// starts at column k0, as 16 fp16 pairs in decode order (see a_chunk_off).
+// The first stage's values are loaded at the start of a work item, long
+// before the stage is stored, which takes the latency of these loads off the
+// critical path.
 template <int MODE>
-__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, int dt, uint32_t (&w)[16]) {
+__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, int dt, int k0, uint32_t (&w)[16]) {
   const int r = p.rank;
   if constexpr (!kAMnMajor<MODE>) {
     // A[m, j], j in [32 half, 32 half + 32): LoRA B rows (rank contiguous)
@@ -214,14 +215,14 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, 
       float v[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int jj = 32 * half + 2 * t + u - jlo;
+        const int jj = k0 + 32 * half + 2 * t + u - jlo;
         v[u] = (src != nullptr && jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
       }
       w[t] = pack_h2(v[0], v[1]);
     }
   } else {
     // A[m, kr], m in [32 qq, 32 qq + 32): LoRA A rows (feature contiguous)
-    const int kr = mn_kr(dt), f = fc + 32 * mn_qq(dt);
+    const int kr = k0 + mn_kr(dt), f = fc + 32 * mn_qq(dt);
     const uint16_t* src = nullptr;
     if (f < p.feat) {
       if (kr < r)
@@ -324,6 +325,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_rowblk = p.n_rowblk;
   const int n_tiles = (p.need_saved && p.hdr->saved != 1u) ? 0 : p.hdr->n_tok_tiles * n_rowblk;
   const int n_main = p.n_main;
+  // LoRA side product: 64-wide reduction stages over the rank blocks (two
+  // for the gate/up pair with a rank above 32)
+  const int n_lora = (kext_steps<MODE>(p.rpad) + kBlockK / 16 - 1) / (kBlockK / 16);
   const int tile0 = (int)cluster_id_x();
   const int tile_step = (int)cluster_count_x();
   uint32_t* status = p.status;
@@ -391,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int nb = pair_n(tt.z) / 2;  // this CTA's token rows (multiple of 16)
       const int row0 = tt.y + cta * nb;
-      for (int s = 0; s <= n_main; ++s) {
+      for (int s = 0; s < n_main + n_lora; ++s) {
         if (!wait_warp(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_b;
         if (lane == 0) {
           uint8_t* dst = sB + ring.stage * kBBytes;
@@ -404,7 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (s < n_main)
                 tma_load_2d_pair(dst + row * 128, &maps.b[lvl], bar, s * kBlockK, row0 + row);
               else
-                tma_load_2d_pair(dst + row * 128, &maps.bx[lvl], bar, 0, row0 + row);
+                tma_load_2d_pair(dst + row * 128, &maps.bx[lvl], bar, kBlockK * (s - n_main), row0 + row);
               row += h;
             }
           }
@@ -451,10 +455,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           {
             const uint32_t d_tmem = tmem + (uint32_t)(ab * 256);
             uint32_t acc = 0u;  // the item's first UMMA overwrites the accumulator
-            // main stages in groups of kGroup, then the LoRA stage alone
+            // main stages in groups of kGroup, then the LoRA stages as a group
             for (int s = 0; s <= n_main; s += kGroup) {
               const bool lora = s == n_main;
-              const int nb = lora ? 1 : min(kGroup, n_main - s);
+              const int nb = lora ? n_lora : min(kGroup, n_main - s);
               if (!wait_issuer(&a_full[rg.stage], rg.phase, abort_flag, status, lim)) {
                 aborted = true;
                 goto mma_out;
@@ -470,7 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     acc = 1u;
                   }
                 } else {
-                  for (int kk = 0; kk < ksteps_x; ++kk) {
+                  const int ks = min(kBlockK / 16, ksteps_x - (kBlockK / 16) * b);
+                  for (int kk = 0; kk < ks; ++kk) {
                     umma_f16_pair(d_tmem, ad + kAStep * kk, bd + (uint64_t)(2 * kk), idesc, acc);
                     acc = 1u;
                   }
@@ -657,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       const int e = tt.x;
       uint32_t lora_w[16];
-      lora_values<MODE>(p, e, fc, dt, lora_w);
+      lora_values<MODE>(p, e, fc, dt, 0, lora_w);
       for (int s = 0; s < n_main; s += kGroup) {
         const int nb = min(kGroup, n_main - s);
         // decode the group into registers (needs only its packed and scale
@@ -716,18 +721,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
         rg.advance(kAGroups);
       }
-      // the LoRA reduction stage, a group of its own
+      // the LoRA reduction stages, a group of their own (the second one, for a
+      // rank above 32, loaded here)
       {
+        uint32_t lora_w1[16];
+        if (n_lora > 1) lora_values<MODE>(p, e, fc, dt, kBlockK, lora_w1);
         if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
         uint8_t* A = sA + (kGroup * rg.stage) * kABytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
               make_uint4(lora_w[4 * j], lora_w[4 * j + 1], lora_w[4 * j + 2], lora_w[4 * j + 3]);
+        if (n_lora > 1) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(A + kABytes + a_chunk_off<MODE>(dt, j)) =
+                make_uint4(lora_w1[4 * j], lora_w1[4 * j + 1], lora_w1[4 * j + 2], lora_w1[4 * j + 3]);
+        }
         fence_proxy_async_smem();
         if (b_watch) {
-          if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
-          rbd.advance(kStagesB);
+          for (int b = 0; b < n_lora; ++b) {
+            if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+            rbd.advance(kStagesB);
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));

@@ -344,11 +344,13 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Row m, reduction group g of the LoRA stage (columns [32 g, 32 g + 32)) as
-// 16 fp16 pairs: the LoRA B row of the weight row (rank contiguous), placed at
-// the rank block of its projection.
+// Row m, reduction group g of the LoRA stage that starts at column k0
+// (columns [k0 + 32 g, k0 + 32 g + 32)) as 16 fp16 pairs: the LoRA B row of
+// the weight row (rank contiguous), placed at the rank block of its
+// projection.
 template <int MODE>
-__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, int m, int g, uint32_t (&w)[16]) {
+__device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, int m, int g, int k0,
+                                            uint32_t (&w)[16]) {
   const int r = p.rank;
   const uint16_t* src = nullptr;
   int jlo = 0;
@@ -365,7 +367,7 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, 
     float v[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int jj = 32 * g + 2 * t + u - jlo;
+      const int jj = k0 + 32 * g + 2 * t + u - jlo;
       v[u] = (src != nullptr && jj >= 0 && jj < r) ? bf16_bits_to_float(__ldg(src + jj)) : 0.0f;
     }
     w[t] = pack_h2(v[0], v[1]);
@@ -373,11 +375,12 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, 
 }
 
 // MN-major: weight row m (feature fc + m), reduction group g of the LoRA
-// stage: the LoRA A column of the feature (rank rows [32 g, 32 g + 32) of the
-// 64-wide stage: gate/up^T stacks gate ranks at [0, r) and up ranks at
-// [rpad, rpad + r)), as 16 fp16 pairs.
+// stage that starts at column k0: the LoRA A column of the feature (rank rows
+// [k0 + 32 g, k0 + 32 g + 32); gate/up^T stacks gate ranks at [0, r) and up
+// ranks at [rpad, rpad + r)), as 16 fp16 pairs.
 template <int MODE>
-__device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int fc, int m, int g, uint32_t (&w)[16]) {
+__device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int fc, int m, int g, int k0,
+                                               uint32_t (&w)[16]) {
   const int r = p.rank;
   const int f = fc + m;
 #pragma unroll
@@ -385,7 +388,7 @@ __device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int f
     float v[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int kr = 32 * g + 2 * t + u;
+      const int kr = k0 + 32 * g + 2 * t + u;
       const uint16_t* src = nullptr;
       if (f < p.feat) {
         if (kr < r)
@@ -478,6 +481,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_main = p.n_main;
   constexpr int PS = kPSub<MODE>;                   // reduction stages per packed slot
   const int n_slots = (n_main + PS - 1) / PS;
+  // LoRA side product: 64-wide reduction stages over the rank blocks (two
+  // for the gate/up pair with a rank above 32)
+  const int n_lora = (kext_steps<MODE>(p.rpad) + kBlockK / 16 - 1) / (kBlockK / 16);
   const int tile0 = (int)cluster_id_x();
   const int tile_step = (int)cluster_count_x();
   uint32_t* status = p.status;
@@ -558,12 +564,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int nb = pair_n(tt.z) / 2;  // this CTA's token rows (multiple of 16)
       const int row0 = tt.y + cta * nb;
       const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
-      // the item's stage order: slot-rotated main stages, then the LoRA stage
+      // the item's stage order: slot-rotated main stages, then the LoRA stages
       for (int j0 = 0; j0 <= n_slots; ++j0) {
         const int j = j0 < n_slots ? rotated(j0, rot, n_slots) : 0;
-        const int nsub = j0 < n_slots ? min(PS, n_main - PS * j) : 1;
+        const int nsub = j0 < n_slots ? min(PS, n_main - PS * j) : n_lora;
         for (int u = 0; u < nsub; ++u) {
-        const int s = j0 < n_slots ? PS * j + u : n_main;
+        const int s = j0 < n_slots ? PS * j + u : n_main + u;
         if (!wait_warp(&b_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_b;
         if (lane == 0) {
           uint8_t* dst = sB + ring.stage * kBBytes;
@@ -576,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (s < n_main)
                 tma_load_2d_pair(dst + row * 128, &maps.b[lvl], bar, s * kBlockK, row0 + row);
               else
-                tma_load_2d_pair(dst + row * 128, &maps.bx[lvl], bar, 0, row0 + row);
+                tma_load_2d_pair(dst + row * 128, &maps.bx[lvl], bar, kBlockK * (s - n_main), row0 + row);
               row += h;
             }
           }
@@ -626,7 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // slot, then the LoRA stage as a group of its own
             for (int j0 = 0; j0 <= n_slots; ++j0) {
               const bool lora = j0 == n_slots;
-              const int nsub = lora ? 1 : min(PS, n_main - PS * rotated(j0, rot, n_slots));
+              const int nsub = lora ? n_lora : min(PS, n_main - PS * rotated(j0, rot, n_slots));
               for (int u = 0; u < nsub; u += kGroup) {
                 const int nb = min(kGroup, nsub - u);
                 if (!wait_issuer(&a_full[rg.stage], rg.phase, abort_flag, status, lim)) {
@@ -644,7 +650,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       acc = 1u;
                     }
                   } else {
-                    for (int kk = 0; kk < ksteps_x; ++kk) {
+                    const int ks = min(kBlockK / 16, ksteps_x - (kBlockK / 16) * (u + b));
+                    for (int kk = 0; kk < ks; ++kk) {
                       umma_f16_pair_ts(d_tmem, a_tm + (uint32_t)(8 * kk), bd + (uint64_t)(2 * kk), idesc, acc);
                       acc = 1u;
                     }
@@ -895,9 +902,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
       uint32_t lora_w[16];
       if constexpr (kAMnMajor<MODE>)
-        lora_values_mn<MODE>(p, e, fc, m, g, lora_w);
+        lora_values_mn<MODE>(p, e, fc, m, g, 0, lora_w);
       else
-        lora_values<MODE>(p, e, fc, m, g, lora_w);
+        lora_values<MODE>(p, e, fc, m, g, 0, lora_w);
       for (int j0 = 0; j0 < n_slots; ++j0) {
         const int j = rotated(j0, rot, n_slots);
         const int nsub = min(PS, n_main - PS * j);
@@ -939,14 +946,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         rp.advance(kStagesP<MODE>);
         rs.advance(kStagesS);
       }
-      // the LoRA stage, a group of its own
+      // the LoRA stages, a group of their own (the second one, for a rank
+      // above 32, loaded here)
+      uint32_t lora_w1[16];
+      if (n_lora > 1) {
+        if constexpr (kAMnMajor<MODE>)
+          lora_values_mn<MODE>(p, e, fc, m, g, kBlockK, lora_w1);
+        else
+          lora_values<MODE>(p, e, fc, m, g, kBlockK, lora_w1);
+      }
       if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
       tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 16 * g), lora_w);
+      if (n_lora > 1) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 32 + 16 * g), lora_w1);
       tmem_wait_st();
       tc_fence_before();
       if (b_watch) {
-        if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
-        rbd.advance(kStagesB);
+        for (int b = 0; b < n_lora; ++b) {
+          if (!wait_warp(&b_full[rbd.stage], rbd.phase, abort_flag, status, lim)) goto done;
+          rbd.advance(kStagesB);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));

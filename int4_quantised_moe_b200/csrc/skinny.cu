@@ -74,21 +74,22 @@ __device__ __forceinline__ uint32_t grad_pair(uint32_t old, float a, float b, in
   return (uint32_t)bf16_bits_rn(a) | ((uint32_t)bf16_bits_rn(b) << 16);
 }
 
-// The `rank` gradient values of feature pp of expert e in one output buffer:
-// buf = (accumulate ? buf : 0) + gs * D[j], D read from the accumulator
-// columns in `v` (all zero when `zero`). [E, pout, r] rows are contiguous and
-// go out as 16-byte vectors when r is a multiple of 8 and the buffer is
-// 16-byte aligned; [E, r, pout] columns are written one element per rank
-// index, contiguous across the warp's lanes.
-__device__ __forceinline__ void grad_row(uint16_t* buf, const SkJob& jb, int rank, int e, int pp, const uint32_t (&v)[32],
-                                         float gs, int accumulate, bool zero) {
+// Ranks [jlo, jlo + n) (n <= 32) of feature pp of expert e in one output
+// buffer whose rank extent is `ld`: buf = (accumulate ? buf : 0) + gs * D[j],
+// D read from the accumulator columns in `v` (all zero when `zero`).
+// [E, pout, ld] rows are contiguous and go out as 16-byte vectors when n, ld
+// and jlo are multiples of 8 and the buffer is 16-byte aligned; [E, ld, pout]
+// columns are written one element per rank index, contiguous across the
+// warp's lanes.
+__device__ __forceinline__ void grad_row(uint16_t* buf, const SkJob& jb, int ld, int jlo, int n, int e, int pp,
+                                         const uint32_t (&v)[32], float gs, int accumulate, bool zero) {
   if (zero) accumulate = 0;
   if (!jb.transposed) {
-    uint16_t* dst = buf + ((int64_t)e * jb.pout + pp) * rank;
-    if ((rank & 7) == 0 && (reinterpret_cast<uintptr_t>(buf) & 15u) == 0) {
+    uint16_t* dst = buf + ((int64_t)e * jb.pout + pp) * ld + jlo;
+    if (((n | ld | jlo) & 7) == 0 && (reinterpret_cast<uintptr_t>(buf) & 15u) == 0) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        if (8 * c < rank) {
+        if (8 * c < n) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + 8 * c);
           const uint4 old = accumulate ? *d4 : make_uint4(0u, 0u, 0u, 0u);
           const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
@@ -105,41 +106,48 @@ __device__ __forceinline__ void grad_row(uint16_t* buf, const SkJob& jb, int ran
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (j < rank) grad_store(dst, j, zero ? 0.f : gs * __uint_as_float(v[j]), accumulate);
+        if (j < n) grad_store(dst, j, zero ? 0.f : gs * __uint_as_float(v[j]), accumulate);
     }
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (j < rank)
-        grad_store(buf, ((int64_t)e * rank + j) * jb.pout + pp, zero ? 0.f : gs * __uint_as_float(v[j]), accumulate);
+      if (j < n)
+        grad_store(buf, ((int64_t)e * ld + jlo + j) * jb.pout + pp, zero ? 0.f : gs * __uint_as_float(v[j]),
+                   accumulate);
   }
 }
 
-// The [E, r, pout] outputs of one 128-feature block (two for the rank split):
-// the four epilogue warps write their features' gradients into shared memory,
-// then store whole 256-byte rows (8 features per thread and step) with the
-// authoritative-window rule (accumulate: add the old value, round once).
-// All 128 epilogue threads take part (named barrier 1).
-__device__ __forceinline__ void grad_block_transposed(const SkJob& jb, int rank, int e, int p0, uint16_t* out0, bool both,
-                                                      const uint32_t (&v0)[32], const uint32_t (&v1)[32], float gs,
-                                                      int accumulate, bool zero, float* st, int c, int tid) {
+// One part of the [E, ld, pout] outputs of a 128-feature block: ranks
+// [jlo, jlo + n) (n <= 32) of buffer `buf`, from `v`.
+struct GradPart {
+  uint16_t* buf;
+  int jlo, n;
+};
+
+// The transposed outputs of one 128-feature block, in up to two parts (the
+// two buffers of the rank split, or the two rank halves of a rank above 32):
+// the four epilogue warps write their features' gradients into shared
+// memory, then store whole 256-byte rows (8 features per thread and step)
+// with the authoritative-window rule (accumulate: add the old value, round
+// once). All 128 epilogue threads take part (named barrier 1).
+__device__ __forceinline__ void grad_block_transposed(const SkJob& jb, int ld, int e, int p0, GradPart q0, GradPart q1,
+                                                      int nparts, const uint32_t (&v0)[32], const uint32_t (&v1)[32],
+                                                      float gs, int accumulate, bool zero, float* st, int c, int tid) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    if (j < rank) {
-      st[j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v0[j]);
-      if (both) st[4096 + j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v1[j]);
-    }
+    if (j < q0.n) st[j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v0[j]);
+    if (nparts > 1 && j < q1.n) st[4096 + j * 128 + c] = zero ? 0.f : gs * __uint_as_float(v1[j]);
   }
   named_bar_sync(1, 128);
-  const int nout = both ? 2 : 1;
-  for (int idx = tid; idx < nout * rank * 16; idx += 128) {
-    const int o = idx / (rank * 16);
-    const int rem = idx - o * rank * 16;
+  const int n_all = q0.n * 16 + (nparts > 1 ? q1.n * 16 : 0);
+  for (int idx = tid; idx < n_all; idx += 128) {
+    const int o = idx < q0.n * 16 ? 0 : 1;
+    const int rem = o ? idx - q0.n * 16 : idx;
     const int j = rem >> 4, v8 = rem & 15;
     const float* src = st + o * 4096 + j * 128 + 8 * v8;
     if (p0 + 8 * v8 >= jb.pout) continue;  // past the last feature (a partial last block)
-    uint16_t* buf = o ? jb.out_hi : out0;
-    uint4* dst = reinterpret_cast<uint4*>(buf + ((int64_t)e * rank + j) * jb.pout + p0 + 8 * v8);
+    const GradPart& q = o ? q1 : q0;
+    uint4* dst = reinterpret_cast<uint4*>(q.buf + ((int64_t)e * ld + q.jlo + j) * jb.pout + p0 + 8 * v8);
     const uint4 old = accumulate ? *dst : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
     uint32_t nw[4];
@@ -226,9 +234,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             uint8_t* st = smem + ring.stage * kSkStage;
             mbar_expect_tx(&full[ring.stage], kSkA + kSkB);
             const int x = jb.lcol + 128 * g.fb;
-            tma_load_2d(st, &maps.a[g.job], &full[ring.stage], x, row0 + 64 * k);
-            tma_load_2d(st + kSkA / 2, &maps.a[g.job], &full[ring.stage], x + 64, row0 + 64 * k);
-            tma_load_2d(st + kSkA, &maps.b[g.job], &full[ring.stage], 0, row0 + 64 * k);
+            tma_load_2d(st, &maps.a[jb.amap], &full[ring.stage], x, row0 + 64 * k);
+            tma_load_2d(st + kSkA / 2, &maps.a[jb.amap], &full[ring.stage], x + 64, row0 + 64 * k);
+            tma_load_2d(st + kSkA, &maps.b[jb.bmap], &full[ring.stage], jb.scol, row0 + 64 * k);
           }
           __syncwarp();
           ring.advance(kSkStages);
@@ -323,7 +331,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const float w = (p.out1 && m < nrows) ? __ldg(p.w_perm + row) : 0.f;
         // output column c = s * sw + j  <-  accumulator column s * 64 + j,
         // kept when j lies inside a rank block (j % rpad < rank)
-        for (int c0 = 0; c0 < 64; c0 += 16) {
+        const int ncols = p.nseg * p.sw > 64 ? kLoraPad : 64;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
           const int s = c0 / p.sw;
           const int j0 = c0 - s * p.sw;
           uint32_t v[16];
@@ -342,11 +351,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
               __half2 hw = __floats2half2_rn(w * a, w * b);
               o1[t] = *reinterpret_cast<uint32_t*>(&hw);
             }
-            uint4* d0 = reinterpret_cast<uint4*>(p.out0 + row * 64 + c0);
+            uint4* d0 = reinterpret_cast<uint4*>(p.out0 + row * kLoraPad + c0);
             d0[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
             d0[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
             if (p.out1) {
-              uint4* d1 = reinterpret_cast<uint4*>(p.out1 + row * 64 + c0);
+              uint4* d1 = reinterpret_cast<uint4*>(p.out1 + row * kLoraPad + c0);
               d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
               d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
             }
@@ -377,6 +386,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           pbase = jb.P / 2;
         }
         const bool both = jb.split == kSplitRank;
+        const bool wide = !both && p.rank > 32;  // one buffer, ranks from D columns [0, rank)
+        // the parts this lane writes: (buffer, first rank, ranks) from v0 and v1
+        GradPart q0{out0, 0, min(p.rank, 32)}, q1{nullptr, 0, 0};
+        int nparts = 1;
+        if (both) {
+          q1 = GradPart{jb.out_hi, 0, p.rank};
+          nparts = 2;
+        } else if (wide) {
+          q1 = GradPart{out0, 32, p.rank - 32};
+          nparts = 2;
+        }
         const bool live = pf < jb.P;
         uint32_t v0[32], v1[32];
         if (rows == 0) {
@@ -385,11 +405,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
           if (jb.transposed) {
-            grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, 0.f, 0, true, gstage,
+            grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, q0, q1, nparts, v0, v1, 0.f, 0, true, gstage,
                                   32 * q + lane, threadIdx.x - 64);
           } else if (live) {
-            grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, 0.f, 0, true);
-            if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v0, 0.f, 0, true);
+            grad_row(q0.buf, jb, p.rank, q0.jlo, q0.n, g.e, pf - pbase, v0, 0.f, 0, true);
+            if (nparts > 1) grad_row(q1.buf, jb, p.rank, q1.jlo, q1.n, g.e, pf - pbase, v1, 0.f, 0, true);
           }
           continue;
         }
@@ -399,16 +419,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const uint32_t t0 = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * 128);
         tmem_ld32(t0 + col0, v0);
         if (both) tmem_ld32(t0 + (uint32_t)p.rpad, v1);
+        if (wide) tmem_ld32(t0 + 32u, v1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
         ++it;
         if (jb.transposed) {
-          grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, out0, both, v0, v1, gsc, p.accumulate,
+          grad_block_transposed(jb, p.rank, g.e, 128 * g.fb - pbase, q0, q1, nparts, v0, v1, gsc, p.accumulate,
                                 false, gstage, 32 * q + lane, threadIdx.x - 64);
         } else if (live) {
-          grad_row(out0, jb, p.rank, g.e, pf - pbase, v0, gsc, p.accumulate, false);
-          if (both) grad_row(jb.out_hi, jb, p.rank, g.e, pf, v1, gsc, p.accumulate, false);
+          grad_row(q0.buf, jb, p.rank, q0.jlo, q0.n, g.e, pf - pbase, v0, gsc, p.accumulate, false);
+          if (nparts > 1) grad_row(q1.buf, jb, p.rank, q1.jlo, q1.n, g.e, pf - pbase, v1, gsc, p.accumulate, false);
         }
       }
     }
@@ -470,7 +491,7 @@ __global__ void __launch_bounds__(256) lora_convert_kernel(LoraCvt j0, LoraCvt j
       dst[idx] = out;
     }
   } else {
-    __shared__ float tile[64][33];
+    __shared__ float tile[64][65];  // 64 source rows x up to 64 ranks (+1: no bank conflicts)
     const int tiles_per_e = cols / 64;
     for (int t = blockIdx.x; t < experts * tiles_per_e; t += gridDim.x) {
       const int e = t / tiles_per_e;

@@ -10,14 +10,20 @@ namespace r4 {
 //   out0[p, seg*sw + j] = scale * sum_k L[p, lcol[seg] + k] * R_seg[e][j][k]
 //   out1[p, ...]        = w_perm[p] * out0[p, ...]               (optional)
 //   (tokens on M, rank on N; R_seg are the FP16 LoRA tensors laid out
-//   [E, sw, K] so that both operands are K-major; sw is a multiple of 16.)
-//   Within a segment, column j is kept when j % rpad < rank (the rest are
-//   the zero rows that pad each rank block to rpad = roundup16(rank)).
+//   [E, sw, K] so that both operands are K-major; sw is a multiple of 16,
+//   at most 64.) Within a segment, column j is kept when j % rpad < rank (the
+//   rest are the zero rows that pad each rank block to rpad =
+//   roundup16(rank)). The side matrices are kLoraPad columns wide; columns
+//   past the segments are written as zeros up to 64 (all kLoraPad when the
+//   segments reach past 64).
 // kSkGrads: the six LoRA gradients, per (job, expert, 128-feature block)
-//   D[p, j] = sum over the expert's rows of L[row, lcol + p] * S[row, j]
-//   (features on M, rank on N, reduction over the expert's rows; both
-//   operands MN-major) stored with the authoritative window of the contract
-//   test: buf = (accumulate ? buf : 0) + grad_scale * D.
+//   D[p, j] = sum over the expert's rows of L[row, lcol + p] * S[row, scol + j]
+//   (features on M, 64 rank columns on N, reduction over the expert's rows;
+//   both operands MN-major) stored with the authoritative window of the
+//   contract test: buf = (accumulate ? buf : 0) + grad_scale * D. A rank up
+//   to 32 lets one job carry the gate and up rank blocks (the splits below);
+//   a larger rank gives every output buffer a job of its own (kSplitNone,
+//   ranks from D columns [0, rank)).
 enum SkMode : int { kSkRows = 0, kSkGrads = 1 };
 
 constexpr int kSkThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
@@ -34,6 +40,9 @@ enum SkSplit : int {
 struct SkJob {
   int P;           // features of L used by the job (M extent)
   int lcol;        // first column of L
+  int amap;        // tensor map of L (SkMaps::a)
+  int bmap;        // tensor map of S (SkMaps::b)
+  int scol;        // first column of S
   int nfb;         // 128-feature blocks: ceil(P / 128)
   int split;       // SkSplit
   int transposed;  // 0: out[e][p][j] ([E, Pout, r]); 1: out[e][j][p] ([E, r, Pout])
@@ -62,14 +71,14 @@ struct SkParams {
   const int32_t* offsets;
   int experts;
   int njobs;
-  SkJob job[4];
+  SkJob job[6];
   int accumulate;
   float grad_scale;
 };
 
 struct SkMaps {
-  CUtensorMap a[4];  // rows: [0] L (box {64, 128}); grads: L of each job (box {64, 64})
-  CUtensorMap b[4];  // rows: R of each segment (3D, box {64, 64, 1}); grads: S of each job (box {64, 64})
+  CUtensorMap a[4];  // rows: [0] L (box {64, 128}); grads: the L tensors of the jobs (box {64, 64})
+  CUtensorMap b[4];  // rows: R of each segment (3D, box {64, sw, 1}); grads: the S tensors of the jobs (box {64, 64})
 };
 
 cudaError_t launch_skinny(int mode, const SkParams& p, const SkMaps& m, int grid, cudaStream_t stream);

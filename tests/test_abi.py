@@ -49,12 +49,14 @@ def test_workspace_size_and_cfg_validation(lib):
     assert lib.rawint4_moe_lora_workspace_size(big) > n
     gemma = lib.make_cfg(128, 8, 2816, 704, 8, 16.0, 0.0, 32)  # H, I multiples of 64 (not of 128)
     assert lib.rawint4_moe_lora_workspace_size(gemma) > 0
+    for r in (33, 48, 64):  # ranks above 32: two rank segments and LoRA stages
+        assert lib.rawint4_moe_lora_workspace_size(lib.make_cfg(4, 2, 256, 256, r, 2.0 * r, 0.0, 32)) > 0
     bad = [
         lib.make_cfg(4, 2, 200, 256, 8, 16.0, 0.0, 32),   # H not a multiple of 64
         lib.make_cfg(4, 2, 256, 96, 8, 16.0, 0.0, 32),    # I not a multiple of 64
         lib.make_cfg(4, 5, 256, 256, 8, 16.0, 0.0, 32),   # top_k > experts
         lib.make_cfg(4, 2, 256, 256, 0, 16.0, 0.0, 32),   # rank 0
-        lib.make_cfg(4, 2, 256, 256, 33, 16.0, 0.0, 32),  # rank > 32
+        lib.make_cfg(4, 2, 256, 256, 65, 16.0, 0.0, 32),  # rank > 64
         lib.make_cfg(4, 2, 256, 256, 8, float("nan"), 0.0, 32),
         lib.make_cfg(4, 2, 256, 256, 8, 16.0, -1.0, 32),  # negative clamp limit
         lib.make_cfg(4, 2, 256, 256, 8, 16.0, float("inf"), 32),

@@ -41,6 +41,42 @@ def oracle(wl: Workload):
     return out, gin, groute, grads
 
 
+MASK_DELTA = 4e-3  # bound on |G_gpu - G_oracle| (fp32 accumulation vs float64), as in test_gpu_fullsize
+
+
+def oracle_gpu_masks(wl: Workload, perm, G, U):
+    """The oracle with the clamp masks decided the GPU's way inside the band
+    where both decisions are correct within fp32 (|G - L|, |U +- L| below
+    MASK_DELTA): the GPU's saved fp32 pre-activations (perm, G, U from
+    Layer.saved_preacts) must lie within MASK_DELTA of the oracle's, and
+    every mask decision outside the band is the oracle's own. Returns the
+    oracle's (out, grad_in, grad_route, grads) and the number of elements
+    decided inside the band."""
+    layer = oracle_layer(wl)
+    L = float(wl.cfg.swiglu_limit)
+    k = wl.cfg.top_k
+    out, ctx = omoe.forward(layer, f64(wl.x), wl.expert_ids.cpu().numpy(), f64(wl.route_weights))
+    perm_h = perm.cpu().numpy()
+    inv = np.full(perm_h.size, -1, dtype=np.int64)
+    inv[perm_h] = np.arange(perm_h.size)
+    Gh, Uh = G.double().cpu().numpy(), U.double().cpu().numpy()
+    masks, band = {}, 0
+    for e, c in ctx.experts.items():
+        rows = inv[c.slots]
+        g_gpu, u_gpu = Gh[rows], Uh[rows]
+        assert np.abs(g_gpu - c.G).max() <= MASK_DELTA and np.abs(u_gpu - c.U).max() <= MASK_DELTA, e
+        if L > 0:
+            pass_g, pass_u = c.G <= L, (c.U >= -L) & (c.U <= L)
+            near_g = np.abs(c.G - L) < MASK_DELTA
+            near_u = (np.abs(c.U - L) < MASK_DELTA) | (np.abs(c.U + L) < MASK_DELTA)
+            pass_g = np.where(near_g, g_gpu <= L, pass_g)
+            pass_u = np.where(near_u, (u_gpu >= -L) & (u_gpu <= L), pass_u)
+            band += int(near_g.sum() + near_u.sum())
+            masks[e] = (pass_g, pass_u)
+    gin, groute, grads = omoe.backward(layer, ctx, f64(wl.grad_out), masks=masks if L > 0 else None)
+    return (out, gin, groute, grads), band
+
+
 def base_hash(wl: Workload) -> str:
     h = hashlib.sha256()
     for t in (wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s):
@@ -432,6 +468,45 @@ def test_gemma4_shape_parity(limit):
     close("grad_route", groute, groute_r, TOL_ROUTE)
     for n in LORA_NAMES:
         close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("rank,fmt,limit", [(40, "rawint4", 0.0), (64, "rawint4", 0.0), (64, "mxfp4", 0.0),
+                                            (40, "rawint4", 2.0), (64, "rawint4", 2.0)])
+def test_large_rank_parity(rank, fmt, limit):
+    """LoRA ranks above 32 (the boundary allows any positive rank; the
+    kernels take up to 64): the gate and up rank blocks no longer share one
+    64-wide reduction stage, so the gate/up GEMMs run two LoRA stages, the
+    rank-side matrices two segments, and the gate/up LoRA gradients one job
+    per buffer. Config 1's shape, training step against the oracle, with the
+    accumulate/grad_scale window. With the clamp, mask decisions inside the
+    fp32 band are taken from the GPU's saved pre-activations (at rank 40 a
+    gate pre-activation lies 2.6e-5 from the bound)."""
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS[1], rank=rank, alpha=2.0 * rank, weight_format=fmt, swiglu_limit=limit)
+    wl = make_workload(cfg)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out = layer.forward(g.expert_ids, g.route_weights, g.x)
+    perm, G, U = layer.saved_preacts()
+    (out_r, gin_r, groute_r, grads_r), band = oracle_gpu_masks(wl, perm, G, U)
+    gin = torch.full_like(g.x, float("nan"))
+    groute = torch.full(g.expert_ids.shape, float("nan"), dtype=torch.float32, device=DEV)
+    layer.backward(g.grad_out, grads, accumulate=False, grad_scale=0.5, grad_in=gin, grad_route=groute)
+    assert layer.status() == 0
+    print(f"rank {rank} {fmt} L={limit}: clamp elements within {MASK_DELTA} of a bound: {band}")
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], 0.5 * grads_r[n], TOL_LORA)
+    # a second micro-step of the window adds to the buffers
+    run_fwd_bwd(layer, g, grads, grad_scale=0.5, accumulate=True)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+    # the frozen-base forward of the same layer ignores the LoRA tensors
+    base = layer.forward(g.expert_ids, g.route_weights, g.x, save_for_backward=False, use_lora=False)
+    assert torch.isfinite(base.float()).all()
 
 
 @pytest.mark.parametrize("cfg_id,limit", [(0, 0.0), (1, 2.0), (1, 0.0)])
