@@ -12,7 +12,9 @@
 // columns fit, and the epilogue of an item always overlaps the next item's
 // mainloop. Warp roles, in each CTA:
 //   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP)
-//   warp 3      loader of the group scales (cp.async, ring of kStagesS)
+//   warp 3      loader of the group scales (cp.async into the scale slot of
+//               each packed stage; its completion is counted on the packed
+//               stage's barrier, so a decoder waits once per stage for both)
 //   warp 2      TMA producer of this CTA's half of the token tile (ring of kStagesB)
 //   warps 8-15  decoders: int4 -> fp16 into the UMMA A layout (ring of kStagesA)
 //   warp 1      leader CTA: pair-wide UMMA issuer; both CTAs: TMEM allocation
@@ -52,7 +54,7 @@ constexpr int kGroup = 2;          // stages per hand-off (issuer wait, decoder 
 constexpr int kAGroups = kStagesA / kGroup;
 constexpr int kStagesB = 6;        // TMA-loaded B tiles (this CTA's half of up to kTileRows tokens)
 constexpr int kStagesP = 16;       // TMA-loaded packed int4 tiles (4 KB each)
-constexpr int kStagesS = 16;       // group scales of one stage (512 B each)
+constexpr int kStagesS = kStagesP;  // group scales of one stage (512 B each), one slot per packed stage
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
@@ -259,8 +261,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem + kOffP;
   uint8_t* sS = smem + kOffS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
-  uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read it
+  uint64_t* p_full = bars;                   // local: this CTA's packed tile and its scales landed
+  uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read them
   uint64_t* a_full = p_empty + kStagesP;     // leader [kAGroups]: the group's A (both CTAs) and B are ready
   uint64_t* a_empty = a_full + kStagesA;     // both [kAGroups]: the pair MMA finished reading the group's A
   uint64_t* b_full = a_empty + kStagesA;     // leader: both CTAs' B halves landed
@@ -281,7 +283,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStagesP; ++i) {
-      mbar_init(&p_full[i], 1);
+      mbar_init(&p_full[i], 1 + 32);  // the TMA producer's arrival (with its bytes) + the scale loader's lanes
       mbar_init(&p_empty[i], kDecThreads / 32);
     }
     for (int i = 0; i < kAGroups; ++i) {
@@ -291,10 +293,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStagesB; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
-    }
-    for (int i = 0; i < kStagesS; ++i) {
-      mbar_init(&s_full[i], 32);
-      mbar_init(&s_empty[i], kDecThreads / 32);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -379,9 +377,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       for (int s = 0; s < n_main; ++s) {
-        if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
+        if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         load_stage_scales<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
-        cp_async_arrive_noinc(&s_full[ring.stage]);
+        cp_async_arrive_noinc(&p_full[ring.stage]);
         ring.advance(kStagesS);
       }
     }
@@ -674,7 +672,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           rp_[b] = rp;
           rs_[b] = rs;
           if (b < nb) {
-            if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
             if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
             const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
             const uint4 q4 = packed_group<MODE>(sP + rp.stage * kPBytes, dt);
@@ -696,7 +693,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           for (int b = 0; b < nb; ++b) {
             mbar_arrive(&p_empty[rp_[b].stage]);
-            mbar_arrive(&s_empty[rs_[b].stage]);
           }
         }
         if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;

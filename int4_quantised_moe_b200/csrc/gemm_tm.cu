@@ -29,7 +29,9 @@
 //   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP)
 //   warp 1      leader CTA: pair-wide UMMA issuer; both CTAs: TMEM allocation
 //   warp 2      TMA producer of this CTA's half of the token tile (ring of kStagesB)
-//   warp 3      loader of the group scales (cp.async, ring of kStagesS)
+//   warp 3      loader of the group scales (cp.async into the scale slot of
+//               each packed slot; its completion is counted on the packed
+//               slot's barrier, so a decoder waits once per slot for both)
 //   warps 4-7   epilogue: this CTA's TMEM rows -> fused math -> global
 //   warps 8-15  decoders: int4 -> fp16 -> tensor memory (two warps per lane quarter)
 //
@@ -75,7 +77,8 @@ template <int MODE>
 constexpr int kStagesP = kPRing / (kPSub<MODE> * 4096);  // packed slots
 constexpr int kMaxStagesP = 16;
 constexpr int kSSlotBytes = 2048;                 // largest scale slot
-constexpr int kStagesS = 8;                       // scale slots
+constexpr int kStagesS = 8;                       // scale slots: one per packed slot (at most 8 packed slots)
+static_assert(kStagesS >= kPRing / (2 * 4096), "a scale slot for every packed slot");
 constexpr int kThreads = 512;                     // 16 warps
 constexpr int kEpiWarp0 = 4;                      // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                      // warps 8..15: decoders
@@ -413,8 +416,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem + kOffP;
   uint8_t* sS = smem + kOffS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* p_full = bars;                   // local: this CTA's packed tile landed
-  uint64_t* p_empty = p_full + kMaxStagesP;  // local: this CTA's decoders read it
+  uint64_t* p_full = bars;                   // local: this CTA's packed slot and its scales landed
+  uint64_t* p_empty = p_full + kMaxStagesP;  // local: this CTA's decoders read them
   uint64_t* a_full = p_empty + kMaxStagesP;  // leader [kAGroups]: the group's A (both CTAs) and B are ready
   uint64_t* a_empty = a_full + kAStages;     // both [kAGroups]: the pair MMA finished reading the group's A
   uint64_t* b_full = a_empty + kAStages;     // leader: both CTAs' B halves landed
@@ -435,7 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStagesP<MODE>; ++i) {
-      mbar_init(&p_full[i], 1);
+      mbar_init(&p_full[i], 1 + 32);  // the TMA producer's arrival (with its bytes) + the scale loader's lanes
       mbar_init(&p_empty[i], kDecWarps);
     }
     for (int i = 0; i < kAGroups; ++i) {
@@ -445,10 +448,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStagesB; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
-    }
-    for (int i = 0; i < kStagesS; ++i) {
-      mbar_init(&s_full[i], 32);
-      mbar_init(&s_empty[i], kDecWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -544,13 +543,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int rot = k_rotation(tile % n_rowblk, n_rowblk, n_slots);
       for (int j0 = 0; j0 < n_slots; ++j0) {
         const int j = rotated(j0, rot, n_slots);
-        if (!wait_warp(&s_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
+        if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         if constexpr (kAMnMajor<MODE>)
           load_slot_scales_mn<MODE, FMT>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
         else
           load_slot_scales<MODE, FMT>(p, tt.x, fc, j, n_main, lane, sS + ring.stage * kSSlotBytes);
-        cp_async_arrive_noinc(&s_full[ring.stage]);
-        ring.advance(kStagesS);
+        cp_async_arrive_noinc(&p_full[ring.stage]);
+        ring.advance(kStagesP<MODE>);
       }
     }
   drain_s:
@@ -908,7 +907,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int j0 = 0; j0 < n_slots; ++j0) {
         const int j = rotated(j0, rot, n_slots);
         const int nsub = min(PS, n_main - PS * j);
-        if (!wait_warp(&s_full[rs.stage], rs.phase, abort_flag, status, lim)) goto done;
         if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
         // the slot's stages a group at a time: decoded into registers first
         // (that needs only the packed and scale slots), then one wait for the
@@ -921,6 +919,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < kGroup; ++b)
             if (b < nb) decode_stage(rs, rp, u + b, tab + 16 * b, w[b]);
+          if (u + kGroup >= nsub) {
+            // the slot's last group decoded: release the packed and scale
+            // slot once every lane has used the values it loaded (the empty
+            // asm makes the decoded words, which depend on every loaded byte
+            // and scale, inputs, so the loads have returned)
+#pragma unroll
+            for (int b = 0; b < kGroup; ++b)
+              if (b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+          }
           if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
 #pragma unroll
           for (int b = 0; b < kGroup; ++b)
@@ -937,14 +946,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[rg.stage], 0));
           rg.advance(kAGroups);
         }
-        // the packed and scale slots are released after the values that
-        // consume their bytes were stored
-        if (lane == 0) {
-          mbar_arrive(&p_empty[rp.stage]);
-          mbar_arrive(&s_empty[rs.stage]);
-        }
         rp.advance(kStagesP<MODE>);
-        rs.advance(kStagesS);
+        rs.advance(kStagesP<MODE>);
       }
       // the LoRA stages, a group of their own (the second one, for a rank
       // above 32, loaded here)
