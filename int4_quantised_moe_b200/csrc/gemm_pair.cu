@@ -11,10 +11,11 @@
 // CTA's TMEM holds only its 128 rows x N: two accumulators of up to 256
 // columns fit, and the epilogue of an item always overlaps the next item's
 // mainloop. Warp roles, in each CTA:
-//   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP)
-//   warp 3      loader of the group scales (cp.async into the scale slot of
-//               each packed stage; its completion is counted on the packed
-//               stage's barrier, so a decoder waits once per stage for both)
+//   warp 0      TMA producer of this CTA's packed int4 tiles (ring of kStagesP
+//               stages, filled and released in slots of kGroup stages)
+//   warp 3      loader of the group scales (cp.async beside each packed
+//               stage; its completion is counted on the packed slot's
+//               barrier, so a decoder waits once per group for both)
 //   warp 2      TMA producer of this CTA's half of the token tile (ring of kStagesB)
 //   warps 8-15  decoders: int4 -> fp16 into the UMMA A layout (ring of kStagesA)
 //   warp 1      leader CTA: pair-wide UMMA issuer; both CTAs: TMEM allocation
@@ -54,7 +55,10 @@ constexpr int kGroup = 2;          // stages per hand-off (issuer wait, decoder 
 constexpr int kAGroups = kStagesA / kGroup;
 constexpr int kStagesB = 6;        // TMA-loaded B tiles (this CTA's half of up to kTileRows tokens)
 constexpr int kStagesP = 16;       // TMA-loaded packed int4 tiles (4 KB each)
-constexpr int kStagesS = kStagesP;  // group scales of one stage (512 B each), one slot per packed stage
+constexpr int kStagesS = kStagesP;  // group scales of one stage (512 B each), one per packed stage
+// Packed stages and their scales are filled and released in slots of kGroup
+// consecutive stages (a hand-off group): one barrier per slot.
+constexpr int kSlotsP = kStagesP / kGroup;
 constexpr int kThreads = 512;      // 16 warps
 constexpr int kEpiWarp0 = 4;       // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
@@ -69,7 +73,7 @@ constexpr int kOffB = kOffA + kStagesA * kABytes;
 constexpr int kOffP = kOffB + kStagesB * kBBytes;
 constexpr int kOffS = kOffP + kStagesP * kPBytes;
 constexpr int kOffBar = kOffS + kStagesS * kSBytes;
-constexpr int kNumBars = 2 * kStagesP + 2 * kStagesA + 2 * kStagesB + 2 * kStagesS + 4 + 1;
+constexpr int kNumBars = 2 * kSlotsP + 2 * kAGroups + 2 * kStagesB + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kOffEpi = (kOffMisc + 16 + 127) / 128 * 128;
 constexpr int kEpiFloats = 4 * 32 * 33 + 4 * 32;  // DOWN_T route partials; gate/up exchange uses the first 2 * 32 * 33
@@ -261,15 +265,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem + kOffP;
   uint8_t* sS = smem + kOffS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* p_full = bars;                   // local: this CTA's packed tile and its scales landed
-  uint64_t* p_empty = p_full + kStagesP;     // local: this CTA's decoders read them
-  uint64_t* a_full = p_empty + kStagesP;     // leader [kAGroups]: the group's A (both CTAs) and B are ready
-  uint64_t* a_empty = a_full + kStagesA;     // both [kAGroups]: the pair MMA finished reading the group's A
-  uint64_t* b_full = a_empty + kStagesA;     // leader: both CTAs' B halves landed
+  uint64_t* p_full = bars;                   // local [kSlotsP]: this CTA's packed slot and its scales landed
+  uint64_t* p_empty = p_full + kSlotsP;      // local [kSlotsP]: this CTA's decoders read them
+  uint64_t* a_full = p_empty + kSlotsP;      // leader [kAGroups]: the group's A (both CTAs) and B are ready
+  uint64_t* a_empty = a_full + kAGroups;     // both [kAGroups]: the pair MMA finished reading the group's A
+  uint64_t* b_full = a_empty + kAGroups;     // leader: both CTAs' B halves landed
   uint64_t* b_empty = b_full + kStagesB;     // both: the pair MMA finished reading B
-  uint64_t* s_full = b_empty + kStagesB;     // local: a stage's scales landed
-  uint64_t* s_empty = s_full + kStagesS;     // local: this CTA's decoders read them
-  uint64_t* acc_full = s_empty + kStagesS;   // both [2]: accumulator complete
+  uint64_t* acc_full = b_empty + kStagesB;   // both [2]: accumulator complete
   uint64_t* acc_empty = acc_full + 2;        // leader [2]: both epilogues drained it
   uint64_t* mma_drain = acc_empty + 2;       // leader: all issued MMAs finished (abort path)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -282,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint64_t lim = p.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStagesP; ++i) {
+    for (int i = 0; i < kSlotsP; ++i) {
       mbar_init(&p_full[i], 1 + 32);  // the TMA producer's arrival (with its bytes) + the scale loader's lanes
       mbar_init(&p_empty[i], kDecThreads / 32);
     }
@@ -338,14 +340,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
       const int e = tt.x;
-      for (int s = 0; s < n_main; ++s) {
+      for (int s0 = 0; s0 < n_main; s0 += kGroup) {
+        const int nsub = min(kGroup, n_main - s0);
         if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_p;
         if (lane == 0) {
           uint64_t* bar = &p_full[ring.stage];
-          uint8_t* dst = sP + ring.stage * kPBytes;
           // every box is counted in full, also where it reaches past the
           // tensor (zero-filled rows of a half block)
-          mbar_expect_tx(bar, kPBytes);
+          mbar_expect_tx(bar, nsub * kPBytes);
+          for (int u = 0; u < nsub; ++u) {
+          const int s = s0 + u;
+          uint8_t* dst = sP + (ring.stage * kGroup + u) * kPBytes;
           if constexpr (MODE == kModeGateUp) {
             tma_load_3d(dst, &tq0, bar, s * (kBlockK / 2), fc, e);
             tma_load_3d(dst + kPBytes / 2, &tq1, bar, s * (kBlockK / 2), fc, e);
@@ -360,15 +365,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             else
               tma_load_3d(dst, &tq1, bar, fc / 2, k0 - p.stored_rows, e);
           }
+          }
         }
         __syncwarp();
-        ring.advance(kStagesP);
+        ring.advance(kSlotsP);
         ++issued;
       }
     }
     goto done;
   drain_p:
-    if (lane == 0) drain_ring(p_full, ring, issued, kStagesP);
+    if (lane == 0) drain_ring(p_full, ring, issued, kSlotsP);
     __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------- scale loader
@@ -376,11 +382,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
-      for (int s = 0; s < n_main; ++s) {
+      for (int s0 = 0; s0 < n_main; s0 += kGroup) {
+        const int nsub = min(kGroup, n_main - s0);
         if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
-        load_stage_scales<MODE>(p, tt.x, fc, s, lane, sS + ring.stage * kSBytes);
+        for (int u = 0; u < nsub; ++u)
+          load_stage_scales<MODE>(p, tt.x, fc, s0 + u, lane, sS + (ring.stage * kGroup + u) * kSBytes);
         cp_async_arrive_noinc(&p_full[ring.stage]);
-        ring.advance(kStagesS);
+        ring.advance(kSlotsP);
       }
     }
   drain_s:
@@ -653,7 +661,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int dt = threadIdx.x - kDecWarp0 * 32;
     // the leader's first decoder warp also waits for each group's B tiles
     const bool b_watch = cta == 0 && warp == kDecWarp0;
-    Ring rg, rp, rs, rbd;
+    Ring rg, rp, rbd;
     const uint32_t s_off = scale_off<MODE>(dt);
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
@@ -665,19 +673,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nb = min(kGroup, n_main - s);
         // decode the group into registers (needs only its packed and scale
         // stages), then wait for its A tiles to be free and store
-        Ring rp_[kGroup], rs_[kGroup];
         uint32_t w[kGroup][16];
+        if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
 #pragma unroll
         for (int b = 0; b < kGroup; ++b) {
-          rp_[b] = rp;
-          rs_[b] = rs;
           if (b < nb) {
-            if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
-            const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + rs.stage * kSBytes + s_off);
-            const uint4 q4 = packed_group<MODE>(sP + rp.stage * kPBytes, dt);
+            const int st = rp.stage * kGroup + b;
+            const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + st * kSBytes + s_off);
+            const uint4 q4 = packed_group<MODE>(sP + st * kPBytes, dt);
             decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
-            rp.advance(kStagesP);
-            rs.advance(kStagesS);
           }
         }
         // The packed and scale stages are released once every lane has used
@@ -690,11 +694,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int b = 0; b < kGroup; ++b)
           if (b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
         __syncwarp();
-        if (lane == 0) {
-          for (int b = 0; b < nb; ++b) {
-            mbar_arrive(&p_empty[rp_[b].stage]);
-          }
-        }
+        if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+        rp.advance(kSlotsP);
         if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
 #pragma unroll
         for (int b = 0; b < kGroup; ++b) {
