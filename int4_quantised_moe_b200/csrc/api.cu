@@ -352,7 +352,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   const int max_tiles = max_tok_tiles(maxR, E);
   {
     R4_PROF("gather_x", st);
-    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.xp), H, maxR, &hdr->status, 0, 0,
+    R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.inv), k, hdr, at<uint16_t>(ws, L.xp), H, qlen, &hdr->status, 0, 0,
                               st));
   }
   if (has_lora) {
@@ -532,7 +532,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   }
   {
     R4_PROF("gather_dy", st);
-    R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.perm), k, hdr, at<uint16_t>(ws, L.gp), H, maxR,
+    R4_TRY(launch_gather_rows(grad_out, at<int32_t>(ws, L.inv), k, hdr, at<uint16_t>(ws, L.gp), H, maxQ,
                               &hdr->status, 1, 1, st));
   }
   {

@@ -10,16 +10,18 @@ namespace {
 __device__ __forceinline__ bool bwd_enabled(const WsHeader* hdr) { return hdr->saved == 1u; }
 
 // ------------------------------------------------------------------ gather
-// One warp per permuted row: the source token is looked up once, then the
-// row is converted 8 elements per lane and step with 16-byte loads/stores.
+// One warp per token: each 16-byte piece of the token's row is loaded and
+// converted once and stored to every permuted row the token was routed to
+// (inv[t * top_k + s], -1 for an entry that routes nowhere), so the source
+// matrix is read once instead of once per routed copy.
 // scale_dy (grad_out): every value is multiplied by 2^s first, s from the
 // largest magnitude found by absmax_rows_kernel (exact: a power of two).
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ inv,
                                                           int top_k, WsHeader* hdr, uint4* __restrict__ dst,
                                                           int vecs_per_row, uint32_t* status, int need_saved,
                                                           int scale_dy) {
   if (need_saved && !bwd_enabled(hdr)) return;
-  const int64_t rows = hdr->routed;
+  const int64_t tokens = hdr->qlen;
   float sc = 1.0f;
   if (scale_dy) {
     const int e = dy_scale_exponent(hdr->dy_amax);
@@ -30,11 +32,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   bool overflow = false;
-  for (int64_t row = warp0; row < rows; row += nwarps) {
-    const int32_t t = perm[row] / top_k;
-    const uint4* s = src + (int64_t)t * vecs_per_row;
-    uint4* d = dst + row * vecs_per_row;
-#pragma unroll 4
+  for (int64_t t = warp0; t < tokens; t += nwarps) {
+    const uint4* s = src + t * vecs_per_row;
+    const int32_t* slots = inv + t * top_k;
+#pragma unroll 2
     for (int c = lane; c < vecs_per_row; c += 32) {
       const uint4 v = __ldg(s + c);
       const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -49,7 +50,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
         overflow |= (__hisinf(__low2half(h)) != 0 && isfinite(lo)) || (__hisinf(__high2half(h)) != 0 && isfinite(hi));
         out[j] = *reinterpret_cast<uint32_t*>(&h);
       }
-      d[c] = make_uint4(out[0], out[1], out[2], out[3]);
+      const uint4 o = make_uint4(out[0], out[1], out[2], out[3]);
+      for (int k = 0; k < top_k; ++k) {
+        const int32_t row = __ldg(slots + k);
+        if (row >= 0) dst[(int64_t)row * vecs_per_row + c] = o;
+      }
     }
   }
   if (overflow) raise_status(status, RAWINT4_DEV_FP16_OVERFLOW);
@@ -211,12 +216,12 @@ int grid_for(int64_t work, int threads) {
 
 }  // namespace
 
-cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, WsHeader* hdr,
-                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved, int scale_dy,
+cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* inv, int top_k, WsHeader* hdr,
+                               uint16_t* dst_f16, int H, int max_tokens, uint32_t* status, int need_saved, int scale_dy,
                                cudaStream_t stream) {
   const int vecs = H / 8;
-  gather_rows_kernel<<<grid_for((int64_t)max_rows * 32, 256), 256, 0, stream>>>(
-      reinterpret_cast<const uint4*>(src_bf16), perm, top_k, hdr, reinterpret_cast<uint4*>(dst_f16), vecs, status,
+  gather_rows_kernel<<<grid_for((int64_t)max_tokens * 32, 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src_bf16), inv, top_k, hdr, reinterpret_cast<uint4*>(dst_f16), vecs, status,
       need_saved, scale_dy);
   return cudaGetLastError();
 }

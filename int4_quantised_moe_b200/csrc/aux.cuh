@@ -3,12 +3,13 @@
 
 namespace r4 {
 
-// dst[p, :] = fp16(src[perm[p] / top_k, :]) for p < hdr->routed (bf16 src [Q, H]).
+// dst[inv[t * top_k + s], :] = fp16(src[t, :]) for t < hdr->qlen and every s with
+// inv[t * top_k + s] >= 0 (bf16 src [Q, H]): each permuted row receives its token's row.
 // need_saved: the kernel does nothing unless the header holds a pending saved forward (backward use).
 // scale_dy: grad_out; values are multiplied by 2^s (dy_scale_exponent of hdr->dy_amax) and s is
 // recorded in hdr->dy_exp.
-cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* perm, int top_k, WsHeader* hdr,
-                               uint16_t* dst_f16, int H, int max_rows, uint32_t* status, int need_saved, int scale_dy,
+cudaError_t launch_gather_rows(const uint16_t* src_bf16, const int32_t* inv, int top_k, WsHeader* hdr,
+                               uint16_t* dst_f16, int H, int max_tokens, uint32_t* status, int need_saved, int scale_dy,
                                cudaStream_t stream);
 
 // hdr->dy_amax = max(hdr->dy_amax, largest |v| of the first hdr->qlen rows of bf16 src [*, H]);
