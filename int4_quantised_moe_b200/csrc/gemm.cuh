@@ -62,12 +62,15 @@ __device__ __forceinline__ bool wait_lim(uint64_t* bar, uint32_t parity, volatil
   }
 }
 // The UMMA issuer's wait: never suspends (a suspended issuer resumes late and
-// the tensor pipe drains meanwhile); the bound is checked every 256 polls.
+// the tensor pipe drains meanwhile) but naps 32 ns between polls, which
+// leaves the issue slots of its scheduler to the decoder warps that share it;
+// the bound is checked every 256 polls.
 __device__ __forceinline__ bool wait_issuer(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
                                             uint64_t limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
+    __nanosleep(32);
     if (mbar_test_wait(bar, parity)) return true;
     if ((n & 255u) == 0) {
       if (*abort_flag) return false;
