@@ -475,20 +475,32 @@ __global__ void __launch_bounds__(256) lora_convert_kernel(LoraCvt j0, LoraCvt j
     const int vpr = cols / 8;
     const int64_t total = (int64_t)experts * rows_out * vpr;
     uint4* dst = reinterpret_cast<uint4*>(jb.dst);
-    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-      const int64_t row_g = idx / vpr;
-      const int v = (int)(idx - row_g * vpr);
-      const int e = (int)(row_g / rows_out);
-      const int row = (int)(row_g - (int64_t)e * rows_out);
-      const int blk = row / rp, j = row - blk * rp;
-      uint4 out = make_uint4(0u, 0u, 0u, 0u);
-      if (j < r) {
-        const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * cols;
-        const uint4 in = __ldg(reinterpret_cast<const uint4*>(src) + v);
-        out = make_uint4(bf16x2_to_h2(in.x), bf16x2_to_h2(in.y), bf16x2_to_h2(in.z), bf16x2_to_h2(in.w));
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    // four vectors per thread and pass, all loads issued before the stores
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total; base += 4 * step) {
+      uint4 out[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t idx = base + q * step;
+        out[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (idx < total) {
+          const int64_t row_g = idx / vpr;
+          const int v = (int)(idx - row_g * vpr);
+          const int e = (int)(row_g / rows_out);
+          const int row = (int)(row_g - (int64_t)e * rows_out);
+          const int blk = row / rp, j = row - blk * rp;
+          if (j < r) {
+            const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * cols;
+            const uint4 in = __ldg(reinterpret_cast<const uint4*>(src) + v);
+            out[q] = make_uint4(bf16x2_to_h2(in.x), bf16x2_to_h2(in.y), bf16x2_to_h2(in.z), bf16x2_to_h2(in.w));
+          }
+        }
       }
-      dst[idx] = out;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t idx = base + q * step;
+        if (idx < total) dst[idx] = out[q];
+      }
     }
   } else {
     __shared__ float tile[64][65];  // 64 source rows x up to 64 ranks (+1: no bank conflicts)
@@ -535,7 +547,7 @@ cudaError_t launch_lora_convert(const LoraCvt* jobs, int njobs, int experts, cud
   LoraCvt z{};
   LoraCvt j[3] = {njobs > 0 ? jobs[0] : z, njobs > 1 ? jobs[1] : z, njobs > 2 ? jobs[2] : z};
   if (njobs <= 0) return cudaSuccess;
-  dim3 grid(148 * 4, njobs > 3 ? 3 : njobs, 1);
+  dim3 grid(148 * 8, njobs > 3 ? 3 : njobs, 1);
   lora_convert_kernel<<<grid, 256, 0, stream>>>(j[0], j[1], j[2], experts);
   return cudaGetLastError();
 }
