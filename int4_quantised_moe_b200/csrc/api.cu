@@ -376,7 +376,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   sp.scale = scaling;
   sp.w_perm = at<float>(ws, L.w_perm);
   SkMaps sm;
-  const int rows_grid = grid_for_tiles(sms, 2 * max_tiles, 1);
+  const int rows_grid = grid_for_tiles(kSkCtasPerSm * sms, 2 * max_tiles, 1);
 
   // xa = c * X_perm [A_g; A_u]^T: gate in columns [0, r), up in [rp, rp + r);
   // both rank blocks in one 64-wide segment up to rank 32, one segment each
@@ -553,7 +553,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   sp.scale = scaling;
   sp.w_perm = at<float>(ws, L.w_perm);
   SkMaps sm;
-  const int rows_grid = grid_for_tiles(sms, 2 * max_tiles, 1);
+  const int rows_grid = grid_for_tiles(kSkCtasPerSm * sms, 2 * max_tiles, 1);
 
   // gd = c * g B_d and gdw = w * gd
   if (!map_act(&sm.a[0], at<uint16_t>(ws, L.gp), L.rows, H, 128) ||
@@ -718,7 +718,7 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     int items = 0;
     for (int j = 0; j < gq.njobs; ++j) items += E * gq.job[j].nfb;
     R4_PROF("lora_grads", st);
-    R4_TRY(launch_skinny(kSkGrads, gq, gm, grid_for_tiles(sms, items, 1), st));
+    R4_TRY(launch_skinny(kSkGrads, gq, gm, grid_for_tiles(kSkCtasPerSm * sms, items, 1), st));
   }
   {
     R4_PROF("header_end", st);

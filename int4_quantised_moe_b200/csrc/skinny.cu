@@ -1,7 +1,10 @@
 // Rank-r LoRA products on the tensor cores (see skinny.cuh).
 //
-// One persistent CTA per SM; warp 0 issues TMA loads of both operands into a
-// ring of stages, warp 1 issues the UMMAs into a double-buffered TMEM
+// Two persistent CTAs per SM (about 105 KB of shared memory and 256 TMEM
+// columns each): the UMMAs of these products are small (M = 128, N = 64), so
+// one issuer leaves the tensor pipe mostly idle and a second CTA's stream
+// fills it. In each CTA warp 0 issues TMA loads of both operands into a ring
+// of stages, warp 1 issues the UMMAs into a double-buffered TMEM
 // accumulator, warps 2-5 run the epilogue. No thread ever writes an operand
 // tile except to clear the rows past an expert's last row in the gradient
 // mode (constant stores, fenced for the async proxy before the MMA reads).
@@ -20,7 +23,7 @@ constexpr int kSkOffMisc = kSkOffBar + kSkNumBars * 8;
 constexpr int kSkOffStage = (kSkOffMisc + 16 + 15) / 16 * 16;
 constexpr int kSkStageFloats = 2 * 32 * 128;
 constexpr int kSkSmem = kSkOffStage + kSkStageFloats * 4 + 1024;
-static_assert(kSkSmem <= 232448, "shared memory budget");
+static_assert(2 * (kSkSmem + 1024) <= 233472, "two CTAs per SM (228 KB per SM, 1 KB reserved per CTA)");
 constexpr uint32_t kSkTmemCols = 256;
 
 struct GradItem {
@@ -448,6 +451,9 @@ cudaError_t launch_sk(const SkParams& p, const SkMaps& m, int grid, cudaStream_t
   int dev = 0;
   if (!device_flag_test(attr, &dev)) {
     cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmem);
+    if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so that two CTAs fit on an SM
+    e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     device_flag_set(attr, dev);
   }

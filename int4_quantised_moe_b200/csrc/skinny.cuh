@@ -27,7 +27,8 @@ namespace r4 {
 enum SkMode : int { kSkRows = 0, kSkGrads = 1 };
 
 constexpr int kSkThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kSkStages = 6;
+constexpr int kSkStages = 3;
+constexpr int kSkCtasPerSm = 2;   // resident skinny CTAs per SM (grid = kSkCtasPerSm x SMs)
 
 // How a gradient job maps D columns/rows to the output buffers.
 enum SkSplit : int {
