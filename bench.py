@@ -45,7 +45,8 @@ UNIT = "routed tokens/s"
 def gemm_source_hash():
     import hashlib
     d = os.path.join(ROOT, "int4_quantised_moe_b200", "csrc")
-    src = b"".join(open(os.path.join(d, f), "rb").read() for f in ("gemm_tm.cu", "gemm_pair.cu", "gemm.cuh", "common.cuh"))
+    src = b"".join(open(os.path.join(d, f), "rb").read() for f in ("gemm_tm.cu", "gemm_pair.cu", "gemm_tm_narrow.cu", "gemm_pair_narrow.cu",
+                                                                  "gemm.cuh", "common.cuh", "route.cuh"))
     return hashlib.sha256(src).hexdigest()[:16]
 
 

@@ -15,7 +15,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librawint4_moe.so")
-SOURCES = ["api.cu", "gemm_pair.cu", "gemm_tm.cu", "skinny.cu", "route.cu", "aux.cu", "prof.cu", "noalloc.cu", "router.cu"]
+SOURCES = ["api.cu", "gemm_pair.cu", "gemm_tm.cu", "gemm_pair_narrow.cu", "gemm_tm_narrow.cu", "skinny.cu", "route.cu",
+           "aux.cu", "prof.cu", "noalloc.cu", "router.cu"]
 HEADERS = ["common.cuh", "gemm.cuh", "skinny.cuh", "route.cuh", "aux.cuh", "prof.cuh", "router.cuh"]
 
 NVCC_FLAGS = [

@@ -37,7 +37,7 @@ Layout make_layout(const rawint4_moe_cfg& c) {
   // capacity rounded to whole 256-row tiles plus one spare tile: TMA boxes of
   // the last token tile and zero-padded LoRA side rows stay inside the buffers
   L.rows = (R + kTileRows - 1) / kTileRows * kTileRows + kTileRows;
-  L.max_tiles = max_tok_tiles((int32_t)R, c.experts);
+  L.max_tiles = max_tok_tiles((int32_t)R, c.experts, kTileRowsNarrow);  // either tile configuration
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -234,33 +234,47 @@ int grid_for_tiles(int sms, int max_tiles, int rowblk) {
 
 // CTA pairs for a pair-kernel launch: all that fit at once, or fewer for a small
 // problem (work items = token tiles x feature blocks).
-int gemm_clusters(int mode, int sms, int max_tiles, int rowblk) {
-  static std::atomic<int> cached[64][4];  // per device and mode; 0 = not queried yet
+int gemm_clusters(int mode, bool narrow, int sms, int max_tiles, int rowblk) {
+  static std::atomic<int> cached[64][2][4];  // per device, configuration and mode; 0 = not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  int fit = cached[dev][mode].load();
+  int fit = cached[dev][narrow][mode].load();
   if (fit <= 0) {
-    const int n = gemm_pair_max_clusters(mode);
+    const int n = narrow ? gemm_pair_max_clusters_narrow(mode) : gemm_pair_max_clusters(mode);
     fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
-    cached[dev][mode].store(fit);
+    cached[dev][narrow][mode].store(fit);
   }
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
 }
 
 // CTA pairs for a launch of the tensor-memory GEMM (gemm_tm.cu).
-int tm_clusters(int mode, int fmt, int sms, int max_tiles, int rowblk) {
-  static std::atomic<int> cached[64][2][4];  // per device, format and mode; 0 = not queried yet
+int tm_clusters(int mode, int fmt, bool narrow, int sms, int max_tiles, int rowblk) {
+  static std::atomic<int> cached[64][2][2][4];  // per device, configuration, format and mode; 0 = not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  int fit = cached[dev][fmt][mode].load();
+  int fit = cached[dev][narrow][fmt][mode].load();
   if (fit <= 0) {
-    const int n = gemm_tm_max_clusters(mode, fmt);
+    const int n = narrow ? gemm_tm_max_clusters_narrow(mode, fmt) : gemm_tm_max_clusters(mode, fmt);
     fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);
-    cached[dev][fmt][mode].store(fit);
+    cached[dev][narrow][fmt][mode].store(fit);
   }
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
+}
+
+// Token-tile configuration of a call: narrow (tiles of at most
+// kTileRowsNarrow rows, the GEMMs' narrow configurations) for a RAWINT4 base
+// whose workspace averages at most kTileRowsNarrow / 2 routed rows per expert
+// (max_tokens x top_k / experts), wide otherwise. The choice depends on the
+// configuration only, so a backward always matches its forward. The
+// environment may force it (RAWINT4_TILES=narrow or wide) for testing.
+bool narrow_tiles(const rawint4_moe_cfg& c) {
+  if (c.weight_format != RAWINT4_FORMAT_RAWINT4) return false;
+  const char* e = getenv("RAWINT4_TILES");
+  if (e && strcmp(e, "narrow") == 0) return true;
+  if (e && strcmp(e, "wide") == 0) return false;
+  return 2LL * c.max_tokens * c.top_k <= (long long)kTileRowsNarrow * c.experts;
 }
 
 // Which kernel runs the transpose-free backward GEMMs (down^T, gate/up^T):
@@ -336,6 +350,7 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   const float scaling = c.alpha / (float)r;
   void* ws = workspace;
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  const bool nar = narrow_tiles(c);  // token-tile configuration of this layer
 
   {
     R4_PROF("header_fwd", st);
@@ -345,11 +360,11 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     R4_PROF("route", st);
     R4_TRY(launch_route(expert_ids, route_weights, qlen, k, E, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                         at<int32_t>(ws, L.inv), at<float>(ws, L.w_perm), at<int4>(ws, L.tiles),
-                        at<int32_t>(ws, L.hist), hdr, st));
+                        at<int32_t>(ws, L.hist), hdr, st, nar ? kTileRowsNarrow : kTileRows));
   }
   if (qlen == 0) return RAWINT4_OK;
   const int maxR = qlen * k;
-  const int max_tiles = max_tok_tiles(maxR, E);
+  const int max_tiles = max_tok_tiles(maxR, E, nar ? kTileRowsNarrow : kTileRows);
   {
     R4_PROF("gather_x", st);
     R4_TRY(launch_gather_rows(x, at<int32_t>(ws, L.inv), k, hdr, at<uint16_t>(ws, L.xp), H, qlen, &hdr->status, 0, 0,
@@ -446,7 +461,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = I;
   {
     R4_PROF("gemm_gate_up", st);
-    R4_TRY(launch_gemm_tm(kModeGateUp, fmt, gp, mp, tm_clusters(kModeGateUp, fmt, sms, max_tiles, gp.n_rowblk), st));
+    const int ncl = tm_clusters(kModeGateUp, fmt, nar, sms, max_tiles, gp.n_rowblk);
+    R4_TRY(nar ? launch_gemm_tm_narrow(kModeGateUp, fmt, gp, mp, ncl, st) : launch_gemm_tm(kModeGateUp, fmt, gp, mp, ncl, st));
   }
 
   // ha = c * h A_d^T and hw = w * ha
@@ -486,7 +502,8 @@ int rawint4_moe_lora_fwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   gp.ld_out = H;
   {
     R4_PROF("gemm_down", st);
-    R4_TRY(launch_gemm_tm(kModeDown, fmt, gp, mp, tm_clusters(kModeDown, fmt, sms, max_tiles, gp.n_rowblk), st));
+    const int ncl = tm_clusters(kModeDown, fmt, nar, sms, max_tiles, gp.n_rowblk);
+    R4_TRY(nar ? launch_gemm_tm_narrow(kModeDown, fmt, gp, mp, ncl, st) : launch_gemm_tm(kModeDown, fmt, gp, mp, ncl, st));
   }
   {
     R4_PROF("combine_out", st);
@@ -518,7 +535,8 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
   const int maxQ = c.max_tokens;
   const int maxR = maxQ * k;
-  const int max_tiles = max_tok_tiles(maxR, E);
+  const bool nar = narrow_tiles(c);  // the forward's tile configuration
+  const int max_tiles = max_tok_tiles(maxR, E, nar ? kTileRowsNarrow : kTileRows);
 
   {
     R4_PROF("header_bwd", st);
@@ -611,9 +629,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_down_t", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeDownT, fmt, gp, mp, tm_clusters(kModeDownT, fmt, sms, max_tiles, gp.n_rowblk), st));
-    else
-      R4_TRY(launch_gemm_pair(kModeDownT, gp, mp, gemm_clusters(kModeDownT, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeDownT, fmt, gp, mp, tm_clusters(kModeDownT, fmt, false, sms, max_tiles, gp.n_rowblk), st));
+    else {
+      const int ncl = gemm_clusters(kModeDownT, nar, sms, max_tiles, gp.n_rowblk);
+      R4_TRY(nar ? launch_gemm_pair_narrow(kModeDownT, gp, mp, ncl, st) : launch_gemm_pair(kModeDownT, gp, mp, ncl, st));
+    }
   }
 
   // gb = c * [dG B_g, dU B_u]: gate in columns [0, r), up in [rp, rp + r)
@@ -659,9 +679,11 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
   {
     R4_PROF("gemm_gate_up_t", st);
     if (tm)
-      R4_TRY(launch_gemm_tm(kModeGateUpT, fmt, gp, mp, tm_clusters(kModeGateUpT, fmt, sms, max_tiles, gp.n_rowblk), st));
-    else
-      R4_TRY(launch_gemm_pair(kModeGateUpT, gp, mp, gemm_clusters(kModeGateUpT, sms, max_tiles, gp.n_rowblk), st));
+      R4_TRY(launch_gemm_tm(kModeGateUpT, fmt, gp, mp, tm_clusters(kModeGateUpT, fmt, false, sms, max_tiles, gp.n_rowblk), st));
+    else {
+      const int ncl = gemm_clusters(kModeGateUpT, nar, sms, max_tiles, gp.n_rowblk);
+      R4_TRY(nar ? launch_gemm_pair_narrow(kModeGateUpT, gp, mp, ncl, st) : launch_gemm_pair(kModeGateUpT, gp, mp, ncl, st));
+    }
   }
   {
     R4_PROF("combine_dx", st);

@@ -171,5 +171,14 @@ int gemm_pair_max_clusters(int mode);
 cudaError_t launch_gemm_tm(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
                            cudaStream_t stream);
 int gemm_tm_max_clusters(int mode, int fmt);
+// The narrow configurations (token tiles of at most kTileRowsNarrow rows,
+// hand-off groups of four stages): gemm_tm_narrow.cu for the RAWINT4 forward
+// modes, gemm_pair_narrow.cu for the transpose-free backward modes.
+cudaError_t launch_gemm_tm_narrow(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+                                  cudaStream_t stream);
+int gemm_tm_max_clusters_narrow(int mode, int fmt);
+cudaError_t launch_gemm_pair_narrow(int mode, const GemmParams& p, const GemmMaps& maps, int clusters,
+                                    cudaStream_t stream);
+int gemm_pair_max_clusters_narrow(int mode);
 
 }  // namespace r4

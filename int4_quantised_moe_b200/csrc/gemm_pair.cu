@@ -42,19 +42,38 @@
 // (transpose-free dX, rawint4_sft_reference.py transpose_free_rawint4_dx):
 // the decoders write the same packed bytes into an MN-major A tile, so no
 // transposed or dense copy of any base weight ever exists.
+//
+// Two configurations are built from this file: the wide one (this
+// translation unit: token tiles of up to kTileRows rows, hand-off groups of
+// two stages) and the narrow one (gemm_pair_narrow.cu, R4_PAIR_NARROW = 1:
+// tiles of at most kTileRowsNarrow rows, whose small activation tiles leave
+// shared memory for eight A tiles in groups of four stages).
 #include "gemm.cuh"
 #include "route.cuh"
 
+#ifndef R4_PAIR_NARROW
+#define R4_PAIR_NARROW 0
+#endif
+#if R4_PAIR_NARROW
+#define R4_PAIR_NS pairk_narrow
+#define R4_PAIR_LAUNCH launch_gemm_pair_narrow
+#define R4_PAIR_MAXCL gemm_pair_max_clusters_narrow
+#else
+#define R4_PAIR_NS pairk
+#define R4_PAIR_LAUNCH launch_gemm_pair
+#define R4_PAIR_MAXCL gemm_pair_max_clusters
+#endif
+
 namespace r4 {
 
-namespace pairk {
+namespace R4_PAIR_NS {
 
 constexpr int kRowsM = 128;        // weight rows per CTA (256 per CTA pair)
-constexpr int kStagesA = 4;        // decoded FP16 A tiles (16 KB each): two groups
-constexpr int kGroup = 2;          // stages per hand-off (issuer wait, decoder arrival)
+constexpr int kStagesA = R4_PAIR_NARROW ? 8 : 4;  // decoded FP16 A tiles (16 KB each): two groups
+constexpr int kGroup = R4_PAIR_NARROW ? 4 : 2;    // stages per hand-off (issuer wait, decoder arrival)
 constexpr int kAGroups = kStagesA / kGroup;
 constexpr int kStagesB = 6;        // TMA-loaded B tiles (this CTA's half of up to kTileRows tokens)
-constexpr int kStagesP = 16;       // TMA-loaded packed int4 tiles (4 KB each)
+constexpr int kStagesP = R4_PAIR_NARROW ? 12 : 16;  // TMA-loaded packed int4 tiles (4 KB each)
 constexpr int kStagesS = kStagesP;  // group scales of one stage (512 B each), one per packed stage
 // Packed stages and their scales are filled and released in slots of kGroup
 // consecutive stages (a hand-off group): one barrier per slot.
@@ -65,7 +84,8 @@ constexpr int kDecWarp0 = 8;       // warps 8..15: decoders
 constexpr int kDecThreads = 256;
 
 constexpr int kABytes = kRowsM * kBlockK * 2;  // 16 KB
-constexpr int kBBytes = (kTileRows / 2) * kBlockK * 2;  // 12 KB: this CTA's half of <= kTileRows tokens
+constexpr int kTileMax = R4_PAIR_NARROW ? kTileRowsNarrow : kTileRows;  // rows of a token tile
+constexpr int kBBytes = (kTileMax / 2) * kBlockK * 2;  // this CTA's half of <= kTileMax tokens (12 KB wide)
 constexpr int kPBytes = kRowsM * kBlockK / 2;  // 4 KB
 constexpr int kSBytes = 512;                   // 256 bf16 group scales of one stage
 constexpr int kOffA = 0;
@@ -673,38 +693,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nb = min(kGroup, n_main - s);
         // decode the group into registers (needs only its packed and scale
         // stages), then wait for its A tiles to be free and store
-        uint32_t w[kGroup][16];
         if (!wait_warp(&p_full[rp.stage], rp.phase, abort_flag, status, lim)) goto done;
+        // two stages at a time (decoded words of more would not stay in
+        // registers); the group's A tiles are waited for once
+        for (int h = 0; h < nb; h += 2) {
+          uint32_t w[2][16];
 #pragma unroll
-        for (int b = 0; b < kGroup; ++b) {
-          if (b < nb) {
-            const int st = rp.stage * kGroup + b;
-            const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + st * kSBytes + s_off);
-            const uint4 q4 = packed_group<MODE>(sP + st * kPBytes, dt);
-            decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
+          for (int b = 0; b < 2; ++b) {
+            if (h + b < nb) {
+              const int st = rp.stage * kGroup + h + b;
+              const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + st * kSBytes + s_off);
+              const uint4 q4 = packed_group<MODE>(sP + st * kPBytes, dt);
+              decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
+            }
           }
-        }
-        // The packed and scale stages are released once every lane has used
-        // the values it loaded from them: the empty asm makes the decoded
-        // words (which depend on every loaded byte and on the scale) inputs,
-        // so the loads have returned before the release. A release right after
-        // the loads were issued could let the refill of the stage land under
-        // loads still in flight.
+          if (h + 2 >= nb) {
+            // The packed slot and its scales are released once every lane has
+            // used the values it loaded from them: the empty asm makes the
+            // decoded words (which depend on every loaded byte and on the
+            // scale) inputs, so the loads have returned before the release. A
+            // release right after the loads were issued could let the refill
+            // of the slot land under loads still in flight.
 #pragma unroll
-        for (int b = 0; b < kGroup; ++b)
-          if (b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
-        rp.advance(kSlotsP);
-        if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
+            for (int b = 0; b < 2; ++b)
+              if (h + b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+            rp.advance(kSlotsP);
+          }
+          if (h == 0)
+            if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
 #pragma unroll
-        for (int b = 0; b < kGroup; ++b) {
-          if (b < nb) {
-            uint8_t* A = sA + (kGroup * rg.stage + b) * kABytes;
+          for (int b = 0; b < 2; ++b) {
+            if (h + b < nb) {
+              uint8_t* A = sA + (kGroup * rg.stage + h + b) * kABytes;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
-                  make_uint4(w[b][4 * j], w[b][4 * j + 1], w[b][4 * j + 2], w[b][4 * j + 3]);
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(A + a_chunk_off<MODE>(dt, j)) =
+                    make_uint4(w[b][4 * j], w[b][4 * j + 1], w[b][4 * j + 2], w[b][4 * j + 3]);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -795,20 +822,20 @@ int max_clusters_mode() {
   return n;
 }
 
-}  // namespace pairk
+}  // namespace R4_PAIR_NS
 
 // The library runs the two transpose-free backward GEMMs (MN-major decoded
 // A tiles in shared memory) on this kernel; the kernel itself is written for
 // every mode.
-cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
-  if (mode == kModeDownT) return pairk::launch_mode<kModeDownT>(p, maps, clusters, stream);
-  if (mode == kModeGateUpT) return pairk::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
+cudaError_t R4_PAIR_LAUNCH(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
+  if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT>(p, maps, clusters, stream);
+  if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
   return cudaErrorInvalidValue;
 }
 
-int gemm_pair_max_clusters(int mode) {
-  if (mode == kModeDownT) return pairk::max_clusters_mode<kModeDownT>();
-  if (mode == kModeGateUpT) return pairk::max_clusters_mode<kModeGateUpT>();
+int R4_PAIR_MAXCL(int mode) {
+  if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT>();
+  if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT>();
   return 0;
 }
 

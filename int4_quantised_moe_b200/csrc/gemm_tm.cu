@@ -54,14 +54,36 @@
 // reduction stage in the same accumulators: its A operand is the LoRA tensor
 // of the expert (loaded into registers at the start of the item and stored by
 // the decoders), its B operand the precomputed c-scaled rank-r side matrix.
+//
+// Two configurations are built from this file. The wide one (this
+// translation unit) holds token tiles of up to kTmAccCols rows with groups of
+// two stages; the narrow one (gemm_tm_narrow.cu, R4_TM_NARROW = 1), for
+// layers with few rows per expert, holds tiles of at most kTileRowsNarrow
+// rows, so tensor memory has room for eight A stages and the hand-off groups
+// are four stages long (half the synchronisations per weight byte).
 #include "gemm.cuh"
+#include "route.cuh"
+
+#ifndef R4_TM_NARROW
+#define R4_TM_NARROW 0
+#endif
+#if R4_TM_NARROW
+#define R4_TM_NS tmk_narrow
+#define R4_TM_LAUNCH launch_gemm_tm_narrow
+#define R4_TM_MAXCL gemm_tm_max_clusters_narrow
+#else
+#define R4_TM_NS tmk
+#define R4_TM_LAUNCH launch_gemm_tm
+#define R4_TM_MAXCL gemm_tm_max_clusters
+#endif
 
 namespace r4 {
 
-namespace tmk {
+namespace R4_TM_NS {
 
-constexpr int kAStages = 4;                       // A stages in tensor memory (32 columns each)
-constexpr uint32_t kACol0 = 2 * kTmAccCols;       // first A column
+constexpr int kAccCols = R4_TM_NARROW ? kTileRowsNarrow : kTmAccCols;  // columns of one accumulator
+constexpr int kAStages = R4_TM_NARROW ? 8 : 4;    // A stages in tensor memory (32 columns each)
+constexpr uint32_t kACol0 = 2 * kAccCols;         // first A column
 static_assert(kACol0 + 32 * kAStages <= 512, "tensor memory columns");
 constexpr int kStagesB = 10;                      // TMA-loaded B half tiles
 // Packed weights and their scales arrive in slots of several reduction
@@ -83,11 +105,11 @@ constexpr int kThreads = 512;                     // 16 warps
 constexpr int kEpiWarp0 = 4;                      // warps 4..7: epilogue
 constexpr int kDecWarp0 = 8;                      // warps 8..15: decoders
 constexpr int kDecWarps = 8;
-constexpr int kGroup = 2;                         // stages per hand-off (issuer wait, decoder arrival)
+constexpr int kGroup = R4_TM_NARROW ? 4 : 2;      // stages per hand-off (issuer wait, decoder arrival)
 constexpr int kAGroups = kAStages / kGroup;       // groups of A stages in tensor memory
 static_assert(kAGroups >= 2, "the MMA consumes one group while the next is decoded");
 
-constexpr int kBBytes = (kTmAccCols / 2) * kBlockK * 2;  // this CTA's half of <= kTmAccCols tokens
+constexpr int kBBytes = (kAccCols / 2) * kBlockK * 2;    // this CTA's half of <= kAccCols tokens
 template <int MODE>
 constexpr int kPBytes = kPSub<MODE> * 4096;              // one packed slot (4 KB per stage)
 template <int MODE>
@@ -625,7 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           {
-            const uint32_t d_tmem = tmem + (uint32_t)(ab * kTmAccCols);
+            const uint32_t d_tmem = tmem + (uint32_t)(ab * kAccCols);
             uint32_t acc = 0u;  // the item's first UMMA overwrites the accumulator
             // the item's stages: slot-rotated main stages in groups within each
             // slot, then the LoRA stage as a group of its own
@@ -640,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 for (int b = 0; b < nb; ++b) {
-                  const uint32_t a_tm = a_col0 + (uint32_t)(64 * rg.stage + 32 * b);
+                  const uint32_t a_tm = a_col0 + (uint32_t)(32 * (kGroup * rg.stage + b));
                   const uint64_t bd = bdesc0 + (uint64_t)((rbr.stage * kBBytes) >> 4);
                   if (!lora) {
 #pragma unroll
@@ -695,7 +717,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool ok = wait_warp(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status, lim);
       if (!named_bar_and(3, 128, ok)) goto done;
       tc_fence_after();
-      const uint32_t d_tmem = tmem + lane_base + (uint32_t)(ab * kTmAccCols);
+      const uint32_t d_tmem = tmem + lane_base + (uint32_t)(ab * kAccCols);
       for (int c0 = 0; c0 < n_rows; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(d_tmem + (uint32_t)c0, v);
@@ -915,25 +937,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // release of the A stages to their next fill
         for (int u = 0; u < nsub; u += kGroup) {
           const int nb = min(kGroup, nsub - u);
-          uint32_t w[kGroup][16];
+          // two stages at a time (decoded words of more would not stay in
+          // registers); the group's A stages are waited for once
+          for (int h = 0; h < nb; h += 2) {
+            uint32_t w[2][16];
 #pragma unroll
-          for (int b = 0; b < kGroup; ++b)
-            if (b < nb) decode_stage(rs, rp, u + b, tab + 16 * b, w[b]);
-          if (u + kGroup >= nsub) {
-            // the slot's last group decoded: release the packed and scale
-            // slot once every lane has used the values it loaded (the empty
-            // asm makes the decoded words, which depend on every loaded byte
-            // and scale, inputs, so the loads have returned)
+            for (int b = 0; b < 2; ++b)
+              if (h + b < nb) decode_stage(rs, rp, u + h + b, tab + 16 * b, w[b]);
+            if (h + 2 >= nb && u + kGroup >= nsub) {
+              // the slot's last stages decoded: release the packed and scale
+              // slot once every lane has used the values it loaded (the empty
+              // asm makes the decoded words, which depend on every loaded byte
+              // and scale, inputs, so the loads have returned)
 #pragma unroll
-            for (int b = 0; b < kGroup; ++b)
-              if (b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+              for (int b = 0; b < 2; ++b)
+                if (h + b < nb) asm volatile("" ::"r"(w[b][0]), "r"(w[b][15]) : "memory");
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&p_empty[rp.stage]);
+            }
+            if (h == 0)
+              if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              if (h + b < nb)
+                tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * (kGroup * rg.stage + h + b) + 16 * g), w[b]);
           }
-          if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
-#pragma unroll
-          for (int b = 0; b < kGroup; ++b)
-            if (b < nb) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 32 * b + 16 * g), w[b]);
           tmem_wait_st();
           tc_fence_before();
           if (b_watch) {
@@ -959,8 +987,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           lora_values<MODE>(p, e, fc, m, g, kBlockK, lora_w1);
       }
       if (!wait_warp(&a_empty[rg.stage], rg.phase ^ 1u, abort_flag, status, lim)) goto done;
-      tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 16 * g), lora_w);
-      if (n_lora > 1) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(64 * rg.stage + 32 + 16 * g), lora_w1);
+      tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * kGroup * rg.stage + 16 * g), lora_w);
+      if (n_lora > 1) tmem_st16(tmem + lane_base + kACol0 + (uint32_t)(32 * kGroup * rg.stage + 32 + 16 * g), lora_w1);
       tmem_wait_st();
       tc_fence_before();
       if (b_watch) {
@@ -1022,35 +1050,39 @@ int max_clusters_mode() {
   return n;
 }
 
-}  // namespace tmk
+}  // namespace R4_TM_NS
 
-cudaError_t launch_gemm_tm(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+cudaError_t R4_TM_LAUNCH(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
                            cudaStream_t stream) {
-  constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
+  [[maybe_unused]] constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
   switch (mode * 2 + (fmt == X ? 1 : 0)) {
-    case kModeGateUp * 2: return tmk::launch_mode<kModeGateUp, R>(p, maps, clusters, stream);
-    case kModeGateUp * 2 + 1: return tmk::launch_mode<kModeGateUp, X>(p, maps, clusters, stream);
-    case kModeDown * 2: return tmk::launch_mode<kModeDown, R>(p, maps, clusters, stream);
-    case kModeDown * 2 + 1: return tmk::launch_mode<kModeDown, X>(p, maps, clusters, stream);
-    case kModeDownT * 2: return tmk::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
-    case kModeDownT * 2 + 1: return tmk::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
-    case kModeGateUpT * 2: return tmk::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
-    case kModeGateUpT * 2 + 1: return tmk::launch_mode<kModeGateUpT, X>(p, maps, clusters, stream);
+    case kModeGateUp * 2: return R4_TM_NS::launch_mode<kModeGateUp, R>(p, maps, clusters, stream);
+    case kModeDown * 2: return R4_TM_NS::launch_mode<kModeDown, R>(p, maps, clusters, stream);
+#if !R4_TM_NARROW  // the narrow configuration serves the RAWINT4 forward only
+    case kModeGateUp * 2 + 1: return R4_TM_NS::launch_mode<kModeGateUp, X>(p, maps, clusters, stream);
+    case kModeDown * 2 + 1: return R4_TM_NS::launch_mode<kModeDown, X>(p, maps, clusters, stream);
+    case kModeDownT * 2: return R4_TM_NS::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
+    case kModeDownT * 2 + 1: return R4_TM_NS::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
+    case kModeGateUpT * 2: return R4_TM_NS::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
+    case kModeGateUpT * 2 + 1: return R4_TM_NS::launch_mode<kModeGateUpT, X>(p, maps, clusters, stream);
+#endif
     default: return cudaErrorInvalidValue;
   }
 }
 
-int gemm_tm_max_clusters(int mode, int fmt) {
-  constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
+int R4_TM_MAXCL(int mode, int fmt) {
+  [[maybe_unused]] constexpr int R = RAWINT4_FORMAT_RAWINT4, X = RAWINT4_FORMAT_MXFP4;
   switch (mode * 2 + (fmt == X ? 1 : 0)) {
-    case kModeGateUp * 2: return tmk::max_clusters_mode<kModeGateUp, R>();
-    case kModeGateUp * 2 + 1: return tmk::max_clusters_mode<kModeGateUp, X>();
-    case kModeDown * 2: return tmk::max_clusters_mode<kModeDown, R>();
-    case kModeDown * 2 + 1: return tmk::max_clusters_mode<kModeDown, X>();
-    case kModeDownT * 2: return tmk::max_clusters_mode<kModeDownT, R>();
-    case kModeDownT * 2 + 1: return tmk::max_clusters_mode<kModeDownT, X>();
-    case kModeGateUpT * 2: return tmk::max_clusters_mode<kModeGateUpT, R>();
-    case kModeGateUpT * 2 + 1: return tmk::max_clusters_mode<kModeGateUpT, X>();
+    case kModeGateUp * 2: return R4_TM_NS::max_clusters_mode<kModeGateUp, R>();
+    case kModeDown * 2: return R4_TM_NS::max_clusters_mode<kModeDown, R>();
+#if !R4_TM_NARROW  // the narrow configuration serves the RAWINT4 forward only
+    case kModeGateUp * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeGateUp, X>();
+    case kModeDown * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeDown, X>();
+    case kModeDownT * 2: return R4_TM_NS::max_clusters_mode<kModeDownT, R>();
+    case kModeDownT * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeDownT, X>();
+    case kModeGateUpT * 2: return R4_TM_NS::max_clusters_mode<kModeGateUpT, R>();
+    case kModeGateUpT * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeGateUpT, X>();
+#endif
     default: return 0;
   }
 }

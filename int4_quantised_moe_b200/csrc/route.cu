@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kRouteChunk) route_count_kernel(const int64_t*
 // per-(block, expert) scatter bases, and the token-tile list.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ block_hist, int32_t nblocks, int32_t experts,
                                                           int32_t* __restrict__ offsets, int4* __restrict__ tok_tiles,
-                                                          WsHeader* hdr, int32_t qlen) {
+                                                          WsHeader* hdr, int32_t qlen, int32_t tile_rows) {
   extern __shared__ int32_t sm[];
   int32_t* total = sm;                 // [experts]
   int32_t* ntile = sm + experts;       // [experts]
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ 
     total[e] = run;
     int32_t nt = 0;
     if (run > 0) {
-      const int32_t per = (run + kTileRows - 1) / kTileRows;
+      const int32_t per = (run + tile_rows - 1) / tile_rows;
       int32_t sz = (run + per - 1) / per;
       sz = (sz + 15) / 16 * 16;
       nt = (run + sz - 1) / sz;
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ 
       for (int e = e0; e < e1; ++e) {
         const int32_t run = total[e];
         if (run > 0) {
-          const int32_t per = (run + kTileRows - 1) / kTileRows;
+          const int32_t per = (run + tile_rows - 1) / tile_rows;
           int32_t sz = (run + per - 1) / per;
           sz = (sz + 15) / 16 * 16;
           for (int i = 0; i < ntile[e]; ++i) {
@@ -173,7 +173,7 @@ size_t route_scratch_bytes(int32_t routed_slots, int32_t experts) {
 
 cudaError_t launch_route(const int64_t* ids, const float* rw, int32_t qlen, int32_t top_k, int32_t experts,
                          int32_t* offsets, int32_t* perm, int32_t* inv, float* w_perm, int4* tok_tiles,
-                         int32_t* block_hist, WsHeader* hdr, cudaStream_t stream) {
+                         int32_t* block_hist, WsHeader* hdr, cudaStream_t stream, int32_t tile_rows) {
   const int32_t slots = qlen * top_k;
   const int32_t nblocks = (slots + kRouteChunk - 1) / kRouteChunk;
   uint32_t* status = hdr ? &hdr->status : nullptr;
@@ -182,7 +182,8 @@ cudaError_t launch_route(const int64_t* ids, const float* rw, int32_t qlen, int3
                                                                                    status);
   }
   const size_t scan_smem = (2 * (size_t)experts + 1024) * sizeof(int32_t);
-  route_scan_kernel<<<1, 1024, scan_smem, stream>>>(block_hist, nblocks, experts, offsets, tok_tiles, hdr, qlen);
+  route_scan_kernel<<<1, 1024, scan_smem, stream>>>(block_hist, nblocks, experts, offsets, tok_tiles, hdr, qlen,
+                                                     tile_rows);
   if (nblocks > 0) {
     route_scatter_kernel<<<nblocks, kRouteChunk, experts * sizeof(int32_t), stream>>>(ids, rw, slots, experts,
                                                                                      block_hist, perm, inv, w_perm);

@@ -509,6 +509,39 @@ def test_large_rank_parity(rank, fmt, limit):
     assert torch.isfinite(base.float()).all()
 
 
+@pytest.mark.parametrize("tiles", ["narrow", "wide"])
+@pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64"])
+def test_tile_configurations(case, tiles, monkeypatch):
+    """Both token-tile configurations of the GEMMs on the same inputs: narrow
+    (tiles of at most 64 rows, hand-off groups of four stages; chosen for
+    layers with few rows per expert) and wide (tiles of up to 192 rows,
+    groups of two), forced through RAWINT4_TILES. Config 1 has 32 rows per
+    expert on average (some experts need two narrow tiles); the Gemma-4 shape
+    has partial feature blocks; rank 64 (without the clamp, whose decisions
+    near a bound the plain oracle may take the other way) runs two LoRA
+    stages."""
+    import dataclasses
+    monkeypatch.setenv("RAWINT4_TILES", tiles)
+    if case == "config1":
+        wl = make_workload(CONFIGS[1])
+    elif case == "gemma4_clamp":
+        cfg = small_config("gemma4", 128, 8, 2816, 704, 8, 48, swiglu_limit=5.0, routing="normal_topk", x_std=1.0)
+        wl = make_workload(cfg, seed=2027)
+    else:
+        wl = make_workload(dataclasses.replace(CONFIGS[1], rank=64, alpha=128.0, swiglu_limit=0.0))
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+
+
 @pytest.mark.parametrize("cfg_id,limit", [(0, 0.0), (1, 2.0), (1, 0.0)])
 def test_mxfp4_base_parity(cfg_id, limit):
     """The sibling MXFP4 base (E2M1 codes, UE8M0 group scales; the
