@@ -326,6 +326,18 @@ RAWINT4_API int rawint4_moe_lora_saved_preacts(const rawint4_moe_cfg* cfg, const
  * while another host thread launches layer calls. */
 RAWINT4_API int rawint4_moe_set_wait_limit_ns(uint64_t ns);
 
+/* Kernel selection (read from the environment at each call; for testing both
+ * kernel paths on one shape, the results agree within the layer tolerances):
+ *   RAWINT4_TILES=narrow|wide  token tiles of at most 64 rows with the GEMMs'
+ *                              narrow configuration, or of up to 192 rows.
+ *                              Default: narrow for a RAWINT4 base when
+ *                              max_tokens * top_k <= 32 * experts, else wide.
+ *                              Must not change between a forward and its
+ *                              backward.
+ *   RAWINT4_GEMM=tm            the transpose-free backward GEMMs of a RAWINT4
+ *                              base on the tensor-memory kernel instead of
+ *                              the shared-memory one (read once per process). */
+
 #ifdef __cplusplus
 }
 #endif
