@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from workloads import CONFIGS, LORA_NAMES, LayerConfig, expert_counts, lora_shapes, make_batch, make_workload  # noqa: E402
+from workloads import CONFIGS, GEMMA4, LORA_NAMES, LayerConfig, expert_counts, lora_shapes, make_batch, make_workload  # noqa: E402
 
 METRIC = "routed tokens/s per MoE layer (fwd+bwd) and % of HBM/tensor roofline, 1×B200"
 METRIC_INFER = "routed tokens/s per MoE layer (frozen-base inference forward) and % of HBM/tensor roofline, 1×B200"
@@ -59,6 +59,12 @@ def peaks():
     return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def weight_bytes_per_value(cfg: LayerConfig) -> float:
+    """Packed code plus group-scale bytes per base weight: half a byte, and a
+    bf16 (RAWINT4) or UE8M0 byte (MXFP4) scale per 32 weights."""
+    return 0.5 + (1.0 / 32.0 if cfg.weight_format == "mxfp4" else 2.0 / 32.0)
+
+
 def algorithmic(cfg: LayerConfig, counts: torch.Tensor, infer: bool = False):
     """Algorithmic bytes and FLOPs of one fwd+bwd (weights of hit experts read
     in fwd and bwd, LoRA params read twice and grads written, x/out/dY/grad_in
@@ -67,7 +73,7 @@ def algorithmic(cfg: LayerConfig, counts: torch.Tensor, infer: bool = False):
     Q, k, H, I, r = cfg.qlen, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank
     R = int(counts.sum())
     hit = int((counts > 0).sum())
-    w_e = 3 * H * I * (0.5 + 1.0 / 16.0)
+    w_e = 3 * H * I * weight_bytes_per_value(cfg)
     if infer:
         return w_e * hit + 4 * Q * H, 6 * R * H * I + 2 * R * I, R, hit
     flops = 12 * R * H * I + 18 * R * r * (H + I) + 2 * R * I
@@ -174,16 +180,22 @@ def oracle_sample(wl, target_s: float, infer: bool = False):
     rows = 0
     spent = 0.0
     used = []
+    mx = wl.cfg.weight_format == "mxfp4"
+
+    def scales(t):
+        # UE8M0 scale bytes as stored (MXFP4), else bf16 bit patterns
+        return t.detach().cpu().contiguous().numpy() if mx else bits(t)
+
     for e in order:
         sel = np.nonzero((ids == e).any(axis=1))[0]
         sub_ids = np.where(ids[sel] == e, 0, -1)
         layer = omoe.Layer(
-            gate_q=wl.gate_q[e:e + 1].cpu().numpy(), gate_s=bits(wl.gate_s[e:e + 1]),
-            up_q=wl.up_q[e:e + 1].cpu().numpy(), up_s=bits(wl.up_s[e:e + 1]),
-            down_q=wl.down_q[e:e + 1].cpu().numpy(), down_s=bits(wl.down_s[e:e + 1]),
+            gate_q=wl.gate_q[e:e + 1].cpu().numpy(), gate_s=scales(wl.gate_s[e:e + 1]),
+            up_q=wl.up_q[e:e + 1].cpu().numpy(), up_s=scales(wl.up_s[e:e + 1]),
+            down_q=wl.down_q[e:e + 1].cpu().numpy(), down_s=scales(wl.down_s[e:e + 1]),
             lora={n: (0.0 if infer and n.endswith("_b") else 1.0) * orq.bf16_bits_to_f64(bits(wl.lora[n][e:e + 1]))
                   for n in LORA_NAMES},
-            alpha=wl.cfg.alpha, swiglu_limit=wl.cfg.swiglu_limit)
+            alpha=wl.cfg.alpha, swiglu_limit=wl.cfg.swiglu_limit, weight_format=wl.cfg.weight_format)
         x = orq.bf16_bits_to_f64(bits(wl.x[torch.as_tensor(sel, device=wl.x.device)]))
         dy = orq.bf16_bits_to_f64(bits(wl.grad_out[torch.as_tensor(sel, device=wl.x.device)]))
         rw = wl.route_weights.cpu().numpy()[sel].astype(np.float64)
@@ -310,6 +322,10 @@ def main():
                     help="skip the extra measurements of the memory-bound and skewed layers")
     ap.add_argument("--experts", type=int, default=None, help="override the expert count (profiling cases)")
     ap.add_argument("--qlen", type=int, default=None, help="override the token count (profiling cases)")
+    ap.add_argument("--format", default="rawint4", choices=["rawint4", "mxfp4"],
+                    help="base weight format of the layer (the sibling MXFP4 base: E2M1 codes, UE8M0 scales)")
+    ap.add_argument("--shape", default=None, choices=["gemma4"],
+                    help="gemma4: the Gemma-4 MoE layer shape (E=128, top-8, H=2816, I=704) instead of --config")
     ap.add_argument("--mode", default="train", choices=["train", "infer"],
                     help="train: fwd+bwd step (default); infer: frozen-base inference forward")
     args = ap.parse_args()
@@ -320,11 +336,15 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = CONFIGS[args.config]
+    import dataclasses
+    cfg = GEMMA4 if args.shape == "gemma4" else CONFIGS[args.config]
     if args.experts is not None or args.qlen is not None:
-        import dataclasses
         cfg = dataclasses.replace(cfg, name=cfg.name + "_override", experts=args.experts or cfg.experts,
                                   qlen=args.qlen or cfg.qlen)
+    if args.format != cfg.weight_format:
+        cfg = dataclasses.replace(cfg, name=cfg.name + "_" + args.format, weight_format=args.format)
+    # the ncu traffic counters were taken on the default workload's kernels
+    traffic_key = args.config if (args.shape is None and args.format == "rawint4") else None
     workload_name = describe(cfg)
 
     if args.impl == "reference":
@@ -359,7 +379,8 @@ def main():
     counts = expert_counts(wl.expert_ids, cfg.experts)
     nbytes, flops, R, hit = algorithmic(cfg, counts, infer)
     layer = B.Layer.create(cfg.experts, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank, cfg.alpha, cfg.swiglu_limit,
-                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora)
+                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora,
+                           weight_format=cfg.weight_format)
     grads = {n: torch.zeros(s, dtype=torch.bfloat16, device=dev) for n, s in lora_shapes(cfg).items()}
     out = torch.empty_like(wl.x)
     gin = torch.empty_like(wl.x)
@@ -380,7 +401,7 @@ def main():
                                              max_over_ranks)
     value = cfg.qlen * cfg.top_k * world / (ms_step / 1e3)
     kern = kernel_table(launches)
-    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, args.config)
+    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, traffic_key)
     step_roofline["experts_hit"] = hit
 
     # ---- end to end through the public API from pinned host buffers. Steps
@@ -481,8 +502,12 @@ def main():
     # ---- the memory-bound and the skewed layer, and the base-only forward of
     # the memory-bound one (one GPU, default workload only)
     others = None
-    if world == 1 and args.config == 4 and args.experts is None and args.qlen is None and not args.no_other_configs:
-        others = [other_config(c, m, B, dev, stream) for c, m in ((2, "train"), (3, "train"), (2, "infer"))]
+    if (world == 1 and args.config == 4 and args.shape is None and args.format == "rawint4" and args.experts is None
+            and args.qlen is None and not args.no_other_configs):
+        others = [other_config(c, m, B, dev, stream, key) for c, m, key in (
+            (CONFIGS[2], "train", 2), (CONFIGS[3], "train", 3), (CONFIGS[2], "infer", 2),
+            (dataclasses.replace(CONFIGS[4], name="largest_mxfp4", weight_format="mxfp4"), "train", None),
+            (GEMMA4, "train", None))]
 
     if rank == 0:
         line = {
@@ -505,15 +530,15 @@ def describe(cfg: LayerConfig) -> str:
             f"alpha={cfg.alpha:g} qlen={cfg.qlen} swiglu_limit={cfg.swiglu_limit:g} routing={cfg.routing}")
 
 
-def other_config(index: int, mode: str, B, dev, stream, steps: int = 10, warmup: int = 3) -> dict:
+def other_config(cfg: LayerConfig, mode: str, B, dev, stream, traffic_key, steps: int = 10, warmup: int = 3) -> dict:
     """Device-timed steps of another workload (no e2e pass, no CPU baseline)."""
-    cfg = CONFIGS[index]
     infer = mode == "infer"
     wl = make_workload(cfg, device=dev)
     counts = expert_counts(wl.expert_ids, cfg.experts)
     nbytes, flops, R, hit = algorithmic(cfg, counts, infer)
     layer = B.Layer.create(cfg.experts, cfg.top_k, cfg.hidden, cfg.inter, cfg.rank, cfg.alpha, cfg.swiglu_limit,
-                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora)
+                           cfg.qlen, wl.gate_q, wl.gate_s, wl.up_q, wl.up_s, wl.down_q, wl.down_s, wl.lora,
+                           weight_format=cfg.weight_format)
     grads = {n: torch.zeros(s, dtype=torch.bfloat16, device=dev) for n, s in lora_shapes(cfg).items()}
     out = torch.empty_like(wl.x)
     gin = torch.empty_like(wl.x)
@@ -528,8 +553,8 @@ def other_config(index: int, mode: str, B, dev, stream, steps: int = 10, warmup:
 
     ms_step, launches, clocks = device_timed(step, steps, warmup, layer, B, dev, stream, lambda: None, lambda v: v)
     kern = kernel_table(launches)
-    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, index)
-    res = {"workload": describe(cfg), "mode": mode, "steps": steps, "warmup": warmup,
+    roofline, step_roofline = rooflines(kern, R, cfg, infer, nbytes, flops, ms_step, clocks, traffic_key)
+    res = {"workload": describe(cfg), "weight_format": cfg.weight_format, "mode": mode, "steps": steps, "warmup": warmup,
            "ms_per_step": round(ms_step, 4), "value": round(cfg.qlen * cfg.top_k / (ms_step / 1e3), 1), "unit": UNIT,
            "expert_rows": count_stats(counts), "experts_hit": hit, "step_roofline": step_roofline,
            "roofline": roofline, "clocks": clocks, "device_status": layer.status(), "kernels": kernel_summary(kern)}
@@ -544,7 +569,8 @@ def arm_config(cfg: LayerConfig, world: int, workload_name: str, R: int, hit: in
             "global_batch_tokens": cfg.qlen * world, "routed_rows_per_gpu": R,
             "expert_rows": count_stats(counts),
             "l2": "inputs larger than L2: every step streams all hit experts' packed weights "
-                  f"({2 * hit * 3 * cfg.hidden * cfg.inter * (0.5 + 1 / 16) / 1e9:.1f} GB)"}
+                  f"({2 * hit * 3 * cfg.hidden * cfg.inter * weight_bytes_per_value(cfg) / 1e9:.1f} GB)",
+            "weight_format": cfg.weight_format}
 
 
 def run_reference(args, cfg: LayerConfig, workload_name: str) -> int:

@@ -234,15 +234,15 @@ int grid_for_tiles(int sms, int max_tiles, int rowblk) {
 
 // CTA pairs for a pair-kernel launch: all that fit at once, or fewer for a small
 // problem (work items = token tiles x feature blocks).
-int gemm_clusters(int mode, bool narrow, int sms, int max_tiles, int rowblk) {
-  static std::atomic<int> cached[64][2][4];  // per device, configuration and mode; 0 = not queried yet
+int gemm_clusters(int mode, int fmt, bool narrow, int sms, int max_tiles, int rowblk) {
+  static std::atomic<int> cached[64][2][2][4];  // per device, configuration, format and mode; 0 = not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  int fit = cached[dev][narrow][mode].load();
+  int fit = cached[dev][narrow][fmt][mode].load();
   if (fit <= 0) {
-    const int n = narrow ? gemm_pair_max_clusters_narrow(mode) : gemm_pair_max_clusters(mode);
+    const int n = narrow ? gemm_pair_max_clusters_narrow(mode, fmt) : gemm_pair_max_clusters(mode, fmt);
     fit = n > 0 ? n : (sms / 2 > 0 ? sms / 2 : 1);  // occupancy query unavailable: one pair per SM pair
-    cached[dev][narrow][mode].store(fit);
+    cached[dev][narrow][fmt][mode].store(fit);
   }
   const int64_t items = (int64_t)max_tiles * rowblk;
   return (int)(items < fit ? (items > 0 ? items : 1) : fit);
@@ -279,16 +279,16 @@ bool narrow_tiles(const rawint4_moe_cfg& c) {
 
 // Which kernel runs the transpose-free backward GEMMs (down^T, gate/up^T):
 // the shared-memory operand pair kernel (gemm_pair.cu: MN-major decoded
-// tiles, no transposition), or the tensor-memory pair kernel (gemm_tm.cu) for
-// an MXFP4 base or when the environment selects it (RAWINT4_GEMM=tm). The
-// forward GEMMs always run on the tensor-memory kernel.
-bool use_tm_gemm(int fmt) {
+// tiles, no transposition), or the tensor-memory pair kernel (gemm_tm.cu)
+// when the environment selects it (RAWINT4_GEMM=tm). The forward GEMMs
+// always run on the tensor-memory kernel.
+bool use_tm_gemm(int) {
   static int v = -1;
   if (v < 0) {
     const char* e = getenv("RAWINT4_GEMM");
     v = (e && strcmp(e, "tm") == 0) ? 1 : 0;
   }
-  return v == 1 || fmt == RAWINT4_FORMAT_MXFP4;
+  return v == 1;
 }
 
 // Bound on any pipeline wait of the GEMM kernels (test export can shorten it).
@@ -631,8 +631,8 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     if (tm)
       R4_TRY(launch_gemm_tm(kModeDownT, fmt, gp, mp, tm_clusters(kModeDownT, fmt, false, sms, max_tiles, gp.n_rowblk), st));
     else {
-      const int ncl = gemm_clusters(kModeDownT, nar, sms, max_tiles, gp.n_rowblk);
-      R4_TRY(nar ? launch_gemm_pair_narrow(kModeDownT, gp, mp, ncl, st) : launch_gemm_pair(kModeDownT, gp, mp, ncl, st));
+      const int ncl = gemm_clusters(kModeDownT, fmt, nar, sms, max_tiles, gp.n_rowblk);
+      R4_TRY(nar ? launch_gemm_pair_narrow(kModeDownT, fmt, gp, mp, ncl, st) : launch_gemm_pair(kModeDownT, fmt, gp, mp, ncl, st));
     }
   }
 
@@ -681,8 +681,8 @@ int rawint4_moe_lora_bwd(const rawint4_moe_cfg* cfg, const rawint4_moe_base* bas
     if (tm)
       R4_TRY(launch_gemm_tm(kModeGateUpT, fmt, gp, mp, tm_clusters(kModeGateUpT, fmt, false, sms, max_tiles, gp.n_rowblk), st));
     else {
-      const int ncl = gemm_clusters(kModeGateUpT, nar, sms, max_tiles, gp.n_rowblk);
-      R4_TRY(nar ? launch_gemm_pair_narrow(kModeGateUpT, gp, mp, ncl, st) : launch_gemm_pair(kModeGateUpT, gp, mp, ncl, st));
+      const int ncl = gemm_clusters(kModeGateUpT, fmt, nar, sms, max_tiles, gp.n_rowblk);
+      R4_TRY(nar ? launch_gemm_pair_narrow(kModeGateUpT, fmt, gp, mp, ncl, st) : launch_gemm_pair(kModeGateUpT, fmt, gp, mp, ncl, st));
     }
   }
   {

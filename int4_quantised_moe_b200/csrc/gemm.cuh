@@ -160,11 +160,12 @@ struct GemmMaps {
 };
 
 // CTA pairs with the decoded weights in shared memory (gemm_pair.cu), the
-// transpose-free modes down^T and gate/up^T of a RAWINT4 base; `clusters`
-// pairs (at most the number resident at once).
-cudaError_t launch_gemm_pair(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream);
+// transpose-free modes down^T and gate/up^T of a RAWINT4 or an MXFP4 base
+// (fmt); `clusters` pairs (at most the number resident at once).
+cudaError_t launch_gemm_pair(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+                             cudaStream_t stream);
 // CTA pairs of the pair kernel's mode resident at once on this device (0 on error).
-int gemm_pair_max_clusters(int mode);
+int gemm_pair_max_clusters(int mode, int fmt);
 // CTA pairs with the decoded weights in tensor memory (gemm_tm.cu), every
 // mode; fmt: RAWINT4_FORMAT_RAWINT4 (bf16 scales s0/s1) or
 // RAWINT4_FORMAT_MXFP4 (E2M1 codes, UE8M0 scale bytes e0/e1).
@@ -177,8 +178,8 @@ int gemm_tm_max_clusters(int mode, int fmt);
 cudaError_t launch_gemm_tm_narrow(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
                                   cudaStream_t stream);
 int gemm_tm_max_clusters_narrow(int mode, int fmt);
-cudaError_t launch_gemm_pair_narrow(int mode, const GemmParams& p, const GemmMaps& maps, int clusters,
+cudaError_t launch_gemm_pair_narrow(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
                                     cudaStream_t stream);
-int gemm_pair_max_clusters_narrow(int mode);
+int gemm_pair_max_clusters_narrow(int mode, int fmt);
 
 }  // namespace r4

@@ -174,7 +174,7 @@ __device__ __forceinline__ uint32_t scale_off(int dt) {
 
 // Loader lane `ln` issues the cp.async copies of stage s's scales into slot
 // `S` (zero-filled past the mode's features).
-template <int MODE>
+template <int MODE, int FMT>
 __device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, int fc, int s, int ln, uint8_t* S) {
   if constexpr (!kAMnMajor<MODE>) {
 #pragma unroll
@@ -191,6 +191,23 @@ __device__ __forceinline__ void load_stage_scales(const GemmParams& p, int e, in
       const bool ok = f < p.feat;
       const uint16_t* src = ok ? sp + (int64_t)e * p.s_expert + (int64_t)f * p.s_row + 2 * s : p.s0;
       cp_async_4(S + row * 4, src, ok ? 4u : 0u);
+    }
+  } else if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {
+    // [64 stored rows][4] UE8M0 bytes: the 4 groups of this CTA's 128
+    // features (H and I are multiples of 128, so a row's 4 bytes are 4-byte
+    // aligned and all inside the features)
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int kr = ln + 32 * t;
+      int row = s * kBlockK + kr;
+      const uint8_t* sp = p.e0;
+      if (MODE == kModeGateUpT && row >= p.stored_rows) {
+        row -= p.stored_rows;
+        sp = p.e1;
+      }
+      const bool ok = fc < p.feat;
+      const uint8_t* src = sp + (int64_t)e * p.s_expert + (int64_t)row * p.s_row + fc / 32;
+      cp_async_4(S + kr * 4, ok ? src : p.e0, ok ? 4u : 0u);
     }
   } else {
 #pragma unroll
@@ -273,9 +290,10 @@ __device__ __forceinline__ void lora_values(const GemmParams& p, int e, int fc, 
   }
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  static_assert(FMT == RAWINT4_FORMAT_RAWINT4 || kAMnMajor<MODE>, "an MXFP4 base runs the transpose-free modes only");
   const CUtensorMap& tq0 = maps.q0;
   const CUtensorMap& tq1 = maps.q1;
   extern __shared__ uint8_t smem_raw[];
@@ -406,7 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nsub = min(kGroup, n_main - s0);
         if (!wait_warp(&p_empty[ring.stage], ring.phase ^ 1u, abort_flag, status, lim)) goto drain_s;
         for (int u = 0; u < nsub; ++u)
-          load_stage_scales<MODE>(p, tt.x, fc, s0 + u, lane, sS + (ring.stage * kGroup + u) * kSBytes);
+          load_stage_scales<MODE, FMT>(p, tt.x, fc, s0 + u, lane, sS + (ring.stage * kGroup + u) * kSBytes);
         cp_async_arrive_noinc(&p_full[ring.stage]);
         ring.advance(kSlotsP);
       }
@@ -682,7 +700,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // the leader's first decoder warp also waits for each group's B tiles
     const bool b_watch = cta == 0 && warp == kDecWarp0;
     Ring rg, rp, rbd;
-    const uint32_t s_off = scale_off<MODE>(dt);
+    // this thread's scale in a stage's scale slot (MXFP4: one byte per group)
+    const uint32_t s_off = FMT == RAWINT4_FORMAT_MXFP4 ? (uint32_t)(mn_kr(dt) * 4 + mn_qq(dt)) : scale_off<MODE>(dt);
     for (int tile = tile0; tile < n_tiles; tile += tile_step) {
       const int4 tt = p.tok_tiles[tile / n_rowblk];
       const int fc = cta_f0<MODE>(tile % n_rowblk, cta);
@@ -702,9 +721,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int b = 0; b < 2; ++b) {
             if (h + b < nb) {
               const int st = rp.stage * kGroup + h + b;
-              const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + st * kSBytes + s_off);
               const uint4 q4 = packed_group<MODE>(sP + st * kPBytes, dt);
-              decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
+              if constexpr (FMT == RAWINT4_FORMAT_MXFP4) {
+                const uint32_t hb = ue8m0_to_h(sS[st * kSBytes + s_off]);
+                const uint32_t h2 = hb | (hb << 16);
+                decode_group32_mxfp4(q4, *reinterpret_cast<const __half2*>(&h2), w[b]);
+              } else {
+                const uint16_t sc = *reinterpret_cast<const uint16_t*>(sS + st * kSBytes + s_off);
+                decode_group32(q4, bf16_scale_to_h2(sc), w[b]);
+              }
             }
           }
           if (h + 2 >= nb) {
@@ -784,28 +809,28 @@ done:
   if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 bool set_smem_attr() {
   static std::atomic<unsigned long long> done{0};
   int dev = 0;
   if (!device_flag_test(done, &dev)) {
-    if (cudaFuncSetAttribute(gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_pair_kernel<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
       return false;
     device_flag_set(done, dev);
   }
   return true;
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 cudaError_t launch_mode(const GemmParams& p, const GemmMaps& m, int clusters, cudaStream_t stream) {
-  if (!set_smem_attr<MODE>()) return cudaErrorInvalidValue;
-  gemm_pair_kernel<MODE><<<2 * clusters, kThreads, kSmemBytes, stream>>>(p, m);
+  if (!set_smem_attr<MODE, FMT>()) return cudaErrorInvalidValue;
+  gemm_pair_kernel<MODE, FMT><<<2 * clusters, kThreads, kSmemBytes, stream>>>(p, m);
   return cudaGetLastError();
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 int max_clusters_mode() {
-  if (!set_smem_attr<MODE>()) return 0;
+  if (!set_smem_attr<MODE, FMT>()) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -818,7 +843,7 @@ int max_clusters_mode() {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MODE>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MODE, FMT>, &cfg) != cudaSuccess) return 0;
   return n;
 }
 
@@ -827,15 +852,36 @@ int max_clusters_mode() {
 // The library runs the two transpose-free backward GEMMs (MN-major decoded
 // A tiles in shared memory) on this kernel; the kernel itself is written for
 // every mode.
-cudaError_t R4_PAIR_LAUNCH(int mode, const GemmParams& p, const GemmMaps& maps, int clusters, cudaStream_t stream) {
-  if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT>(p, maps, clusters, stream);
-  if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT>(p, maps, clusters, stream);
+cudaError_t R4_PAIR_LAUNCH(int mode, int fmt, const GemmParams& p, const GemmMaps& maps, int clusters,
+                           cudaStream_t stream) {
+  constexpr int R = RAWINT4_FORMAT_RAWINT4;
+  if (fmt == R) {
+    if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
+    if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
+  }
+#if !R4_PAIR_NARROW  // the narrow configuration serves a RAWINT4 base only
+  constexpr int X = RAWINT4_FORMAT_MXFP4;
+  if (fmt == X) {
+    if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
+    if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT, X>(p, maps, clusters, stream);
+  }
+#endif
   return cudaErrorInvalidValue;
 }
 
-int R4_PAIR_MAXCL(int mode) {
-  if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT>();
-  if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT>();
+int R4_PAIR_MAXCL(int mode, int fmt) {
+  constexpr int R = RAWINT4_FORMAT_RAWINT4;
+  if (fmt == R) {
+    if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT, R>();
+    if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT, R>();
+  }
+#if !R4_PAIR_NARROW
+  constexpr int X = RAWINT4_FORMAT_MXFP4;
+  if (fmt == X) {
+    if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT, X>();
+    if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT, X>();
+  }
+#endif
   return 0;
 }
 

@@ -65,6 +65,11 @@ CONFIGS = {
     4: LayerConfig("largest", 384, 8, 7168, 2048, 32, 64.0, 8192, 0.0, "uniform_topk"),
 }
 
+# The adjacent Gemma-4 MoE layer shape (test_gemma4_moe.py,
+# TestGemma4FullLayerIntegration.real_config: hidden 2816, 128 experts, top-8,
+# expert intermediate 704) with a 4096-token batch and a rank-16 adapter.
+GEMMA4 = LayerConfig("gemma4_layer", 128, 8, 2816, 704, 16, 32.0, 4096, 0.0, "normal_topk")
+
 
 def lora_shapes(cfg: LayerConfig) -> Dict[str, tuple]:
     E, H, I, r = cfg.experts, cfg.hidden, cfg.inter, cfg.rank
