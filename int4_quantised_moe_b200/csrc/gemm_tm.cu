@@ -430,6 +430,7 @@ __device__ __forceinline__ void lora_values_mn(const GemmParams& p, int e, int f
 template <int MODE, int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  static_assert(kPSub<MODE> % kGroup == 0, "a hand-off group lies within one packed slot");
   const CUtensorMap& tq0 = maps.q0;
   const CUtensorMap& tq1 = maps.q1;
   extern __shared__ uint8_t smem_raw[];
