@@ -330,8 +330,8 @@ RAWINT4_API int rawint4_moe_set_wait_limit_ns(uint64_t ns);
  * kernel paths on one shape, the results agree within the layer tolerances):
  *   RAWINT4_TILES=narrow|wide  token tiles of at most 64 rows with the GEMMs'
  *                              narrow configuration, or of up to 192 rows.
- *                              Default: narrow for a RAWINT4 base when
- *                              max_tokens * top_k <= 32 * experts, else wide.
+ *                              Default: narrow when max_tokens * top_k <=
+ *                              32 * experts, else wide.
  *                              Must not change between a forward and its
  *                              backward.
  *   RAWINT4_GEMM=tm            the transpose-free backward GEMMs of a RAWINT4

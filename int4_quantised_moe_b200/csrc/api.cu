@@ -264,13 +264,12 @@ int tm_clusters(int mode, int fmt, bool narrow, int sms, int max_tiles, int rowb
 }
 
 // Token-tile configuration of a call: narrow (tiles of at most
-// kTileRowsNarrow rows, the GEMMs' narrow configurations) for a RAWINT4 base
-// whose workspace averages at most kTileRowsNarrow / 2 routed rows per expert
-// (max_tokens x top_k / experts), wide otherwise. The choice depends on the
-// configuration only, so a backward always matches its forward. The
-// environment may force it (RAWINT4_TILES=narrow or wide) for testing.
+// kTileRowsNarrow rows, the GEMMs' narrow configurations) when the workspace
+// averages at most kTileRowsNarrow / 2 routed rows per expert (max_tokens x
+// top_k / experts), wide otherwise. The choice depends on the configuration
+// only, so a backward always matches its forward. The environment may force
+// it (RAWINT4_TILES=narrow or wide) for testing.
 bool narrow_tiles(const rawint4_moe_cfg& c) {
-  if (c.weight_format != RAWINT4_FORMAT_RAWINT4) return false;
   const char* e = getenv("RAWINT4_TILES");
   if (e && strcmp(e, "narrow") == 0) return true;
   if (e && strcmp(e, "wide") == 0) return false;

@@ -859,13 +859,11 @@ cudaError_t R4_PAIR_LAUNCH(int mode, int fmt, const GemmParams& p, const GemmMap
     if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
     if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
   }
-#if !R4_PAIR_NARROW  // the narrow configuration serves a RAWINT4 base only
   constexpr int X = RAWINT4_FORMAT_MXFP4;
   if (fmt == X) {
     if (mode == kModeDownT) return R4_PAIR_NS::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
     if (mode == kModeGateUpT) return R4_PAIR_NS::launch_mode<kModeGateUpT, X>(p, maps, clusters, stream);
   }
-#endif
   return cudaErrorInvalidValue;
 }
 
@@ -875,13 +873,11 @@ int R4_PAIR_MAXCL(int mode, int fmt) {
     if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT, R>();
     if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT, R>();
   }
-#if !R4_PAIR_NARROW
   constexpr int X = RAWINT4_FORMAT_MXFP4;
   if (fmt == X) {
     if (mode == kModeDownT) return R4_PAIR_NS::max_clusters_mode<kModeDownT, X>();
     if (mode == kModeGateUpT) return R4_PAIR_NS::max_clusters_mode<kModeGateUpT, X>();
   }
-#endif
   return 0;
 }
 

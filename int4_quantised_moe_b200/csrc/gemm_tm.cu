@@ -60,7 +60,8 @@
 // two stages; the narrow one (gemm_tm_narrow.cu, R4_TM_NARROW = 1), for
 // layers with few rows per expert, holds tiles of at most kTileRowsNarrow
 // rows, so tensor memory has room for eight A stages and the hand-off groups
-// are four stages long (half the synchronisations per weight byte).
+// are four stages long (half the synchronisations per weight byte); it runs
+// the forward modes of either base format.
 #include "gemm.cuh"
 #include "route.cuh"
 
@@ -1059,9 +1060,9 @@ cudaError_t R4_TM_LAUNCH(int mode, int fmt, const GemmParams& p, const GemmMaps&
   switch (mode * 2 + (fmt == X ? 1 : 0)) {
     case kModeGateUp * 2: return R4_TM_NS::launch_mode<kModeGateUp, R>(p, maps, clusters, stream);
     case kModeDown * 2: return R4_TM_NS::launch_mode<kModeDown, R>(p, maps, clusters, stream);
-#if !R4_TM_NARROW  // the narrow configuration serves the RAWINT4 forward only
     case kModeGateUp * 2 + 1: return R4_TM_NS::launch_mode<kModeGateUp, X>(p, maps, clusters, stream);
     case kModeDown * 2 + 1: return R4_TM_NS::launch_mode<kModeDown, X>(p, maps, clusters, stream);
+#if !R4_TM_NARROW  // the narrow configuration serves the forward modes only
     case kModeDownT * 2: return R4_TM_NS::launch_mode<kModeDownT, R>(p, maps, clusters, stream);
     case kModeDownT * 2 + 1: return R4_TM_NS::launch_mode<kModeDownT, X>(p, maps, clusters, stream);
     case kModeGateUpT * 2: return R4_TM_NS::launch_mode<kModeGateUpT, R>(p, maps, clusters, stream);
@@ -1076,9 +1077,9 @@ int R4_TM_MAXCL(int mode, int fmt) {
   switch (mode * 2 + (fmt == X ? 1 : 0)) {
     case kModeGateUp * 2: return R4_TM_NS::max_clusters_mode<kModeGateUp, R>();
     case kModeDown * 2: return R4_TM_NS::max_clusters_mode<kModeDown, R>();
-#if !R4_TM_NARROW  // the narrow configuration serves the RAWINT4 forward only
     case kModeGateUp * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeGateUp, X>();
     case kModeDown * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeDown, X>();
+#if !R4_TM_NARROW  // the narrow configuration serves the forward modes only
     case kModeDownT * 2: return R4_TM_NS::max_clusters_mode<kModeDownT, R>();
     case kModeDownT * 2 + 1: return R4_TM_NS::max_clusters_mode<kModeDownT, X>();
     case kModeGateUpT * 2: return R4_TM_NS::max_clusters_mode<kModeGateUpT, R>();

@@ -510,7 +510,7 @@ def test_large_rank_parity(rank, fmt, limit):
 
 
 @pytest.mark.parametrize("tiles", ["narrow", "wide"])
-@pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64"])
+@pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64", "mxfp4"])
 def test_tile_configurations(case, tiles, monkeypatch):
     """Both token-tile configurations of the GEMMs on the same inputs: narrow
     (tiles of at most 64 rows, hand-off groups of four stages; chosen for
@@ -519,7 +519,7 @@ def test_tile_configurations(case, tiles, monkeypatch):
     expert on average (some experts need two narrow tiles); the Gemma-4 shape
     has partial feature blocks; rank 64 (without the clamp, whose decisions
     near a bound the plain oracle may take the other way) runs two LoRA
-    stages."""
+    stages; the last case has an MXFP4 base."""
     import dataclasses
     monkeypatch.setenv("RAWINT4_TILES", tiles)
     if case == "config1":
@@ -527,8 +527,10 @@ def test_tile_configurations(case, tiles, monkeypatch):
     elif case == "gemma4_clamp":
         cfg = small_config("gemma4", 128, 8, 2816, 704, 8, 48, swiglu_limit=5.0, routing="normal_topk", x_std=1.0)
         wl = make_workload(cfg, seed=2027)
-    else:
+    elif case == "rank64":
         wl = make_workload(dataclasses.replace(CONFIGS[1], rank=64, alpha=128.0, swiglu_limit=0.0))
+    else:
+        wl = make_workload(dataclasses.replace(CONFIGS[1], weight_format="mxfp4", swiglu_limit=0.0))
     out_r, gin_r, groute_r, grads_r = oracle(wl)
     g = on_gpu(wl)
     layer = make_layer(g)
