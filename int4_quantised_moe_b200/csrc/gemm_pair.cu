@@ -561,6 +561,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int n_rows = tt.z;
       const int p0 = tt.y;
       const int ab = it & 1;
+      if constexpr (MODE == kModeDownT) {
+        // the item's saved G/U rows (this warp's 32 features, 128 bytes a
+        // row) are brought into L2 while its accumulator is computed
+        if (live && fc + 32 * q < p.feat) {
+          for (int n = lane; n < n_rows; n += 32) {
+            const int64_t o = (int64_t)(p0 + n) * p.ld_out + fc + 32 * q;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.in_g + o));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.in_u + o));
+          }
+        }
+      }
       // the four epilogue warps leave together or not at all: a warp that
       // went on alone would wait forever at the exchange barriers
       const bool ok = wait_warp(&acc_full[ab], (uint32_t)(it >> 1) & 1u, abort_flag, status, lim);

@@ -467,46 +467,74 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2(uint32_t v) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One job per blockIdx.y. Copies: 8 elements per thread and step (16-byte
-// loads and stores; K is a multiple of 128). Transposes: tiles of 64 columns
-// of one expert; the tile's 64 source rows of r elements are one contiguous,
-// 16-byte aligned run of 128 r bytes, loaded as 16-byte vectors, turned
-// around in shared memory and stored as rows of 64 fp16.
+// One job per blockIdx.y. Copies: one warp per output row, 8 elements per
+// lane and vector (16-byte loads and stores; K is a multiple of 64).
+// Transposes with a rank that is a multiple of 8: two adjacent columns per
+// thread (below). Other ranks: tiles of 64 columns of one expert; the tile's
+// 64 source rows of r elements are one contiguous, 16-byte aligned run of
+// 128 r bytes, loaded as 16-byte vectors, turned around in shared memory and
+// stored as rows of 64 fp16.
 __global__ void __launch_bounds__(256) lora_convert_kernel(LoraCvt j0, LoraCvt j1, LoraCvt j2, int experts) {
   const LoraCvt jb = blockIdx.y == 0 ? j0 : (blockIdx.y == 1 ? j1 : j2);
   if (!jb.dst) return;
   const int r = jb.rank, rp = jb.rpad, cols = jb.cols;
   if (!jb.transpose) {
+    // one warp per output row: the row's expert and rank are found once, and
+    // its vectors go four per lane and pass, loads ahead of stores
     const int rows_out = rp * jb.nsrc;
     const int vpr = cols / 8;
-    const int64_t total = (int64_t)experts * rows_out * vpr;
+    const int rows_total = experts * rows_out;
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
     uint4* dst = reinterpret_cast<uint4*>(jb.dst);
-    const int64_t step = (int64_t)gridDim.x * blockDim.x;
-    // four vectors per thread and pass, all loads issued before the stores
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total; base += 4 * step) {
-      uint4 out[4];
+    for (int rg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; rg < rows_total; rg += nwarps) {
+      const int e = rg / rows_out;
+      const int row = rg - e * rows_out;
+      const int blk = row / rp, j = row - blk * rp;
+      uint4* d = dst + (int64_t)rg * vpr;
+      if (j >= r) {
+        for (int v = lane; v < vpr; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>((blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * cols);
+      for (int v0 = lane; v0 < vpr; v0 += 128) {
+        uint4 in[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t idx = base + q * step;
-        out[q] = make_uint4(0u, 0u, 0u, 0u);
-        if (idx < total) {
-          const int64_t row_g = idx / vpr;
-          const int v = (int)(idx - row_g * vpr);
-          const int e = (int)(row_g / rows_out);
-          const int row = (int)(row_g - (int64_t)e * rows_out);
-          const int blk = row / rp, j = row - blk * rp;
-          if (j < r) {
-            const uint16_t* src = (blk == 0 ? jb.src0 : jb.src1) + ((int64_t)e * r + j) * cols;
-            const uint4 in = __ldg(reinterpret_cast<const uint4*>(src) + v);
-            out[q] = make_uint4(bf16x2_to_h2(in.x), bf16x2_to_h2(in.y), bf16x2_to_h2(in.z), bf16x2_to_h2(in.w));
-          }
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < vpr) in[q] = __ldg(src + v0 + 32 * q);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < vpr)
+            d[v0 + 32 * q] = make_uint4(bf16x2_to_h2(in[q].x), bf16x2_to_h2(in[q].y), bf16x2_to_h2(in[q].z),
+                                        bf16x2_to_h2(in[q].w));
+      }
+    }
+  } else if (r % 8 == 0) {
+    // transposes of a rank that fills 16-byte vectors: thread -> two adjacent
+    // columns c, c + 1 of one expert, whose 2 r source values are one
+    // contiguous, 16-byte aligned run; for each rank j the warp stores 64
+    // adjacent fp16 (128 bytes) of output row j
+    const int64_t pairs = (int64_t)experts * (cols / 2);
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    const int rv = r / 8;  // 16-byte vectors per source row
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < pairs; t += step) {
+      const int e = (int)(t / (cols / 2));
+      const int c = 2 * (int)(t - (int64_t)e * (cols / 2));
+      const uint4* src = reinterpret_cast<const uint4*>(jb.src0 + ((int64_t)e * cols + c) * r);  // [2][r]
+      uint16_t* d = jb.dst + (int64_t)e * rp * cols + c;
+      for (int j0 = 0; j0 < r; j0 += 8) {
+        const uint4 a = __ldg(src + j0 / 8);       // column c, ranks j0..j0+7
+        const uint4 b = __ldg(src + rv + j0 / 8);  // column c + 1
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float fa = __uint_as_float(((wa[u >> 1] >> (16 * (u & 1))) & 0xFFFFu) << 16);
+          const float fb = __uint_as_float(((wb[u >> 1] >> (16 * (u & 1))) & 0xFFFFu) << 16);
+          const uint32_t h = (uint32_t)f16_bits_rn(fa) | ((uint32_t)f16_bits_rn(fb) << 16);
+          *reinterpret_cast<uint32_t*>(d + (int64_t)(j0 + u) * cols) = h;
         }
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t idx = base + q * step;
-        if (idx < total) dst[idx] = out[q];
-      }
+      for (int j = r; j < rp; ++j) *reinterpret_cast<uint32_t*>(d + (int64_t)j * cols) = 0u;
     }
   } else {
     __shared__ float tile[64][65];  // 64 source rows x up to 64 ranks (+1: no bank conflicts)

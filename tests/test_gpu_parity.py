@@ -510,7 +510,7 @@ def test_large_rank_parity(rank, fmt, limit):
 
 
 @pytest.mark.parametrize("tiles", ["narrow", "wide"])
-@pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64", "mxfp4"])
+@pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64", "rank12", "mxfp4"])
 def test_tile_configurations(case, tiles, monkeypatch):
     """Both token-tile configurations of the GEMMs on the same inputs: narrow
     (tiles of at most 64 rows, hand-off groups of four stages; chosen for
@@ -519,7 +519,8 @@ def test_tile_configurations(case, tiles, monkeypatch):
     expert on average (some experts need two narrow tiles); the Gemma-4 shape
     has partial feature blocks; rank 64 (without the clamp, whose decisions
     near a bound the plain oracle may take the other way) runs two LoRA
-    stages; the last case has an MXFP4 base."""
+    stages; rank 12 (not a multiple of 8) takes the shared-memory transposes
+    of the LoRA fp16 copies; the last case has an MXFP4 base."""
     import dataclasses
     monkeypatch.setenv("RAWINT4_TILES", tiles)
     if case == "config1":
@@ -529,6 +530,8 @@ def test_tile_configurations(case, tiles, monkeypatch):
         wl = make_workload(cfg, seed=2027)
     elif case == "rank64":
         wl = make_workload(dataclasses.replace(CONFIGS[1], rank=64, alpha=128.0, swiglu_limit=0.0))
+    elif case == "rank12":
+        wl = make_workload(dataclasses.replace(CONFIGS[1], rank=12, alpha=24.0, swiglu_limit=0.0))
     else:
         wl = make_workload(dataclasses.replace(CONFIGS[1], weight_format="mxfp4", swiglu_limit=0.0))
     out_r, gin_r, groute_r, grads_r = oracle(wl)
