@@ -16,14 +16,25 @@ namespace {
 constexpr int kSkA = 128 * 64 * 2;  // A tile: 128 rows x 64 fp16
 constexpr int kSkB = 64 * 64 * 2;   // B tile: 64 rows x 64 fp16
 constexpr int kSkStage = kSkA + kSkB;
-constexpr int kSkOffBar = kSkStages * kSkStage;
-constexpr int kSkNumBars = 2 * kSkStages + 4;
-constexpr int kSkOffMisc = kSkOffBar + kSkNumBars * 8;
-// gradient staging of the transposed outputs: [2 outputs][32 rank][128 features] fp32
-constexpr int kSkOffStage = (kSkOffMisc + 16 + 15) / 16 * 16;
+// Shared memory of each mode: the ring of stages, the barriers, and (Grads
+// only) the gradient staging of the transposed outputs:
+// [2 outputs][32 rank][128 features] fp32. Rows mode spends the staging's
+// room on a fourth stage.
+template <int MODE>
+constexpr int kSkStagesOf = MODE == kSkRows ? kSkStages + 1 : kSkStages;
+template <int MODE>
+constexpr int kSkOffBar = kSkStagesOf<MODE> * kSkStage;
+template <int MODE>
+constexpr int kSkNumBars = 2 * kSkStagesOf<MODE> + 4;
+template <int MODE>
+constexpr int kSkOffMisc = kSkOffBar<MODE> + kSkNumBars<MODE> * 8;
+template <int MODE>
+constexpr int kSkOffStage = (kSkOffMisc<MODE> + 16 + 15) / 16 * 16;
 constexpr int kSkStageFloats = 2 * 32 * 128;
-constexpr int kSkSmem = kSkOffStage + kSkStageFloats * 4 + 1024;
-static_assert(2 * (kSkSmem + 1024) <= 233472, "two CTAs per SM (228 KB per SM, 1 KB reserved per CTA)");
+template <int MODE>
+constexpr int kSkSmem = kSkOffStage<MODE> + (MODE == kSkGrads ? kSkStageFloats * 4 : 0) + 1024;
+static_assert(2 * (kSkSmem<kSkRows> + 1024) <= 233472 && 2 * (kSkSmem<kSkGrads> + 1024) <= 233472,
+              "two CTAs per SM (228 KB per SM, 1 KB reserved per CTA)");
 constexpr uint32_t kSkTmemCols = 256;
 
 struct GradItem {
@@ -166,19 +177,20 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     skinny_kernel(const __grid_constant__ SkParams p, const __grid_constant__ SkMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkOffBar);
+  constexpr int kStages = kSkStagesOf<MODE>;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkOffBar<MODE>);
   uint64_t* full = bars;
-  uint64_t* empty = full + kSkStages;
-  uint64_t* acc_full = empty + kSkStages;
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSkOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkOffMisc + 4);
-  float* gstage = reinterpret_cast<float*>(smem + kSkOffStage);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSkOffMisc<MODE>);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkOffMisc<MODE> + 4);
+  float* gstage = reinterpret_cast<float*>(smem + kSkOffStage<MODE>);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSkStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -221,7 +233,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
               tma_load_3d(st + kSkA, &maps.b[s], &full[ring.stage], 64 * k, 0, tt.x);
             }
             __syncwarp();
-            ring.advance(kSkStages);
+            ring.advance(kStages);
           }
         }
       } else {
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             tma_load_2d(st + kSkA, &maps.b[jb.bmap], &full[ring.stage], jb.scol, row0 + 64 * k);
           }
           __syncwarp();
-          ring.advance(kSkStages);
+          ring.advance(kStages);
         }
       }
     }
@@ -309,7 +321,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             umma_commit(&empty[ring.stage]);
           }
           __syncwarp();
-          ring.advance(kSkStages);
+          ring.advance(kStages);
         }
       }
       if (lane == 0) umma_commit(&acc_full[ab]);
@@ -450,14 +462,14 @@ cudaError_t launch_sk(const SkParams& p, const SkMaps& m, int grid, cudaStream_t
   static std::atomic<unsigned long long> attr{0};
   int dev = 0;
   if (!device_flag_test(attr, &dev)) {
-    cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmem);
+    cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmem<MODE>);
     if (e != cudaSuccess) return e;
     // the largest shared-memory carveout, so that two CTAs fit on an SM
     e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     device_flag_set(attr, dev);
   }
-  skinny_kernel<MODE><<<grid, kSkThreads, kSkSmem, stream>>>(p, m);
+  skinny_kernel<MODE><<<grid, kSkThreads, kSkSmem<MODE>, stream>>>(p, m);
   return cudaGetLastError();
 }
 
