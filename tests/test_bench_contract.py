@@ -48,6 +48,27 @@ def test_reference_arm_reports_expert_rows():
     assert 0 <= er["min"] <= er["median"] <= er["max"] and 0 <= er["empty"] <= 4
 
 
+def test_reference_arm_other_format_and_shape():
+    """--format mxfp4 times the layer with an MXFP4 base; --shape gemma4 the
+    Gemma-4 layer shape (here with fewer experts and tokens for speed)."""
+    d = _run("--format", "mxfp4")
+    assert d["config"]["weight_format"] == "mxfp4" and "mxfp4" in d["config"]["workload"]
+    g = _run("--shape", "gemma4", "--experts", "8", "--qlen", "8")
+    assert g["config"]["workload"].startswith("gemma4_layer") and "H=2816 I=704" in g["config"]["workload"]
+    assert g["config"]["weight_format"] == "rawint4"
+
+
+def test_weight_bytes_per_value():
+    """Half a byte of code per weight plus the group scale: a bf16 (RAWINT4)
+    or a UE8M0 byte (MXFP4) per 32 weights."""
+    sys.path.insert(0, ROOT)
+    import dataclasses
+    import bench
+    from workloads import CONFIGS
+    assert bench.weight_bytes_per_value(CONFIGS[4]) == 0.5 + 2 / 32
+    assert bench.weight_bytes_per_value(dataclasses.replace(CONFIGS[4], weight_format="mxfp4")) == 0.5 + 1 / 32
+
+
 def test_phase_split_of_launches():
     """Forward and backward kernel time per step from the launch list in issue order."""
     sys.path.insert(0, ROOT)
