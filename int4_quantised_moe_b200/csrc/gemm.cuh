@@ -11,11 +11,13 @@ namespace r4 {
 // epilogue of an item overlaps the next item's mainloop); they take the same
 // parameters and differ in where the decoded weights go:
 //   gemm_tm.cu    into tensor memory (UMMA A operand read from TMEM): the
-//                 forward GEMMs (K-major decode), and every mode of an MXFP4
-//                 base
+//                 forward GEMMs (K-major decode) of either base format; its
+//                 transpose-free modes are a second path for testing
 //   gemm_pair.cu  into shared memory (UMMA A operand from a descriptor): the
-//                 transpose-free backward GEMMs of a RAWINT4 base, whose
+//                 transpose-free backward GEMMs of either base format, whose
 //                 MN-major tiles need no transposition there
+// Each is also built in a narrow tile configuration (gemm_tm_narrow.cu,
+// gemm_pair_narrow.cu) for layers with few rows per expert.
 enum GemmMode : int {
   kModeGateUp = 0,   // fwd  G/U = X W_{g,u}^T (+ LoRA), SwiGLU epilogue      A: K-major decode of W_g/W_u rows
   kModeDown = 1,     // fwd  y = h W_d^T (+ LoRA), route-weight epilogue       A: K-major decode of W_d rows
@@ -125,7 +127,7 @@ struct GemmParams {
   // frozen base scales of projection 0 and 1 (bf16)
   const uint16_t* s0;
   const uint16_t* s1;
-  const uint8_t* e0;         // MXFP4 base (gemm_tm.cu): UE8M0 scale bytes of projection 0 and 1
+  const uint8_t* e0;         // MXFP4 base: UE8M0 scale bytes of projection 0 and 1
   const uint8_t* e1;
   int64_t s_expert;          // scale elements per expert
   int s_row;                 // scales per stored row

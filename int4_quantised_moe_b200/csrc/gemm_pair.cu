@@ -1,9 +1,10 @@
 // Dequant-fused grouped GEMMs of the routed RAWINT4 MoE-LoRA layer on
 // sm_100a tensor cores: CTA pairs (tcgen05 cta_group::2), TMEM accumulators,
-// TMA-fed operands.
+// TMA-fed operands. The library runs the transpose-free backward modes here,
+// for a RAWINT4 or an MXFP4 base.
 //
 // Clusters of two CTAs on an SM pair walk (token tile, feature block) work
-// items. A token tile is up to 256 permuted rows of one expert; a feature
+// items. A token tile is up to kTileRows permuted rows of one expert; a feature
 // block is 256 weight rows (gate/up: the same 128 features of gate and up),
 // 128 of them decoded in each CTA. The pair-wide MMA (M = 256) reads both
 // CTAs' A tiles and both halves of the token tile (each CTA loads its half),
