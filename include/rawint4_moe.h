@@ -267,6 +267,31 @@ RAWINT4_API int rawint4_moe_permute_static(const int64_t* ids, int32_t qlen, int
                                            int32_t* offsets, int32_t* perm, int32_t* inv, void* stream);
 RAWINT4_API size_t rawint4_moe_permute_static_max_bytes(void);
 
+/* Row moves of expert parallelism (no counterpart in the method, which runs
+ * one process per layer: the layer's experts are split over G processes,
+ * each routed slot travels to the process that owns its expert and its
+ * result travels back). With
+ * rawint4_moe_permute run on the owning process index of every slot
+ * (experts = G), the slots are grouped by destination:
+ *   rawint4_moe_dispatch_rows  dst[p, :] = src[perm[p] / top_k, :] for
+ *     p < n: the bf16 token rows of the n slots that leave, in permuted
+ *     order (src [Q, width], dst [n, width], width % 8 == 0, every perm[p]
+ *     for p < n a valid slot; device pointers).
+ *   rawint4_moe_combine_slots  out[t, :] = bf16 of the fp32 sum, in slot
+ *     order s = 0..top_k-1, of src[inv[t * top_k + s], :] over the slots
+ *     with inv >= 0 (0 where none): the token rows from the per-slot result
+ *     rows that came back (src [n, width] bf16, out [qlen, width] bf16).
+ *   rawint4_moe_gather_slots   out[f] = inv[f] >= 0 ? src[inv[f]] : 0 for
+ *     f < n_slots: per-slot fp32 values (dRoute) back in slot order.
+ * INVALID_ARGUMENT for a null pointer with a positive size, a negative size
+ * or width % 8 != 0; asynchronous on `stream`. */
+RAWINT4_API int rawint4_moe_dispatch_rows(const uint16_t* src, const int32_t* perm, int32_t n, int32_t top_k,
+                                          int32_t width, uint16_t* dst, void* stream);
+RAWINT4_API int rawint4_moe_combine_slots(const uint16_t* src, const int32_t* inv, int32_t qlen, int32_t top_k,
+                                          int32_t width, uint16_t* out, void* stream);
+RAWINT4_API int rawint4_moe_gather_slots(const float* src, const int32_t* inv, int32_t n_slots, float* out,
+                                         void* stream);
+
 /* Timing hook for measurement (no counterpart in the method): while enabled,
  * every kernel launch of the library records a CUDA event pair on the
  * launch's stream (at most max_launches launches). profile_end synchronises

@@ -51,6 +51,9 @@ EXPORTED_SYMBOLS = (
     "rawint4_moe_router_topk",
     "rawint4_moe_router_bwd",
     "rawint4_mxfp4_decode",
+    "rawint4_moe_dispatch_rows",
+    "rawint4_moe_combine_slots",
+    "rawint4_moe_gather_slots",
 )
 
 
@@ -107,6 +110,9 @@ def _load() -> ctypes.CDLL:
     lib.rawint4_moe_router_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
     lib.rawint4_moe_router_bwd.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.rawint4_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+    lib.rawint4_moe_dispatch_rows.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.rawint4_moe_combine_slots.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.rawint4_moe_gather_slots.argtypes = [vp, vp, i32, vp, vp]
     for name in EXPORTED_SYMBOLS:
         if name != "rawint4_moe_lora_strerror":
             getattr(lib, name).restype = ctypes.c_int  # raises AttributeError if the library lacks it
@@ -241,10 +247,54 @@ def rawint4_moe_permute_static_max_bytes() -> int:
     return int(_lib.rawint4_moe_permute_static_max_bytes())
 
 
+def rawint4_moe_dispatch_rows(src: torch.Tensor, perm: torch.Tensor, n: int, top_k: int, dst: torch.Tensor,
+                              stream=None) -> None:
+    """dst[p] = src[perm[p] // top_k] for p < n (bf16 rows)."""
+    _require(src, torch.bfloat16, src.device, "src")
+    _require(dst, torch.bfloat16, src.device, "dst")
+    _require(perm, torch.int32, src.device, "perm")
+    if dst.shape[0] < n or dst.shape[1] != src.shape[1] or perm.numel() < n:
+        raise ValueError("dispatch_rows: dst must hold n rows of src's width and perm n entries")
+    _check(_lib.rawint4_moe_dispatch_rows(_ptr(src), _ptr(perm), int(n), int(top_k), src.shape[1], _ptr(dst),
+                                          _stream(stream)), "rawint4_moe_dispatch_rows")
+
+
+def rawint4_moe_combine_slots(src: torch.Tensor, inv: torch.Tensor, qlen: int, top_k: int, out: torch.Tensor,
+                              stream=None) -> None:
+    """out[t] = bf16(sum over s of src[inv[t * top_k + s]]) in slot order (fp32 sums)."""
+    _require(out, torch.bfloat16, out.device, "out")
+    _require(inv, torch.int32, out.device, "inv")
+    if src.numel():
+        _require(src, torch.bfloat16, out.device, "src")
+        if src.shape[1] != out.shape[1]:
+            raise ValueError("combine_slots: src and out widths differ")
+    if out.shape[0] < qlen or inv.numel() < qlen * top_k:
+        raise ValueError("combine_slots: out needs qlen rows and inv qlen * top_k entries")
+    _check(_lib.rawint4_moe_combine_slots(_ptr(src) if src.numel() else None, _ptr(inv), int(qlen), int(top_k),
+                                          out.shape[1], _ptr(out), _stream(stream)), "rawint4_moe_combine_slots")
+
+
+def rawint4_moe_gather_slots(src: torch.Tensor, inv: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """out[f] = src[inv[f]] where inv[f] >= 0, else 0 (fp32)."""
+    _require(out, torch.float32, out.device, "out")
+    _require(inv, torch.int32, out.device, "inv")
+    if src.numel():
+        _require(src, torch.float32, out.device, "src")
+    if inv.numel() < out.numel():
+        raise ValueError("gather_slots: inv needs one entry per output")
+    _check(_lib.rawint4_moe_gather_slots(_ptr(src) if src.numel() else None, _ptr(inv), out.numel(), _ptr(out),
+                                         _stream(stream)), "rawint4_moe_gather_slots")
+
+
 # ---------------------------------------------------------------------------
 # Convenience holder used by tests and the bench: keeps the layer's tensors
 # and one workspace together and calls the two entry points.
 # ---------------------------------------------------------------------------
+
+def _require(t, dtype: torch.dtype, device: torch.device, name: str) -> None:
+    """Like _expect, without a fixed shape."""
+    _expect(t, name, dtype, tuple(t.shape) if isinstance(t, torch.Tensor) else (), device)
+
 
 def _expect(t, name: str, dtype: torch.dtype, shape: tuple, device: Optional[torch.device] = None) -> None:
     """Host-side argument check: the C ABI sees raw pointers only, so a wrong

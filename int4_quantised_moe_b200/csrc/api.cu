@@ -875,4 +875,41 @@ int rawint4_moe_permute(const int64_t* ids, int32_t qlen, int32_t top_k, int32_t
   return RAWINT4_OK;
 }
 
+int rawint4_moe_dispatch_rows(const uint16_t* src, const int32_t* perm, int32_t n, int32_t top_k, int32_t width,
+                              uint16_t* dst, void* stream) {
+  if (n < 0 || top_k < 1 || width < 8 || width % 8 != 0 || (n > 0 && (!src || !perm || !dst)))
+    return RAWINT4_INVALID_ARGUMENT;
+  if (n == 0) return RAWINT4_OK;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  return launch_dispatch_rows(src, perm, n, top_k, width, dst, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? RAWINT4_OK
+             : RAWINT4_CUDA_ERROR;
+}
+
+int rawint4_moe_combine_slots(const uint16_t* src, const int32_t* inv, int32_t qlen, int32_t top_k, int32_t width,
+                              uint16_t* out, void* stream) {
+  if (qlen < 0 || top_k < 1 || width < 8 || width % 8 != 0 || (qlen > 0 && (!inv || !out)))
+    return RAWINT4_INVALID_ARGUMENT;
+  if (qlen == 0) return RAWINT4_OK;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  return launch_combine_slots(src, inv, qlen, top_k, width, out, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? RAWINT4_OK
+             : RAWINT4_CUDA_ERROR;
+}
+
+int rawint4_moe_gather_slots(const float* src, const int32_t* inv, int32_t n_slots, float* out, void* stream) {
+  if (n_slots < 0 || (n_slots > 0 && (!inv || !out))) return RAWINT4_INVALID_ARGUMENT;
+  if (n_slots == 0) return RAWINT4_OK;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc != RAWINT4_OK) return rc;
+  return launch_gather_slots(src, inv, n_slots, out, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? RAWINT4_OK
+             : RAWINT4_CUDA_ERROR;
+}
+
 }  // extern "C"

@@ -207,6 +207,61 @@ __global__ void decode_mxfp4_kernel(const uint8_t* __restrict__ q, const uint8_t
   }
 }
 
+// ---------------------------------------------- expert-parallel row moves
+// dst[p, :] = src[perm[p] / top_k, :] for p < n (bf16 rows of `vecs` 16-byte
+// vectors; every perm[p] in the range is a valid slot).
+__global__ void __launch_bounds__(256) dispatch_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
+                                                            int32_t n, int top_k, int vecs, uint4* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t p = warp0; p < n; p += nwarps) {
+    const uint4* s = src + (int64_t)(perm[p] / top_k) * vecs;
+    uint4* d = dst + p * vecs;
+#pragma unroll 4
+    for (int c = lane; c < vecs; c += 32) d[c] = __ldg(s + c);
+  }
+}
+
+// out[t, :] = bf16(sum over s of src[inv[t * top_k + s], :]) in slot order,
+// fp32 sums, slots with inv < 0 skipped (8 bf16 per thread and step).
+__global__ void combine_slots_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ inv, int32_t qlen,
+                                     int top_k, int vecs, uint4* __restrict__ out) {
+  const int64_t total = (int64_t)qlen * vecs;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = idx / vecs;
+    const int c = (int)(idx - t * vecs);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < top_k; ++s) {
+      const int32_t p = inv[t * top_k + s];
+      if (p >= 0) {
+        const uint4 v = __ldg(src + (int64_t)p * vecs + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * j] += __uint_as_float(w[j] << 16);
+          acc[2 * j + 1] += __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = (uint32_t)bf16_bits_rn(acc[2 * j]) | ((uint32_t)bf16_bits_rn(acc[2 * j + 1]) << 16);
+    out[idx] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// out[f] = inv[f] >= 0 ? src[inv[f]] : 0 for f < n_slots.
+__global__ void gather_slots_kernel(const float* __restrict__ src, const int32_t* __restrict__ inv, int32_t n_slots,
+                                    float* __restrict__ out) {
+  for (int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f < n_slots; f += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t p = inv[f];
+    out[f] = p >= 0 ? src[p] : 0.f;
+  }
+}
+
 int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
   if (g > 148 * 16) g = 148 * 16;
@@ -246,6 +301,28 @@ cudaError_t launch_combine_route(const float* part, int nparts, const int32_t* i
                                  float* grad_route, int max_tokens, cudaStream_t stream) {
   combine_route_kernel<<<grid_for((int64_t)max_tokens * top_k, 256), 256, 0, stream>>>(part, nparts, inv, top_k, hdr,
                                                                                        grad_route);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_rows(const uint16_t* src, const int32_t* perm, int32_t n, int top_k, int width,
+                                 uint16_t* dst, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  dispatch_rows_kernel<<<grid_for((int64_t)n * 32, 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src), perm, n, top_k, width / 8, reinterpret_cast<uint4*>(dst));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_slots(const uint16_t* src, const int32_t* inv, int32_t qlen, int top_k, int width,
+                                 uint16_t* out, cudaStream_t stream) {
+  if (qlen <= 0) return cudaSuccess;
+  combine_slots_kernel<<<grid_for((int64_t)qlen * (width / 8), 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src), inv, qlen, top_k, width / 8, reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_slots(const float* src, const int32_t* inv, int32_t n_slots, float* out, cudaStream_t stream) {
+  if (n_slots <= 0) return cudaSuccess;
+  gather_slots_kernel<<<grid_for(n_slots, 256), 256, 0, stream>>>(src, inv, n_slots, out);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,13 @@ cudaError_t launch_combine_rows(const float* src, const int32_t* inv, int top_k,
                                 cudaStream_t stream);
 
 // grad_route[t, s] = 2^-hdr->dy_exp sum_b part[inv[f], b] (0 for dropped slots), f = t*k+s < hdr->qlen*k.
+// Expert-parallel row moves (see the C-ABI declarations).
+cudaError_t launch_dispatch_rows(const uint16_t* src, const int32_t* perm, int32_t n, int top_k, int width,
+                                 uint16_t* dst, cudaStream_t stream);
+cudaError_t launch_combine_slots(const uint16_t* src, const int32_t* inv, int32_t qlen, int top_k, int width,
+                                 uint16_t* out, cudaStream_t stream);
+cudaError_t launch_gather_slots(const float* src, const int32_t* inv, int32_t n_slots, float* out, cudaStream_t stream);
+
 cudaError_t launch_combine_route(const float* part, int nparts, const int32_t* inv, int top_k, const WsHeader* hdr,
                                  float* grad_route, int max_tokens, cudaStream_t stream);
 
