@@ -510,6 +510,31 @@ def test_large_rank_parity(rank, fmt, limit):
 
 
 @pytest.mark.parametrize("tiles", ["narrow", "wide"])
+@pytest.mark.parametrize("shape", [("h64_i64", 4, 2, 64, 64, 8, 9, "rawint4"), ("h128_i64", 4, 2, 128, 64, 8, 9, "rawint4"),
+                                   ("one_expert_top1", 1, 1, 256, 128, 16, 7, "rawint4"),
+                                   ("h64_i192_top3", 3, 3, 64, 192, 4, 11, "rawint4"),
+                                   ("mxfp4_h128_i128", 4, 2, 128, 128, 8, 9, "mxfp4")], ids=lambda c: c[0])
+def test_smallest_shapes(shape, tiles, monkeypatch):
+    """The smallest layers the boundary accepts (H and I of one 64-wide stage,
+    a single expert with top_k = 1, I = 192 = three stages with top_k = 3,
+    the smallest MXFP4 layer), in both tile configurations."""
+    name, E, k, H, I, r, Q, fmt = shape
+    monkeypatch.setenv("RAWINT4_TILES", tiles)
+    wl = make_workload(small_config(name, E, k, H, I, r, Q, weight_format=fmt), seed=11)
+    out_r, gin_r, groute_r, grads_r = oracle(wl)
+    g = on_gpu(wl)
+    layer = make_layer(g)
+    grads = grad_buffers(g)
+    out, gin, groute = run_fwd_bwd(layer, g, grads)
+    assert layer.status() == 0
+    close("out", out, out_r, TOL_OUT)
+    close("grad_in", gin, gin_r, TOL_DX)
+    close("grad_route", groute, groute_r, TOL_ROUTE)
+    for n in LORA_NAMES:
+        close(n, grads[n], grads_r[n], TOL_LORA)
+
+
+@pytest.mark.parametrize("tiles", ["narrow", "wide"])
 @pytest.mark.parametrize("case", ["config1", "gemma4_clamp", "rank64", "rank12", "mxfp4"])
 def test_tile_configurations(case, tiles, monkeypatch):
     """Both token-tile configurations of the GEMMs on the same inputs: narrow
