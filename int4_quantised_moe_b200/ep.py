@@ -70,7 +70,10 @@ def _exchange(dist, tensor: torch.Tensor, send_counts, recv_counts) -> torch.Ten
     rows each); bf16 rows (an even width) travel as int32 pairs of bit
     patterns, which every backend carries."""
     bf16 = tensor.dtype == torch.bfloat16
-    src = tensor.contiguous().view(torch.int32) if bf16 else tensor.contiguous()
+    src = tensor.contiguous()
+    if bf16:
+        src = (src.view(torch.int32) if src.numel() else
+               torch.empty(tuple(src.shape[:-1]) + (src.shape[-1] // 2,), dtype=torch.int32, device=src.device))
     out = torch.empty((int(sum(recv_counts)),) + tuple(src.shape[1:]), dtype=src.dtype, device=tensor.device)
     dist.all_to_all_single(out, src, output_split_sizes=list(recv_counts), input_split_sizes=list(send_counts))
     return out.view(torch.bfloat16) if bf16 else out

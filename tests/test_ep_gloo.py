@@ -159,6 +159,65 @@ def test_expert_parallel_matches_whole_layer(tmp_path):
             assert torch.isfinite(p["grads"][n]).all()
 
 
+def _edge_worker(rank: int, world: int, port: int, out_dir: str) -> None:
+    """Rank 1 has no tokens; rank 0's tokens include slots with an expert id
+    outside [0, E) (dropped) and every slot of rank 0 goes to rank 1's
+    experts or nowhere, so rank 0 receives nothing and rank 1 sends nothing."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg = CONFIGS[1]
+        wl = make_workload(cfg, device="cpu")
+        per = cfg.experts // world
+        local = _OracleLocalLayer(wl, rank * per, (rank + 1) * per)
+        ops = ep.KernelOps(permute=_permute, dispatch_rows=_dispatch_rows, combine_slots=_combine_slots,
+                           gather_slots=_gather_slots)
+        layer = ep.ExpertParallelLayer(dist, cfg.experts, cfg.top_k, local, capacity=cfg.qlen * cfg.top_k, ops=ops)
+        q = 16 if rank == 0 else 0
+        ids = torch.remainder(wl.expert_ids[:q], per) + per  # rank 1's experts
+        if q:
+            ids[::3, 1] = -1
+            ids[1::5, 0] = cfg.experts + 2
+        w = wl.route_weights[:q].contiguous()
+        x = wl.x[:q].contiguous()
+        out = layer.forward(ids.contiguous(), w, x)
+        grads = {n: torch.full(wl.lora[n][rank * per:(rank + 1) * per].shape, float("nan"), dtype=torch.bfloat16)
+                 for n in LORA_NAMES}
+        groute = torch.full(ids.shape, float("nan"), dtype=torch.float32)
+        gin = layer.backward(wl.grad_out[:q].contiguous(), grads, grad_route=groute)
+        torch.save({"out": out, "gin": gin, "groute": groute, "grads": grads, "ids": ids},
+                   os.path.join(out_dir, f"edge_rank{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_empty_and_dropped_slots(tmp_path):
+    mp.spawn(_edge_worker, args=(WORLD, _free_port(), str(tmp_path)), nprocs=WORLD, join=True)
+    p0, p1 = (torch.load(os.path.join(tmp_path, f"edge_rank{r}.pt")) for r in range(WORLD))
+    cfg = CONFIGS[1]
+    wl = make_workload(cfg, device="cpu")
+    ids = p0["ids"].numpy()
+    valid = np.where((ids >= 0) & (ids < cfg.experts), ids, -1)
+    layer = oracle_layer(wl)
+    o_out, ctx = omoe.forward(layer, f64(wl.x[:16]), valid, f64(wl.route_weights[:16]))
+    o_gin, o_groute, o_grads = omoe.backward(layer, ctx, f64(wl.grad_out[:16]))
+    for name, got, ref, tol in (("out", p0["out"], o_out, 5e-3), ("grad_in", p0["gin"], o_gin, 5e-3)):
+        rel, _ = metrics.relative_l2_and_cosine(got.double().numpy(), ref)
+        assert rel <= tol, f"{name}: rel-L2 {rel:.3e}"
+    # dropped slots: no route gradient; the others match
+    dropped = valid < 0
+    assert torch.all(p0["groute"][torch.from_numpy(dropped)] == 0)
+    np.testing.assert_allclose(p0["groute"].double().numpy()[~dropped], o_groute[~dropped], rtol=1e-5, atol=1e-7)
+    # rank 0 received nothing: its experts' gradients are zero; rank 1 had no tokens
+    per = cfg.experts // WORLD
+    for n in LORA_NAMES:
+        assert torch.count_nonzero(p0["grads"][n]) == 0
+        rel, _ = metrics.relative_l2_and_cosine(p1["grads"][n].double().numpy(), o_grads[n][per:])
+        assert rel <= 1e-2, f"{n}: rel-L2 {rel:.3e}"
+    assert p1["out"].shape == (0, cfg.hidden) and p1["gin"].shape == (0, cfg.hidden)
+
+
 def test_owner_of_slots():
     ids = torch.tensor([[0, 3], [4, 7], [-1, 8]], dtype=torch.int64)
     assert ep.owner_of(ids, 4).tolist() == [[0, 0], [1, 1], [-1, 2]]
